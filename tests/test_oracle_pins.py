@@ -1,0 +1,361 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each test checks the oracle against a value the OCP MX definition fixes (golden
+fixtures worked by hand), a closed form, brute force on tiny inputs, an
+independent library computation (torch float64, scipy), or an invariance of
+the layer. A wrong table entry, nibble order, sign, tie-break, index or
+transposed operand in the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+from mxfp4_routed_expert_04_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------------------
+# number formats
+# ---------------------------------------------------------------------------
+
+def test_e2m1_table_matches_ocp_fixture():
+    for ln in _lines("e2m1_codes.txt"):
+        code, val = ln.split()
+        got = O.e2m1_decode(np.uint8(int(code, 16)))
+        assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val)), ln
+
+
+def test_e2m1_table_matches_bitfield_definition():
+    # closed form of a 1-2-1 minifloat with exponent bias 1 (subnormal at field 0)
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        mag = (m * 0.5) if e == 0 else (2.0 ** (e - 1)) * (1 + m / 2)
+        assert O.e2m1_decode(np.uint8(c)) == (-mag if s else mag)
+
+
+def test_e8m0_fixture_and_closed_form():
+    for ln in _lines("e8m0_codes.txt"):
+        code, val = ln.split()
+        got = float(O.e8m0_decode(np.int64(int(code))))
+        if val == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(val)
+    c = np.arange(255)
+    assert np.array_equal(O.e8m0_decode(c), np.array([math.ldexp(1.0, int(i) - 127) for i in c]))
+
+
+def test_mxfp4_hand_worked_row():
+    lines = _lines("mxfp4_row.txt")
+    q = np.array([int(b, 16) for b in lines[0].split()[1:]], dtype=np.uint8)[None]
+    s = np.array([int(v) for v in lines[1].split()[1:]], dtype=np.uint8)[None]
+    vals = O.mxfp4_dequant(q, s)[0]
+    expect = np.zeros(64)
+    for ln in lines[2:]:
+        _, i, v = ln.split()
+        expect[int(i)] = float(v)
+    assert np.array_equal(vals, expect)
+    assert math.copysign(1, vals[2]) == -1.0     # code 8 is negative zero
+
+
+def test_mxfp4_nan_scale_poisons_its_block_only():
+    q = np.full((1, 32), 0x22, np.uint8)
+    s = np.array([[255, 127]], np.uint8)
+    v = O.mxfp4_dequant(q, s)[0]
+    assert np.all(np.isnan(v[:32])) and np.all(v[32:] == 1.0)
+
+
+def test_mxfp4_dequant_against_torch_table():
+    # an independent decode: torch float64, nibbles unpacked by integer division
+    rng = np.random.default_rng(5)
+    q = rng.integers(0, 256, (7, 64), dtype=np.uint8)
+    s = rng.integers(100, 140, (7, 4), dtype=np.uint8)
+    tq = torch.from_numpy(q.astype(np.int64))
+    codes = torch.stack([tq % 16, tq // 16], dim=-1).reshape(7, 128)
+    table = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6] * 2, dtype=torch.float64)
+    sign = torch.where(codes >= 8, -1.0, 1.0).double()
+    vals = sign * table[codes]
+    scale = torch.pow(2.0, torch.from_numpy(s.astype(np.float64)) - 127).repeat_interleave(32, 1)
+    assert np.array_equal(O.mxfp4_dequant(q, s), (vals * scale).numpy())
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    f32 = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(1e3),
+        rng.standard_normal(2000).astype(np.float32) * np.float32(1e-39),   # subnormal range
+        np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 3.39e38, 3.4e38, 0.0, -0.0],
+                 np.float32),
+    ])
+    # float32 inputs are exact in float64, so torch's float32 -> bf16 conversion is a
+    # single rounding of the same value
+    want = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.round_to_bf16_bits(f32.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def test_bf16_rounding_of_float64_ties_is_single_rounding():
+    # 1 + 2^-8 + 2^-40 is above the tie: rounds up; a float32 detour would round to the
+    # tie first and then to even (down)
+    v = np.array([1 + 2 ** -8 + 2 ** -40, 1 + 2 ** -8 - 2 ** -40])
+    assert list(O.round_to_bf16_bits(v)) == [0x3F81, 0x3F80]
+
+
+# ---------------------------------------------------------------------------
+# quantiser
+# ---------------------------------------------------------------------------
+
+def test_quantize_hand_worked_blocks():
+    for ln in _lines("mxfp4_quantize_blocks.txt"):
+        _, rest = ln.split(" ", 1)
+        name, vals, scale, codes = [p.strip() for p in rest.split("|")]
+        vals = [float(v) for v in vals.split()]
+        block = np.zeros(32)
+        block[:len(vals)] = vals
+        c, s = O.mxfp4_quantize(block[None])
+        assert int(s[0, 0]) == int(scale), name
+        assert [int(v) for v in c[0, :len(vals)]] == [int(v) for v in codes.split()], name
+        assert np.all(c[0, len(vals):] == 0), name
+
+
+def test_quantize_roundtrips_every_representable_value():
+    # any block whose values are already E2M1 x 2^X with amax in [4, 8) * 2^X
+    # quantises to itself
+    for X in (-20, -3, 0, 5, 40):
+        mags = np.array(list(O.E2M1_MAGNITUDES) * 4)
+        vals = np.where(np.arange(32) % 3 == 0, -1, 1) * mags * 2.0 ** X
+        vals[0] = 6.0 * 2.0 ** X
+        c, s = O.mxfp4_quantize(vals[None])
+        assert int(s[0, 0]) == 127 + X
+        assert np.array_equal(O.mxfp4_values(c, s)[0], vals)
+
+
+def test_quantize_error_bound():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((50, 128)) * 10 ** rng.uniform(-3, 3, (50, 1))
+    c, s = O.mxfp4_quantize(v)
+    d = O.mxfp4_values(c, s)
+    scale = np.repeat(O.e8m0_decode(s), 32, axis=-1)
+    # between representable neighbours the error is at most half the local spacing,
+    # which is at most 1 (between 4 and 6) in units of the scale, and values above
+    # 6 * scale saturate to 6 * scale
+    err = np.abs(v - d) / scale
+    assert np.all((err <= 1.0 + 1e-12) | (np.abs(v) > 6 * scale))
+    assert np.all(np.abs(v) / scale < 8)      # amax / 2^X < 8 by the choice of X
+
+
+def test_quantize_zero_block():
+    c, s = O.mxfp4_quantize(np.zeros((1, 32)))
+    assert s[0, 0] == 0 and np.all(c == 0)
+
+
+def test_pack_is_low_nibble_first():
+    codes = np.tile(np.arange(16, dtype=np.uint8), 2)[None]
+    packed = O.mxfp4_pack(codes)
+    assert packed[0, 0] == 0x10 and packed[0, 1] == 0x32
+
+
+# ---------------------------------------------------------------------------
+# routing
+# ---------------------------------------------------------------------------
+
+def _brute_topk(row, k):
+    order = sorted(range(len(row)), key=lambda e: (-row[e], e))
+    return order[:k]
+
+
+def test_topk_brute_force_with_exact_ties():
+    rng = np.random.default_rng(7)
+    logits = np.round(rng.standard_normal((40, 12)) * 2) / 2     # many exact ties
+    for k in (1, 2, 3, 12):
+        idx, w, flagged = O.topk_route(logits, k)
+        for t in range(40):
+            assert list(idx[t]) == _brute_topk(list(logits[t]), k)
+
+
+def test_topk_weights_equal_renormalised_full_softmax():
+    rng = np.random.default_rng(8)
+    logits = rng.standard_normal((30, 64)) * 1.8
+    idx, w, _ = O.topk_route(logits, 10)
+    p = scipy.special.softmax(logits, axis=1)
+    sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w, sel / sel.sum(axis=1, keepdims=True), rtol=1e-13)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-13)
+    assert np.all(np.diff(w, axis=1) <= 0)      # slots in descending weight
+
+
+def test_topk_near_tie_flag():
+    logits = np.array([[3.0, 2.0, 1.0, 1.0 - 5e-6, 0.0],
+                       [3.0, 2.0, 1.0, 0.5, 0.0],
+                       [3.0, 3.0 - 1e-6, 1.0, 0.5, 0.0]])
+    _, _, flagged = O.topk_route(logits, 3)
+    assert list(flagged) == [True, False, True]
+
+
+def test_router_logits_against_torch():
+    w = synth.WORKLOADS["tiny"]
+    d = synth.dense_inputs(w)
+    x = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).double()
+    wr = torch.from_numpy(d["w_router"].view(np.int16)).view(torch.bfloat16).double()
+    np.testing.assert_allclose(O.router_logits(d["x"], d["w_router"]), (x @ wr.T).numpy(),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_permute_brute_force():
+    rng = np.random.default_rng(9)
+    for T, E, k in ((1, 4, 2), (5, 6, 3), (17, 9, 4), (8, 3, 3)):
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+        counts, offsets, row_token, row_slot, slot_row = O.permute(idx, E)
+        rows = []
+        for e in range(E):
+            for t in range(T):
+                for j in range(k):
+                    if idx[t, j] == e:
+                        rows.append((t, j))
+        assert [(int(a), int(b)) for a, b in zip(row_token, row_slot)] == rows
+        assert list(counts) == [sum(1 for t in range(T) for j in range(k) if idx[t, j] == e)
+                                for e in range(E)]
+        assert offsets[0] == 0 and offsets[-1] == T * k and np.all(np.diff(offsets) == counts)
+        for r, (t, j) in enumerate(rows):
+            assert slot_row[t, j] == r
+
+
+# ---------------------------------------------------------------------------
+# expert FFN, shared expert, combine, whole layer
+# ---------------------------------------------------------------------------
+
+def _torch_dense_swiglu(x, wg, wu, wd):
+    x, wg, wu, wd = (torch.from_numpy(np.asarray(a, np.float64)) for a in (x, wg, wu, wd))
+    return (torch.nn.functional.silu(x @ wg.T) * (x @ wu.T)) @ wd.T
+
+
+def _torch_decode(q, s):
+    tq = torch.from_numpy(np.asarray(q).astype(np.int64))
+    n = tq.shape[-1] * 2
+    codes = torch.stack([tq % 16, tq // 16], dim=-1).reshape(*tq.shape[:-1], n)
+    table = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6] * 2, dtype=torch.float64)
+    vals = torch.where(codes >= 8, -1.0, 1.0).double() * table[codes]
+    return vals * torch.pow(2.0, torch.from_numpy(np.asarray(s).astype(np.float64)) - 127) \
+        .repeat_interleave(32, -1)
+
+
+def _tiny_layer_inputs(E=1, k=1, T=5, H=64, I=96, seed=11):
+    w = synth.MoeWorkload("t", T=T, H=H, I=I, E=E, k=k, I_shared=32, seed=seed)
+    d = synth.dense_inputs(w)
+    ex = synth.expert_weights(w, range(E))
+    get = lambda e: tuple(ex[n][e] for n in ("wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s"))
+    return w, d, ex, get
+
+
+def test_single_expert_top1_equals_dense_swiglu_in_torch():
+    w, d, ex, get = _tiny_layer_inputs(E=1, k=1)
+    out = O.moe_layer(d, 1, get)
+    x = O.bf16_to_f64(d["x"])
+    wg = _torch_decode(ex["wg_q"][0], ex["wg_s"][0]).numpy()
+    wu = _torch_decode(ex["wu_q"][0], ex["wu_s"][0]).numpy()
+    wd = _torch_decode(ex["wd_q"][0], ex["wd_s"][0]).numpy()
+    routed = _torch_dense_swiglu(x, wg, wu, wd).numpy()
+    assert np.all(out["w"] == 1.0)
+    xs = torch.from_numpy(x)
+    bf = lambda a: torch.from_numpy(O.bf16_to_f64(d[a]))
+    shared = torch.sigmoid(xs @ bf("w_sgate"))[:, None] * _torch_dense_swiglu(
+        x, bf("ws_gate").numpy(), bf("ws_up").numpy(), bf("ws_down").numpy())
+    np.testing.assert_allclose(out["y"], routed + shared.numpy(), rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(out["shared"], shared.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_zero_gate_vector_gives_half_gate():
+    w, d, ex, get = _tiny_layer_inputs(E=2, k=1)
+    d = dict(d, w_sgate=np.zeros_like(d["w_sgate"]))
+    _, gate = O.shared_expert(d["x"], d["ws_gate"], d["ws_up"], d["ws_down"], d["w_sgate"])
+    assert np.all(gate == 0.5)
+
+
+def test_dense_masked_equivalence():
+    # sum over ALL experts of mask * weight * FFN_e equals the routed layer
+    w, d, ex, get = _tiny_layer_inputs(E=6, k=3, T=7)
+    out = O.moe_layer(d, 3, get)
+    x = O.bf16_to_f64(d["x"])
+    y = out["shared"].copy()
+    for e in range(6):
+        wg = _torch_decode(ex["wg_q"][e], ex["wg_s"][e]).numpy()
+        wu = _torch_decode(ex["wu_q"][e], ex["wu_s"][e]).numpy()
+        wd = _torch_decode(ex["wd_q"][e], ex["wd_s"][e]).numpy()
+        ffn = _torch_dense_swiglu(x, wg, wu, wd).numpy()
+        mask = np.zeros(7)
+        for t in range(7):
+            for j in range(3):
+                if out["idx"][t, j] == e:
+                    mask[t] = out["w"][t, j]
+        y += mask[:, None] * ffn
+    scale = np.sqrt(np.mean(y ** 2))
+    np.testing.assert_allclose(out["y"], y, rtol=0, atol=1e-11 * scale)
+
+
+def test_expert_relabelling_invariance():
+    w, d, ex, get = _tiny_layer_inputs(E=8, k=3, T=6)
+    base = O.moe_layer(d, 3, get)
+    perm = np.random.default_rng(2).permutation(8)        # new id of old expert e is perm[e]
+    inv = np.argsort(perm)
+    d2 = dict(d, w_router=d["w_router"][inv])
+    get2 = lambda e: get(int(inv[e]))
+    out = O.moe_layer(d2, 3, get2)
+    assert np.array_equal(out["idx"], perm[base["idx"]])
+    np.testing.assert_array_equal(out["y"], base["y"])
+
+
+def test_batch_invariance():
+    w, d, ex, get = _tiny_layer_inputs(E=5, k=2, T=6)
+    full = O.moe_layer(d, 2, get)
+    for t in range(6):
+        one = O.moe_layer(dict(d, x=d["x"][t:t + 1]), 2, get)
+        # equal up to float64 reassociation inside the BLAS matmul
+        np.testing.assert_allclose(one["y"][0], full["y"][t], rtol=1e-12,
+                                   atol=1e-12 * np.abs(full["y"]).max())
+        np.testing.assert_array_equal(one["idx"][0], full["idx"][t])
+
+
+def test_latent_identity_reduces_to_plain_layer():
+    # with L = H and identity projections the latent layer is the plain layer
+    w, d, ex, get = _tiny_layer_inputs(E=4, k=2, T=3, H=64)
+    eye = synth.f32_to_bf16_bits(np.eye(64, dtype=np.float32))
+    plain = O.moe_layer(d, 2, get)
+    lat = O.moe_layer(dict(d, w_lat_down=eye, w_lat_up=eye), 2, get)
+    np.testing.assert_array_equal(lat["x_lat"], d["x"])
+    np.testing.assert_allclose(lat["y"], plain["y"], rtol=1e-13, atol=0)
+
+
+def test_mxfp4_activation_mode_quantises_both_operands():
+    # with act="mxfp4" the layer equals the exact layer run on pre-quantised x,
+    # with h quantised before the down projection
+    w, d, ex, get = _tiny_layer_inputs(E=1, k=1, T=3)
+    wg = O.mxfp4_dequant(ex["wg_q"][0], ex["wg_s"][0])
+    wu = O.mxfp4_dequant(ex["wu_q"][0], ex["wu_s"][0])
+    wd = O.mxfp4_dequant(ex["wd_q"][0], ex["wd_s"][0])
+    x = O.bf16_to_f64(d["x"])
+    y, h = O.expert_ffn(x, wg, wu, wd, act="mxfp4")
+    xq = O.mxfp4_values(*O.mxfp4_quantize(x))
+    h_ref = O.silu(xq @ wg.T) * (xq @ wu.T)
+    hq = O.mxfp4_values(*O.mxfp4_quantize(h_ref))
+    np.testing.assert_array_equal(h, hq)
+    np.testing.assert_allclose(y, hq @ wd.T, rtol=1e-14)
+    assert not np.array_equal(xq, x)
+
+
+def test_silu_sigmoid_match_torch_including_extremes():
+    z = np.concatenate([np.linspace(-50, 50, 1001), [-800.0, 800.0, 0.0]])
+    np.testing.assert_allclose(O.silu(z), torch.nn.functional.silu(torch.from_numpy(z)).numpy(),
+                               rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(O.sigmoid(z), torch.sigmoid(torch.from_numpy(z)).numpy(),
+                               rtol=1e-14, atol=1e-300)
