@@ -1,0 +1,395 @@
+"""Benchmark of the routed MXFP4 MoE layer on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the whole layer (route, permute, routed experts, gated
+shared expert, combine) over one batch of synthetic input, weights resident in
+HBM. Each timed step is a CUDA-graph replay of moe_layer, bracketed by CUDA
+events on the launching stream; L2 is flushed (512 MiB write) before every
+step, outside the events. With N > 1 (torchrun) every rank runs an independent
+replica of the layer (the layer does not shard: no collective on the data
+path); timing is the max over ranks and ``value`` counts the tokens of all
+ranks ("scaling": "weak").
+
+Extra keys: ``roofline`` for the routed-expert call (moe_expert_ffn: the
+gate/up and down grouped GEMVs), timed alone in its own loop with the same
+flushing; ``cpu_baseline`` (the fp64 oracle on the host cores, rank 0 only);
+``e2e`` (the same metric through moe_layer with the step's x copied in from
+pinned host memory and y copied back, inside the timed region); ``clocks``
+(nvidia-smi samples taken during the timed region).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill MXF4 TFLOPS as % of roofline"
+EXPERT_BYTES_PER_ROW_BLOCK = 17   # 16 packed bytes + 1 E8M0 code per 32 weights
+
+
+def workload_label(w):
+    lat = f" L={w.L}" if w.L else ""
+    return (f"{w.name}: T={w.T} H={w.H} I={w.I} E={w.E} k={w.k} I_shared={w.I_shared}{lat}"
+            f" skew={w.skew}")
+
+
+def expert_bytes(w):
+    """HBM bytes of one routed expert (gate + up + down, codes + scales)."""
+    per_matrix = w.I * w.W // 32 * EXPERT_BYTES_PER_ROW_BLOCK
+    return 3 * per_matrix
+
+
+def dense_bytes(w):
+    b = 2 * (w.E * w.H + 3 * w.I_shared * w.H + w.H)
+    if w.L:
+        b += 2 * 2 * w.L * w.H
+    return b
+
+
+def layer_bytes(w, n_active):
+    """Algorithmic bytes of one layer pass: every weight read once plus x in and y out."""
+    return n_active * expert_bytes(w) + dense_bytes(w) + w.T * w.H * 2 + w.T * w.H * 4
+
+
+def ffn_bytes(w, n_active):
+    """Algorithmic bytes of one moe_expert_ffn call: routed weights, x_op rows, y_perm rows."""
+    R = w.T * w.k
+    return n_active * expert_bytes(w) + w.T * w.W * 2 + R * w.W * 4
+
+
+def layer_flops(w):
+    R = w.T * w.k
+    f = 2 * R * 3 * w.I * w.W + 2 * w.T * (3 * w.I_shared * w.H + w.H) + 2 * w.T * w.E * w.H
+    if w.L:
+        f += 2 * 2 * w.T * w.L * w.H
+    return f
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_env():
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), n
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_routed_expert_04_b200 as M
+    from mxfp4_routed_expert_04_b200 import synth
+
+    rank, local_rank, world = _dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = synth.to_device(w)
+    dims = M.MoeDims.of(w, M.ACT_BF16)
+    layer = M.MoeLayer(dims, {k: v for k, v in dev.items() if k != "x"})
+    x = dev["x"]
+    stream = torch.cuda.Stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm up eagerly (first call also does the per-device set-up), then capture
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            layer(x, stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        layer(x, stream)
+    torch.cuda.synchronize()
+    n_active = int((layer.counts > 0).sum())
+
+    launches_per_step = 10 + (3 if w.L else 0)
+
+    def timed(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    def soak(seconds):
+        # the same flushed step, untimed, so the clock samples see the timed region's load
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            with torch.cuda.stream(stream):
+                for _ in range(50):
+                    flush.zero_()
+                    graph.replay()
+            torch.cuda.synchronize()
+
+    with ClockSampler(local_rank) as clk:
+        soak(0.7)
+        ms = timed(graph.replay, args.steps)
+        soak(0.7)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = sum(ms) / len(ms)
+    if world > 1:
+        t = torch.tensor([step_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+
+    # dominant call alone: moe_expert_ffn on the routing of the captured step
+    def ffn():
+        M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.row_token, dev["wg_q"],
+                         dev["wg_s"], dev["wu_q"], dev["wu_s"], dev["wd_q"], dev["wd_s"],
+                         layer.y_perm, layer.ws, stream)
+    timed(ffn, 3)
+    ffn_ms = statistics.mean(timed(ffn, max(5, args.steps)))
+
+    # end to end through moe_layer with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(w.T, w.H, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        graph.replay()
+        y_host.copy_(layer.y, non_blocking=True)
+    timed(e2e_step, 3)
+    e2e_ms = statistics.mean(timed(e2e_step, args.steps))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        if world > 1:
+            del graph
+            dist.destroy_process_group()
+        return None
+    peak, peak_kind = _peaks()
+    fb = ffn_bytes(w, n_active)
+    achieved = fb / (ffn_ms * 1e-3) / 1e9
+    lb = layer_bytes(w, n_active)
+    tokens = w.T * world
+    out = {
+        "metric": METRIC,
+        "value": tokens / (step_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "mxfp4 weights x f16 activations, fp32 accumulate",
+        "data": "synthetic (seeded; BASELINE distributions)",
+        "config": {"workload": workload_label(w), "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (512 MiB write, outside the events)",
+                   "act_mode": "bf16", "active_experts": n_active},
+        "layer": {"algorithmic_bytes": lb, "hbm_gbs": lb / (step_ms * 1e-3) / 1e9,
+                  "hbm_frac": lb / (step_ms * 1e-3) / 1e9 / peak,
+                  "tflops": layer_flops(w) / (step_ms * 1e-3) / 1e12},
+        "roofline": {"kernel": "moe_expert_ffn (k_gateup_mxfp4 + k_down_mxfp4)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "bytes_per_launch": fb, "ms_per_launch": ffn_ms, "traffic": None},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
+                "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+        "clocks_note": "nvidia-smi every 200 ms over the timed steps plus 0.7 s of the same "
+                       "flushed step on either side",
+    }
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    if world > 1:
+        del graph
+        dist.destroy_process_group()
+    return out
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def _oracle_token_pass(w, t, dense, getter):
+    import oracle as O
+    sub = dict(dense, x=dense["x"][t:t + 1])
+    return O.moe_layer(sub, w.k, getter)
+
+
+def cpu_baseline(w, budget_s: float = 20.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
+    tokens of the same batch, one at a time, until about ``budget_s`` seconds."""
+    from mxfp4_routed_expert_04_b200 import synth
+
+    dense = synth.dense_inputs(w)
+    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
+
+    def getter(e):
+        return (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
+
+    t0 = time.perf_counter()
+    n = 0
+    while n < w.T and (n == 0 or time.perf_counter() - t0 < budget_s):
+        _oracle_token_pass(w, n, dense, getter)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{n} token(s) of {w.name}, each a full layer pass (routing, its k experts "
+                      f"decoded to fp64, shared expert, combine), {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    """The reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    rank, _, world = _dist_env()
+    if rank != 0:
+        return None
+    from mxfp4_routed_expert_04_b200 import synth
+
+    dense = synth.dense_inputs(w)
+    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
+
+    def getter(e):
+        return (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
+
+    # each step is one token's full layer pass; keep the whole run within a few minutes
+    t0 = time.perf_counter()
+    _oracle_token_pass(w, 0, dense, getter)            # one warm-up pass (also sizes the run)
+    per = time.perf_counter() - t0
+    steps = max(1, min(args.steps, int(200.0 / max(per, 1e-3))))
+    times = []
+    for i in range(steps):
+        t0 = time.perf_counter()
+        _oracle_token_pass(w, i % w.T, dense, getter)
+        times.append(time.perf_counter() - t0)
+    step = statistics.mean(times)
+    v = 1.0 / step
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": 1, "ms_per_step": step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; BASELINE distributions)",
+        "config": {"workload": workload_label(w), "parallelism": "host cores, rank 0",
+                   "step": "one token of the batch through the whole layer"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"{steps} single-token layer passes of {w.name} "
+                                   f"(steps capped so the run stays near 200 s)"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from mxfp4_routed_expert_04_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    res = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * moe_mxfp4.h -- C ABI of the routed MXFP4 Mixture-of-Experts FFN layer on
+ * B200 (sm_100a).
+ *
+ * The layer (rabbit README, ferrumox/rabbit, model table row "MoE routing":
+ * "softmax top-10 of 512 + gated shared expert", routed experts read as OCP
+ * MXFP4; the "expert matmul" phase of its decode-step breakdown) computes, for
+ * every token t of x [T, H]:
+ *
+ *   logits = Wr x_t                         router, fp32 accumulate
+ *   idx, w = top-k of softmax(logits)       lowest index wins ties, w renormalised
+ *   y_t    = sum_j w_j * FFN_{idx_j}(x_t)  routed SwiGLU experts on MXFP4 weights
+ *          + sigmoid(w_sg . x_t) * FFN_shared(x_t)      gated bf16 shared expert
+ *
+ * with FFN_e(x) = Wd_e (silu(Wg_e x) * (Wu_e x)). The latent-width variant
+ * ("Ran Moonshot's 2.8T-parameter Kimi K3 on a GPU-less mini-PC", architecture
+ * paragraph: Stable LatentMoE, routed experts compute in a narrower latent
+ * width) runs the routed experts on x_lat = bf16(W_ld x) [T, L] and maps their
+ * weighted sum back with W_lu [H, L] before the shared expert is added.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All pointers are DEVICE pointers on the current CUDA device unless a
+ *   parameter says otherwise; the caller owns every buffer. No call allocates
+ *   or frees device memory; scratch comes from the caller's workspace.
+ * - bf16 tensors are passed as uint16_t bit patterns. Matrices are row-major;
+ *   weight matrices are [out, in] with the input dimension contiguous.
+ * - MXFP4 matrix [N, K] (OCP MX v1.0, section 5: E2M1 elements, E8M0 scale per
+ *   32 elements): q [N, K/2] uint8, element 2j of a row is the LOW nibble of
+ *   byte j and element 2j+1 the HIGH nibble; s [N, K/32] uint8, one E8M0 code
+ *   per 32 consecutive elements of a row (value 2^(c-127); code 255 is NaN and
+ *   poisons its block, IEEE propagation, not an error). Experts are stacked:
+ *   Wg, Wu as q [E, I, W/2] + s [E, I, W/32]; Wd as q [E, W, I/2] + s [E, W, I/32],
+ *   where W = L for latent layers, else H.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *   enqueues work on it and returns; nothing is synchronised.
+ * - Synchronous validation: null or misaligned (16-byte) pointers, shapes this
+ *   build does not support, or a workspace smaller than moe_workspace_size()
+ *   return an error status and enqueue NOTHING. moe_last_error() then holds a
+ *   one-line reason (thread-local).
+ * - Data errors found on the device (an expert index outside [0, E) or repeated
+ *   within a token) set a status word in the workspace; the affected call then
+ *   produces empty routing (all counts 0) instead of touching memory out of
+ *   range. Read it with moe_device_status().
+ *
+ * Supported shapes: 1 <= T <= 65536; H, I, I_shared, L multiples of 64;
+ * 1 <= k <= min(E, 32); 1 <= E <= 4096. act_mode MOE_ACT_MXFP4 further needs
+ * W and I multiples of 128.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, null dims, bad enum */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* a dimension outside the supported set */
+  MOE_ERR_ALIGNMENT = 3,          /* a pointer not 16-byte aligned */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+  MOE_ERR_CUDA = 5,               /* a CUDA runtime call failed (launch, event) */
+  MOE_ERR_DEVICE_STATUS = 6       /* returned by moe_device_status() when the
+                                     device flagged a data error */
+} moe_status;
+
+/* How the routed experts receive their activations. */
+typedef enum {
+  /* bf16 activations. x is carried exactly (as f16 scaled by a power of two
+   * per 32-element block); h = silu(g)*u enters the down projection as f16
+   * with a power-of-two scale per 32-element block (relative rounding
+   * <= 2^-11). Decode path: a tensor-core grouped GEMV. */
+  MOE_ACT_BF16 = 0,
+  /* MXFP4 activations: x rows and h are quantised to OCP MXFP4 (32-element
+   * blocks, OCP MX v1.0 section 6.3 conversion) and the experts run as
+   * block-scaled MXF4 tensor-core GEMMs (prefill path). */
+  MOE_ACT_MXFP4 = 1
+} moe_act_mode;
+
+typedef struct {
+  int32_t T;         /* tokens */
+  int32_t H;         /* hidden width */
+  int32_t I;         /* routed-expert intermediate width */
+  int32_t E;         /* routed experts */
+  int32_t k;         /* experts per token */
+  int32_t I_shared;  /* shared-expert intermediate width */
+  int32_t L;         /* latent width of the routed experts; 0 = none (W = H) */
+  int32_t act_mode;  /* moe_act_mode */
+} moe_dims;
+
+/* One-line description of a status code (static storage). */
+const char* moe_status_string(moe_status s);
+
+/* Reason for the last non-OK status returned on this host thread. */
+const char* moe_last_error(void);
+
+/* Bytes of device workspace every call below needs for `dims` (the same
+ * buffer serves all calls; it must stay valid until the enqueued work has
+ * run). Returns 0 for dims that fail validation. */
+size_t moe_workspace_size(const moe_dims* dims);
+
+/* Bytes of the activation operand buffer written by moe_permute and read by
+ * moe_expert_ffn (x_op below). Returns 0 for invalid dims. */
+size_t moe_x_op_size(const moe_dims* dims);
+
+/* Clear the device status word in `ws` (enqueued on `stream`). Call once
+ * after allocating a workspace. */
+moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream);
+
+/* Wait for `stream`, then copy the device status word into *host_status
+ * (HOST pointer; 0 = no data error). Returns MOE_ERR_DEVICE_STATUS when the
+ * word is non-zero, MOE_OK otherwise. Bit 0: an expert index outside [0, E);
+ * bit 1: an expert repeated within one token. */
+moe_status moe_device_status(const void* ws, int32_t* host_status, void* stream);
+
+/* --- a1-a2: router ---------------------------------------------------------
+ * logits[t, e] = sum_h x[t, h] Wr[e, h] (bf16 products are exact, fp32
+ * accumulation), p = softmax(logits[t]) in fp32, the k largest logits are
+ * selected (equal logits: lower expert index first; slots ordered by
+ * descending logit) and topk_w[t, j] = p[idx_j] / sum_j' p[idx_j'].
+ *   x         [T, H] bf16           w_router [E, H] bf16
+ *   topk_idx  [T, k] int32 (out)    topk_w   [T, k] fp32 (out)
+ *   logits    [T, E] fp32 (out, may be NULL)
+ */
+moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
+                     int32_t* topk_idx, float* topk_w, float* logits,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* --- a3-a4: permutation ----------------------------------------------------
+ * Groups the T*k (token, slot) pairs by expert: counts[e] pairs per expert,
+ * offsets = exclusive prefix sum (E+1 entries), permuted rows ordered by
+ * expert and, inside an expert, by ascending token. row_token[r] / row_slot[r]
+ * give the pair at permuted row r; slot_row[t, j] the row of pair (t, j).
+ * It also writes the activation operand x_op from x_in ([T, W] bf16: x, or
+ * x_lat for latent layers), ONE ROW PER TOKEN; the expert kernels gather the
+ * rows they need through row_token, so no duplicated [T*k, W] copy is made.
+ *   x_op format, MOE_ACT_BF16: f16 values [T, W], then fp32 block scales
+ *     [T, W/32] (value = f16 * scale, scale a power of two per 32 elements).
+ *   x_op format, MOE_ACT_MXFP4: codes [T, W/2] uint8 (low nibble first), then
+ *     E8M0 scale codes [T, W/32] uint8 (OCP MX v1.0 conversion, ties to even).
+ *   topk_idx [T, k] int32; counts [E], offsets [E+1], row_token [T*k],
+ *   row_slot [T*k], slot_row [T, k] int32 (out); x_op moe_x_op_size() bytes (out)
+ */
+moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
+                       int32_t* counts, int32_t* offsets, int32_t* row_token,
+                       int32_t* row_slot, int32_t* slot_row, void* x_op,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* --- a5-a7: routed experts (the "expert matmul") ----------------------------
+ * For every permuted row r of expert e (offsets[e] <= r < offsets[e+1]) and
+ * its token t = row_token[r]:
+ *   y_perm[r] = Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) )      [W] fp32
+ * Weights in the canonical MXFP4 layout above, decoded exactly (E2M1 value x
+ * E8M0 scale); products accumulate in fp32.
+ *   x_op, offsets, row_token as written by moe_permute; y_perm [T*k, W] fp32 (out)
+ */
+moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t* offsets,
+                          const int32_t* row_token,
+                          const uint8_t* wg_q, const uint8_t* wg_s,
+                          const uint8_t* wu_q, const uint8_t* wu_s,
+                          const uint8_t* wd_q, const uint8_t* wd_s,
+                          float* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* --- a8-a9 (+a10 up): shared expert and combine ------------------------------
+ *   s_t = sigmoid(w_sgate . x_t) * Ws_down (silu(Ws_gate x_t) * (Ws_up x_t))
+ *   y_t = [W_lu] (sum_j topk_w[t, j] * y_perm[slot_row[t, j]]) + s_t
+ * W_lu is applied only for latent layers (w_lat_up non-NULL iff L > 0).
+ *   x [T, H] bf16; w_sgate [H]; ws_gate, ws_up [I_shared, H]; ws_down
+ *   [H, I_shared]; w_lat_up [H, L] bf16; y [T, H] fp32 (out)
+ */
+moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* slot_row,
+                       const float* topk_w, const uint16_t* x, const uint16_t* w_sgate,
+                       const uint16_t* ws_gate, const uint16_t* ws_up, const uint16_t* ws_down,
+                       const uint16_t* w_lat_up, float* y,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* --- a10: latent down-projection (latent layers only) ------------------------
+ * x_lat[t] = bf16_rne( W_ld x_t ),  W_ld [L, H] bf16, x_lat [T, L] bf16 (out).
+ */
+moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16_t* w_lat_down,
+                           uint16_t* x_lat, void* ws, size_t ws_bytes, void* stream);
+
+/* --- the whole layer ---------------------------------------------------------
+ * Every buffer of the calls above in one struct; moe_layer enqueues the same
+ * kernels as route -> (latent_down) -> permute -> expert_ffn -> combine, with
+ * the shared expert (and the latent projection) running on a second stream
+ * forked from and joined back into `stream` (capturable in a CUDA graph).
+ */
+typedef struct {
+  const uint16_t* x;
+  const uint16_t* w_router;
+  const uint8_t *wg_q, *wg_s, *wu_q, *wu_s, *wd_q, *wd_s;
+  const uint16_t* w_sgate;
+  const uint16_t *ws_gate, *ws_up, *ws_down;
+  const uint16_t *w_lat_down, *w_lat_up;   /* NULL unless L > 0 */
+  /* outputs and intermediates (all caller-owned) */
+  int32_t* topk_idx;   /* [T, k] */
+  float* topk_w;       /* [T, k] */
+  int32_t *counts, *offsets, *row_token, *row_slot, *slot_row;
+  uint16_t* x_lat;     /* [T, L], NULL unless L > 0 */
+  void* x_op;          /* moe_x_op_size() bytes */
+  float* y_perm;       /* [T*k, W] */
+  float* y;            /* [T, H] */
+} moe_layer_args;
+
+moe_status moe_layer(const moe_dims* dims, const moe_layer_args* args,
+                     void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,457 @@
+// C ABI of the routed MXFP4 MoE layer: validation, workspace plan, launch
+// order. Declared in include/moe_mxfp4.h.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/moe_mxfp4.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+constexpr int kNumSMs = 148;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Number of K splits of a dense GEMV: enough warps to cover the GPU, each split
+// a whole number of 32-element steps and at least 4 of them.
+int dense_splits(int N, int T, int K) {
+  const long warps = (long)((N + 15) / 16) * ((T + 31) / 32);
+  const int ksteps = K / 32;
+  int S = 1;
+  for (int c = 1; c <= ksteps; ++c) {
+    if (ksteps % c) continue;
+    if (ksteps / c < 4) break;
+    S = c;
+    if (warps * c >= (long)kNumSMs * 8) break;
+  }
+  return S;
+}
+
+struct Plan {
+  int T, H, I, E, k, Is, L, W, R, mode;
+  int S_router, S_sgu, S_sd, S_ld, S_lu;
+  size_t off_status, off_router, off_h16, off_hscale, off_sgu, off_hs, off_gl, off_sd, off_ld,
+      off_ylat, off_lu, total;
+  size_t xop_bytes, xop_scale_off;
+};
+
+moe_status check_dims(const moe_dims* d) {
+  if (!d) return fail(MOE_ERR_INVALID_ARG, "dims is NULL");
+  if (d->act_mode != MOE_ACT_BF16 && d->act_mode != MOE_ACT_MXFP4)
+    return fail(MOE_ERR_INVALID_ARG, "act_mode %d is not a moe_act_mode", d->act_mode);
+  if (d->T < 1 || d->T > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T=%d outside [1, 65536]", d->T);
+  if (d->E < 1 || d->E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 1024]", d->E);
+  if (d->k < 1 || d->k > 32 || d->k > d->E)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, min(E, 32)]", d->k);
+  const int dims4[4] = {d->H, d->I, d->I_shared, d->L};
+  const char* names[4] = {"H", "I", "I_shared", "L"};
+  for (int i = 0; i < 4; ++i) {
+    if (i == 3 && d->L == 0) continue;
+    if (dims4[i] < 128 || dims4[i] % 128 != 0 || dims4[i] > (1 << 16))
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s=%d is not a multiple of 128 in [128, 65536]",
+                  names[i], dims4[i]);
+  }
+  if ((long)d->T * d->k > (1L << 24))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T*k=%ld above 2^24", (long)d->T * d->k);
+  return MOE_OK;
+}
+
+moe_status make_plan(const moe_dims* d, Plan& p) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  p.T = d->T; p.H = d->H; p.I = d->I; p.E = d->E; p.k = d->k; p.Is = d->I_shared; p.L = d->L;
+  p.W = d->L ? d->L : d->H;
+  p.R = d->T * d->k;
+  p.mode = d->act_mode;
+  p.S_router = dense_splits(p.E, p.T, p.H);
+  p.S_sgu = dense_splits(2 * p.Is + 1, p.T, p.H);
+  p.S_sd = dense_splits(p.H, p.T, p.Is);
+  p.S_ld = p.L ? dense_splits(p.L, p.T, p.H) : 0;
+  p.S_lu = p.L ? dense_splits(p.H, p.T, p.L) : 0;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 256); return r; };
+  p.off_status = take(256);
+  p.off_router = take((size_t)p.S_router * p.T * p.E * 4);
+  p.off_h16 = take((size_t)p.R * p.I * 2);
+  p.off_hscale = take((size_t)(p.I / 16) * p.R * 4);
+  p.off_sgu = take((size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
+  p.off_hs = take((size_t)p.T * p.Is * 4);
+  p.off_gl = take((size_t)p.T * 4);
+  p.off_sd = take((size_t)p.S_sd * p.T * p.H * 4);
+  p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
+  p.off_ylat = take(p.L ? (size_t)p.T * p.L * 4 : 0);
+  p.off_lu = take(p.L ? (size_t)p.S_lu * p.T * p.H * 4 : 0);
+  p.total = o;
+  if (p.mode == MOE_ACT_BF16) {
+    p.xop_scale_off = align_up((size_t)p.T * p.W * 2, 256);
+    p.xop_bytes = p.xop_scale_off + (size_t)p.T * 4;
+  } else {
+    p.xop_scale_off = align_up((size_t)p.T * p.W / 2, 256);
+    p.xop_bytes = p.xop_scale_off + (size_t)p.T * (p.W / 32);
+  }
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+moe_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned16(ws)) return fail(MOE_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+  if (ws_bytes < p.total)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, p.total);
+  return MOE_OK;
+}
+
+#define CHECK_PTR(p)                                                                   \
+  do {                                                                                 \
+    if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #p);                      \
+    if (!aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+moe_status launched(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+// per-device one-time setup: kernel attributes, the side stream and events of moe_layer
+struct DeviceState {
+  bool ready = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_lat = nullptr, ev_shared = nullptr;
+};
+std::mutex g_mu;
+DeviceState g_dev[64];
+
+moe_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(MOE_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    cudaError_t e = cudaFuncSetAttribute(moe::k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)moe::permute_smem_bytes(1024));
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s.side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_lat, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_shared, cudaEventDisableTiming);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "device setup: %s", cudaGetErrorString(e));
+    s.ready = true;
+  }
+  *out = &s;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// launchers (arguments already validated)
+// ---------------------------------------------------------------------------
+moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, const uint16_t* w2,
+                        int r2, const void* x, bool x_f32, float* part, int T, int K, int S,
+                        cudaStream_t st, const char* what) {
+  moe::DenseArgs a;
+  a.w[0] = w0; a.w[1] = w1 ? w1 : w0; a.w[2] = w2 ? w2 : w0;
+  a.rows[0] = r0; a.rows[1] = r1; a.rows[2] = r2;
+  a.N = r0 + r1 + r2;
+  a.x = x; a.x_f32 = x_f32 ? 1 : 0;
+  a.part = part;
+  a.T = T; a.K = K; a.S = S; a.kper = K / S;
+  const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (T + 31) / 32);
+  moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, st>>>(a);
+  return launched(what);
+}
+
+moe_status do_route(const Plan& p, const uint16_t* x, const uint16_t* wr, int32_t* idx, float* w,
+                    float* logits, void* ws, cudaStream_t st) {
+  float* part = at<float>(ws, p.off_router);
+  moe_status s = launch_dense(wr, p.E, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H,
+                              p.S_router, st, "router gemv");
+  if (s != MOE_OK) return s;
+  moe::k_topk<<<(p.T + 7) / 8, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
+  return launched("top-k");
+}
+
+moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, int32_t* counts,
+                      int32_t* offsets, int32_t* row_token, int32_t* row_slot, int32_t* slot_row,
+                      void* x_op, void* ws, cudaStream_t st) {
+  moe::k_permute<<<1, 1024, moe::permute_smem_bytes(p.E), st>>>(
+      idx, p.T, p.k, p.E, counts, offsets, row_token, row_slot, slot_row, at<int32_t>(ws, p.off_status));
+  moe_status s = launched("permute");
+  if (s != MOE_OK) return s;
+  if (p.mode == MOE_ACT_BF16) {
+    moe::k_act_to_f16<<<p.T, 256, 0, st>>>(xin, p.W, static_cast<__half*>(x_op),
+                                            at<float>(x_op, p.xop_scale_off));
+  } else {
+    moe::k_act_to_mxfp4<<<p.T, 256, 0, st>>>(xin, p.W, static_cast<uint8_t*>(x_op),
+                                              at<uint8_t>(x_op, p.xop_scale_off));
+  }
+  return launched("activation operand");
+}
+
+moe_status do_expert_ffn(const Plan& p, const void* x_op, const int32_t* offsets,
+                         const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
+                         const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
+                         const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
+  if (p.mode != MOE_ACT_BF16)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "act_mode MOE_ACT_MXFP4 expert GEMM is not available");
+  const int ny = p.E < p.R ? p.E : p.R;
+  moe::GateUpArgs g;
+  g.x16 = static_cast<const __half*>(x_op);
+  g.xscale = reinterpret_cast<const float*>(static_cast<const char*>(x_op) + p.xop_scale_off);
+  g.offsets = offsets; g.row_token = row_token;
+  g.wg_q = wg_q; g.wg_s = wg_s; g.wu_q = wu_q; g.wu_s = wu_s;
+  g.h16 = at<__half>(ws, p.off_h16);
+  g.hscale = at<float>(ws, p.off_hscale);
+  g.W = p.W; g.I = p.I; g.E = p.E; g.R = p.R;
+  const size_t smem = moe::gemv_mxfp4_smem_bytes();
+  moe::k_gateup_mxfp4<<<dim3(p.I / 16, ny), 32, smem, st>>>(g);
+  moe_status s = launched("expert gate/up");
+  if (s != MOE_OK) return s;
+  moe::DownArgs d;
+  d.h16 = g.h16; d.hscale = g.hscale; d.offsets = offsets;
+  d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
+  d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
+  moe::k_down_mxfp4<<<dim3(p.W / 32, ny), 32, smem, st>>>(d);
+  return launched("expert down");
+}
+
+moe_status do_shared(const Plan& p, const uint16_t* x, const uint16_t* w_sgate,
+                     const uint16_t* ws_gate, const uint16_t* ws_up, const uint16_t* ws_down,
+                     void* ws, cudaStream_t st) {
+  float* sgu = at<float>(ws, p.off_sgu);
+  moe_status s = launch_dense(ws_gate, p.Is, ws_up, p.Is, w_sgate, 1, x, false, sgu, p.T, p.H,
+                              p.S_sgu, st, "shared gate/up gemv");
+  if (s != MOE_OK) return s;
+  moe::k_shared_swiglu<<<dim3((p.Is + 255) / 256, p.T), 256, 0, st>>>(
+      sgu, p.S_sgu, p.T, p.Is, at<float>(ws, p.off_hs), at<float>(ws, p.off_gl));
+  s = launched("shared swiglu");
+  if (s != MOE_OK) return s;
+  return launch_dense(ws_down, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_hs), true,
+                      at<float>(ws, p.off_sd), p.T, p.Is, p.S_sd, st, "shared down gemv");
+}
+
+moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row, const float* topk_w,
+                    const uint16_t* w_lat_up, float* y, void* ws, cudaStream_t st) {
+  moe::CombineArgs c;
+  c.slot_row = slot_row; c.topk_w = topk_w; c.k = p.k;
+  c.gate_logit = at<float>(ws, p.off_gl);
+  c.T = p.T;
+  if (p.L) {
+    // routed weighted sum at width L, then the up-projection, then + shared
+    c.y_perm = y_perm; c.add1 = nullptr; c.S1 = 0; c.add2 = nullptr; c.S2 = 0;
+    c.out = at<float>(ws, p.off_ylat); c.width = p.L;
+    moe::k_combine<<<dim3((p.L / 4 + 255) / 256, p.T), 256, 0, st>>>(c);
+    moe_status s = launched("latent combine");
+    if (s != MOE_OK) return s;
+    s = launch_dense(w_lat_up, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_ylat), true,
+                     at<float>(ws, p.off_lu), p.T, p.L, p.S_lu, st, "latent up gemv");
+    if (s != MOE_OK) return s;
+    c.y_perm = nullptr;
+    c.add1 = at<float>(ws, p.off_lu); c.S1 = p.S_lu;
+  } else {
+    c.y_perm = y_perm; c.add1 = nullptr; c.S1 = 0;
+  }
+  c.add2 = at<float>(ws, p.off_sd); c.S2 = p.S_sd;
+  c.out = y; c.width = p.H;
+  moe::k_combine<<<dim3((p.H / 4 + 255) / 256, p.T), 256, 0, st>>>(c);
+  return launched("combine");
+}
+
+moe_status do_latent_down(const Plan& p, const uint16_t* x, const uint16_t* w_ld, uint16_t* x_lat,
+                          void* ws, cudaStream_t st) {
+  float* part = at<float>(ws, p.off_ld);
+  moe_status s = launch_dense(w_ld, p.L, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_ld, st,
+                              "latent down gemv");
+  if (s != MOE_OK) return s;
+  moe::k_round_bf16<<<dim3((p.L + 255) / 256, p.T), 256, 0, st>>>(part, p.S_ld, p.T, p.L, x_lat);
+  return launched("latent round");
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_STATUS: return "device flagged a data error";
+  }
+  return "unknown status";
+}
+
+const char* moe_last_error(void) { return g_err; }
+
+size_t moe_workspace_size(const moe_dims* dims) {
+  Plan p;
+  return make_plan(dims, p) == MOE_OK ? p.total : 0;
+}
+
+size_t moe_x_op_size(const moe_dims* dims) {
+  Plan p;
+  return make_plan(dims, p) == MOE_OK ? p.xop_bytes : 0;
+}
+
+moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  const cudaError_t e = cudaMemsetAsync(at<char>(ws, p.off_status), 0, 256, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+moe_status moe_device_status(const void* ws, int32_t* host_status, void* stream) {
+  if (!ws || !host_status) return fail(MOE_ERR_INVALID_ARG, "ws or host_status is NULL");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  *host_status = v;
+  return v ? fail(MOE_ERR_DEVICE_STATUS, "device status word 0x%x", v) : MOE_OK;
+}
+
+moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
+                     int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
+                     void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  CHECK_PTR(x); CHECK_PTR(w_router); CHECK_PTR(topk_idx); CHECK_PTR(topk_w);
+  if (logits && !aligned16(logits)) return fail(MOE_ERR_ALIGNMENT, "logits not 16-byte aligned");
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  return do_route(p, x, w_router, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
+                       int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* row_slot,
+                       int32_t* slot_row, void* x_op, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  CHECK_PTR(topk_idx); CHECK_PTR(x_in); CHECK_PTR(counts); CHECK_PTR(offsets);
+  CHECK_PTR(row_token); CHECK_PTR(row_slot); CHECK_PTR(slot_row); CHECK_PTR(x_op);
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  return do_permute(p, topk_idx, x_in, counts, offsets, row_token, row_slot, slot_row, x_op, ws,
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t* offsets,
+                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
+                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
+                          const uint8_t* wd_s, float* y_perm, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  CHECK_PTR(x_op); CHECK_PTR(offsets); CHECK_PTR(row_token);
+  CHECK_PTR(wg_q); CHECK_PTR(wg_s); CHECK_PTR(wu_q); CHECK_PTR(wu_s); CHECK_PTR(wd_q); CHECK_PTR(wd_s);
+  CHECK_PTR(y_perm);
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  return do_expert_ffn(p, x_op, offsets, row_token, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws,
+                       (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* slot_row,
+                       const float* topk_w, const uint16_t* x, const uint16_t* w_sgate,
+                       const uint16_t* ws_gate, const uint16_t* ws_up, const uint16_t* ws_down,
+                       const uint16_t* w_lat_up, float* y, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  CHECK_PTR(y_perm); CHECK_PTR(slot_row); CHECK_PTR(topk_w); CHECK_PTR(x); CHECK_PTR(w_sgate);
+  CHECK_PTR(ws_gate); CHECK_PTR(ws_up); CHECK_PTR(ws_down); CHECK_PTR(y);
+  if (p.L) { CHECK_PTR(w_lat_up); }
+  else if (w_lat_up) return fail(MOE_ERR_INVALID_ARG, "w_lat_up given but L == 0");
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  const cudaStream_t st = (cudaStream_t)stream;
+  if ((s = do_shared(p, x, w_sgate, ws_gate, ws_up, ws_down, ws, st)) != MOE_OK) return s;
+  return do_final(p, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
+}
+
+moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16_t* w_lat_down,
+                           uint16_t* x_lat, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if (!p.L) return fail(MOE_ERR_INVALID_ARG, "moe_latent_down needs L > 0");
+  CHECK_PTR(x); CHECK_PTR(w_lat_down); CHECK_PTR(x_lat);
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  return do_latent_down(p, x, w_lat_down, x_lat, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, size_t ws_bytes,
+                     void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if (!a) return fail(MOE_ERR_INVALID_ARG, "args is NULL");
+  CHECK_PTR(a->x); CHECK_PTR(a->w_router);
+  CHECK_PTR(a->wg_q); CHECK_PTR(a->wg_s); CHECK_PTR(a->wu_q); CHECK_PTR(a->wu_s);
+  CHECK_PTR(a->wd_q); CHECK_PTR(a->wd_s);
+  CHECK_PTR(a->w_sgate); CHECK_PTR(a->ws_gate); CHECK_PTR(a->ws_up); CHECK_PTR(a->ws_down);
+  CHECK_PTR(a->topk_idx); CHECK_PTR(a->topk_w); CHECK_PTR(a->counts); CHECK_PTR(a->offsets);
+  CHECK_PTR(a->row_token); CHECK_PTR(a->row_slot); CHECK_PTR(a->slot_row); CHECK_PTR(a->x_op);
+  CHECK_PTR(a->y_perm); CHECK_PTR(a->y);
+  if (p.L) { CHECK_PTR(a->w_lat_down); CHECK_PTR(a->w_lat_up); CHECK_PTR(a->x_lat); }
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaEventRecord(ds->ev_fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ds->side, ds->ev_fork, 0);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
+  // side stream: latent projection, then the shared expert
+  if (p.L) {
+    if ((s = do_latent_down(p, a->x, a->w_lat_down, a->x_lat, ws, ds->side)) != MOE_OK) return s;
+    if ((e = cudaEventRecord(ds->ev_lat, ds->side)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
+  }
+  if ((s = do_shared(p, a->x, a->w_sgate, a->ws_gate, a->ws_up, a->ws_down, ws, ds->side)) != MOE_OK)
+    return s;
+  if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
+  // main stream: routing, experts, combine
+  if ((s = do_route(p, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st)) != MOE_OK) return s;
+  if (p.L && (e = cudaStreamWaitEvent(st, ds->ev_lat, 0)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
+  if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets, a->row_token,
+                      a->row_slot, a->slot_row, a->x_op, ws, st)) != MOE_OK)
+    return s;
+  if ((s = do_expert_ffn(p, a->x_op, a->offsets, a->row_token, a->wg_q, a->wg_s, a->wu_q, a->wu_s,
+                         a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
+    return s;
+  if ((e = cudaStreamWaitEvent(st, ds->ev_shared, 0)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
+  return do_final(p, a->y_perm, a->slot_row, a->topk_w, a->w_lat_up, a->y, ws, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+// Device helpers shared by the layer's kernels (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MOE_DEV __device__ __forceinline__
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// device status word (bit flags, kept in the caller's workspace)
+// ---------------------------------------------------------------------------
+enum : int32_t {
+  kStatusBadExpertIndex = 1,   // an expert index outside [0, E)
+  kStatusRepeatedExpert = 2,   // the same expert twice in one token's top-k
+};
+
+// ---------------------------------------------------------------------------
+// number formats
+// ---------------------------------------------------------------------------
+
+// bf16 bit pattern -> float (exact).
+MOE_DEV float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+// The two bf16 halves of a 32-bit word -> floats (exact).
+MOE_DEV float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+MOE_DEV float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// float -> bf16 bits, round to nearest even (finite inputs; NaN kept quiet).
+MOE_DEV uint32_t f32_to_bf16_rne(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7FFFFFFFu) > 0x7F800000u) return (b >> 16) | 0x40u;  // NaN
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return b >> 16;
+}
+
+// E8M0 scale code -> float: 2^(c-127); c = 0 gives the subnormal 2^-127 and
+// c = 255 gives NaN (OCP MX v1.0, section 5.4).
+MOE_DEV float e8m0_to_f32(uint32_t c) {
+  uint32_t bits = c << 23;
+  bits = (c == 0u) ? 0x00400000u : bits;
+  bits = (c == 255u) ? 0x7FC00000u : bits;
+  return __uint_as_float(bits);
+}
+
+// Four bytes of packed E2M1 pairs -> four f16x2 words (exact). Byte j of `w`
+// becomes out[j]; its low nibble goes to the low half.
+MOE_DEV void e2m1x8_to_f16x8(uint32_t w, uint32_t (&out)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w));
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core MMA (warp-level m16n8k16, fp32 accumulate)
+// ---------------------------------------------------------------------------
+MOE_DEV void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+MOE_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------
+// memory
+// ---------------------------------------------------------------------------
+MOE_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+MOE_DEV void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+MOE_DEV void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
+}
+MOE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+MOE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+MOE_DEV void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// 16-byte read-only global load that does not allocate in L1 (streamed weights).
+MOE_DEV uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+MOE_DEV uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// ---------------------------------------------------------------------------
+// misc
+// ---------------------------------------------------------------------------
+MOE_DEV float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+MOE_DEV float sigmoid_f32(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+// Expert of the a-th non-empty segment of `offsets` (E+1 entries), or -1.
+// Whole warp calls it; returns the same value in every lane.
+MOE_DEV int nth_active_expert(const int32_t* __restrict__ offsets, int E, int a, int lane) {
+  int seen = 0;
+  for (int base = 0; base < E; base += 32) {
+    const int e = base + lane;
+    const int cnt = (e < E) ? (__ldg(offsets + e + 1) - __ldg(offsets + e)) : 0;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, cnt > 0);
+    const int c = __popc(m);
+    if (seen + c > a) {
+      const int want = a - seen;
+      const int pre = __popc(m & ((1u << lane) - 1u));
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, cnt > 0 && pre == want);
+      return base + __ffs(hit) - 1;
+    }
+    seen += c;
+  }
+  return -1;
+}
+
+}  // namespace moe

@@ -1,0 +1,81 @@
+// Internal kernel interfaces of the MoE layer library (not part of the C ABI).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// --- grouped MXFP4 GEMV (decode) -------------------------------------------
+struct GateUpArgs {
+  const __half* x16;         // [T, W] f16 activation rows (one per token)
+  const float* xscale;       // [T] power-of-two row scales
+  const int32_t* offsets;    // [E+1]
+  const int32_t* row_token;  // [R]
+  const uint8_t *wg_q, *wg_s, *wu_q, *wu_s;
+  __half* h16;               // [R, I]
+  float* hscale;             // [I/16, R]
+  int W, I, E, R;
+};
+
+struct DownArgs {
+  const __half* h16;
+  const float* hscale;
+  const int32_t* offsets;
+  const uint8_t *wd_q, *wd_s;
+  float* y_perm;             // [R, W]
+  int W, I, E, R;
+};
+
+__global__ void k_gateup_mxfp4(GateUpArgs a);
+__global__ void k_down_mxfp4(DownArgs a);
+size_t gemv_mxfp4_smem_bytes();
+
+// --- dense bf16 GEMV with split-K partial sums -----------------------------
+struct DenseArgs {
+  const uint16_t* w[3];      // row segments of the weight matrix, each [rows, K]
+  int rows[3];
+  int N;                     // rows[0] + rows[1] + rows[2]
+  const void* x;             // [T, K] bf16 bits, or fp32 when x_f32
+  int x_f32;
+  float* part;               // [S, T, N] partial sums
+  int T, K, S, kper;         // kper = K / S, a multiple of 32
+};
+__global__ void k_dense_gemv(DenseArgs a);
+constexpr int kDenseWarps = 4;   // warps (16-row tiles) per CTA
+
+// --- router tail ------------------------------------------------------------
+__global__ void k_topk(const float* part, int S, int T, int E, int k, int32_t* idx, float* w,
+                       float* logits);
+
+// --- permutation and activation operands ------------------------------------
+__global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
+                          int32_t* offsets, int32_t* row_token, int32_t* row_slot,
+                          int32_t* slot_row, int32_t* status);
+size_t permute_smem_bytes(int E);
+__global__ void k_act_to_f16(const uint16_t* x, int W, __half* x16, float* xscale);
+__global__ void k_act_to_mxfp4(const uint16_t* x, int W, uint8_t* q, uint8_t* s);
+
+// --- finalisers of split-K partials ----------------------------------------
+__global__ void k_shared_swiglu(const float* part, int S, int T, int Is, float* hs,
+                                float* gate_logit);
+__global__ void k_round_bf16(const float* part, int S, int T, int N, uint16_t* out);
+
+struct CombineArgs {
+  const float* y_perm;       // [R, width] or NULL
+  const int32_t* slot_row;   // [T, k]
+  const float* topk_w;       // [T, k]
+  int k;
+  const float* add1;         // [S1, T, width] partials added as is, or NULL
+  int S1;
+  const float* add2;         // [S2, T, width] partials scaled by sigmoid(gate_logit[t]), or NULL
+  int S2;
+  const float* gate_logit;   // [T]
+  float* out;                // [T, width]
+  int T, width;
+};
+__global__ void k_combine(CombineArgs a);
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+// Token -> expert dispatch and the activation operands of the expert kernels.
+//
+// k_permute: per-expert histogram, exclusive scan and a stable placement of
+// the T*k (token, slot) pairs: rows grouped by expert, ascending token inside
+// an expert. One CTA of 1024 threads walks the pairs in chunks of 1024 in
+// (token, slot) order; inside a chunk a pair's rank among equal experts comes
+// from __match_any_sync within its warp plus a per-(warp, expert) exclusive
+// scan over the 32 warps, so the placement is deterministic.
+//
+// k_act_to_f16: bf16 activation rows -> f16 rows with one power-of-two scale
+// per row (the largest magnitude maps into [2^14, 2^15); bf16 values keep all
+// their bits down to 2^-29 of the row maximum).
+//
+// k_act_to_mxfp4: bf16 activation rows -> OCP MXFP4 (OCP MX v1.0 section 6.3
+// conversion: shared exponent floor(log2 amax) - 2, elements rounded to the
+// nearest E2M1 value with ties to the even code, saturating at 6).
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kPermThreads = 1024;
+constexpr int kPermWarps = kPermThreads / 32;
+
+size_t permute_smem_bytes(int E) {
+  return (size_t)(kPermWarps + 2) * E * sizeof(int32_t) + 16;
+}
+
+// grid 1, block 1024, dynamic smem permute_smem_bytes(E)
+__global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restrict__ idx, int T, int k,
+                                                        int E, int32_t* __restrict__ counts,
+                                                        int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ row_token,
+                                                        int32_t* __restrict__ row_slot,
+                                                        int32_t* __restrict__ slot_row,
+                                                        int32_t* __restrict__ status) {
+  extern __shared__ int32_t sm[];
+  int32_t* cnt = sm;                   // [E]  running cursor per expert
+  int32_t* whist = sm + E;             // [32][E] per-warp counts -> exclusive bases
+  int32_t* flag = sm + (kPermWarps + 1) * E;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = T * k;
+
+  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  if (tid == 0) flag[0] = 0;
+  __syncthreads();
+
+  // validate and count
+  for (int p = tid; p < R; p += kPermThreads) {
+    const int e = idx[p];
+    if (e < 0 || e >= E) {
+      atomicOr(&flag[0], kStatusBadExpertIndex);
+      continue;
+    }
+    const int t = p / k, j = p - t * k;
+    for (int jj = 0; jj < j; ++jj)
+      if (idx[t * k + jj] == e) atomicOr(&flag[0], kStatusRepeatedExpert);
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  const int bad = flag[0];
+  if (bad) {
+    for (int e = tid; e < E; e += kPermThreads) counts[e] = 0;
+    for (int e = tid; e <= E; e += kPermThreads) offsets[e] = 0;
+    if (tid == 0) atomicOr(status, bad);
+    return;
+  }
+
+  // exclusive scan of the counts (E <= 1024: one element per thread)
+  {
+    const int e = tid;
+    const int c = (e < E) ? cnt[e] : 0;
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    __shared__ int32_t wsum[kPermWarps];
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int ws = wsum[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, ws, off);
+        if (lane >= off) ws += y;
+      }
+      wsum[lane] = ws;       // inclusive warp totals
+    }
+    __syncthreads();
+    const int excl = incl - c + (warp > 0 ? wsum[warp - 1] : 0);
+    if (e < E) {
+      counts[e] = c;
+      offsets[e] = excl;
+      cnt[e] = excl;         // cursor
+    }
+    if (e == E - 1) offsets[E] = excl + c;
+  }
+  __syncthreads();
+
+  // stable placement, chunk by chunk
+  for (int base = 0; base < R; base += kPermThreads) {
+    for (int i = tid; i < kPermWarps * E; i += kPermThreads) whist[i] = 0;
+    __syncthreads();
+    const int p = base + tid;
+    const int e = (p < R) ? idx[p] : -1;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) whist[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += kPermThreads) {
+      int run = cnt[ee];
+      for (int w = 0; w < kPermWarps; ++w) {
+        const int c = whist[w * E + ee];
+        whist[w * E + ee] = run;
+        run += c;
+      }
+      cnt[ee] = run;
+    }
+    __syncthreads();
+    if (e >= 0) {
+      const int pos = whist[warp * E + e] + rank;
+      const int t = p / k;
+      row_token[pos] = t;
+      row_slot[pos] = p - t * k;
+      slot_row[p] = pos;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// activation operands, one CTA of 256 threads per token row
+// ---------------------------------------------------------------------------
+
+MOE_DEV float block_max_256(float v) {
+  __shared__ float red[8];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+  __syncthreads();
+  return m;
+}
+
+// grid T, block 256; W a multiple of 8
+__global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__ x, int W,
+                                                  __half* __restrict__ x16,
+                                                  float* __restrict__ xscale) {
+  const int tok = blockIdx.x;
+  const uint16_t* row = x + (size_t)tok * W;
+  float m = 0.0f;
+  for (int i = threadIdx.x * 8; i < W; i += 256 * 8) {
+    const uint4 v = ldg16(row + i);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16lo(wv[j])), fabsf(bf16hi(wv[j]))));
+  }
+  m = block_max_256(m);
+  float scale = 1.0f, inv = 1.0f;
+  if (m > 0.0f && isfinite(m)) {
+    int ex;
+    frexpf(m, &ex);
+    ex = max(-100, min(127, ex));
+    scale = ldexpf(1.0f, ex - 15);
+    inv = ldexpf(1.0f, 15 - ex);
+  }
+  for (int i = threadIdx.x * 8; i < W; i += 256 * 8) {
+    const uint4 v = ldg16(row + i);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2 h = __floats2half2_rn(bf16lo(wv[j]) * inv, bf16hi(wv[j]) * inv);
+      o[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(x16 + (size_t)tok * W + i) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (threadIdx.x == 0) xscale[tok] = scale;
+}
+
+// E2M1 code (0..7 magnitude) of a non-negative value already divided by the
+// block scale: nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even code.
+MOE_DEV uint32_t e2m1_magnitude_code(float s) {
+  return (uint32_t)(s > 0.25f) + (uint32_t)(s >= 0.75f) + (uint32_t)(s > 1.25f) +
+         (uint32_t)(s >= 1.75f) + (uint32_t)(s > 2.5f) + (uint32_t)(s >= 3.5f) +
+         (uint32_t)(s > 5.0f);
+}
+
+// grid T, block 256; W a multiple of 32. Each 4 consecutive threads own one
+// 32-element block (8 elements each).
+__global__ void __launch_bounds__(256) k_act_to_mxfp4(const uint16_t* __restrict__ x, int W,
+                                                    uint8_t* __restrict__ q,
+                                                    uint8_t* __restrict__ s) {
+  const int tok = blockIdx.x;
+  const uint16_t* row = x + (size_t)tok * W;
+  for (int base = 0; base < W; base += 256 * 8) {      // uniform trip count: shuffles below
+    const int i = base + threadIdx.x * 8;
+    const bool ok = i < W;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) v = ldg16(row + i);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { f[2 * j] = bf16lo(wv[j]); f[2 * j + 1] = bf16hi(wv[j]); }
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    int code_s = 0;
+    if (m > 0.0f) {
+      int ex;
+      frexpf(m, &ex);                    // floor(log2 m) = ex - 1
+      code_s = min(254, max(0, 127 + (ex - 1) - 2));
+    }
+    const float inv = ldexpf(1.0f, 127 - code_s);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t c = e2m1_magnitude_code(fabsf(f[j]) * inv) | (signbit(f[j]) ? 8u : 0u);
+      packed |= c << (4 * j);
+    }
+    if (ok) {
+      *reinterpret_cast<uint32_t*>(q + (size_t)tok * (W / 2) + i / 2) = packed;
+      if ((threadIdx.x & 3) == 0) s[(size_t)tok * (W / 32) + i / 32] = (uint8_t)code_s;
+    }
+  }
+}
+
+}  // namespace moe

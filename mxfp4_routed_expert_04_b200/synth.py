@@ -202,3 +202,38 @@ def workload_inputs(w: MoeWorkload, experts=None, threads=None) -> dict:
     d = dense_inputs(w)
     d.update(expert_weights(w, range(w.E) if experts is None else experts, threads))
     return d
+
+
+# ---------------------------------------------------------------------------
+# device copies (plumbing only)
+# ---------------------------------------------------------------------------
+
+def to_device(w: MoeWorkload, dense: dict | None = None, device="cuda", chunk: int = 32,
+              pinned: bool = False) -> dict:
+    """Upload a workload's weights (all E experts) and x to the GPU as torch tensors.
+
+    bf16 arrays become int16 tensors holding the bit patterns. Experts are
+    generated and copied ``chunk`` at a time to bound host memory."""
+    import torch
+
+    dense = dense_inputs(w) if dense is None else dense
+    out = {}
+    for name, arr in dense.items():
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16))
+        out[name] = t.to(device)
+    (Ng, Kg), (Nd, Kd) = expert_shapes(w)
+    shapes = {"wg_q": (Ng, Kg // 2), "wg_s": (Ng, Kg // 32), "wu_q": (Ng, Kg // 2),
+              "wu_s": (Ng, Kg // 32), "wd_q": (Nd, Kd // 2), "wd_s": (Nd, Kd // 32)}
+    for name, shp in shapes.items():
+        out[name] = torch.empty((w.E,) + shp, dtype=torch.uint8, device=device)
+    for e0 in range(0, w.E, chunk):
+        ids = list(range(e0, min(w.E, e0 + chunk)))
+        ex = expert_weights(w, ids)
+        for name in shapes:
+            src = torch.from_numpy(ex[name])
+            if pinned:
+                src = src.pin_memory()
+            out[name][e0:e0 + len(ids)].copy_(src, non_blocking=pinned)
+    if device != "cpu":
+        torch.cuda.synchronize()
+    return out

@@ -76,12 +76,13 @@ def mxfp4_dequant(q, s) -> np.ndarray:
     """
     q = np.asarray(q, dtype=np.uint8)
     s = np.asarray(s, dtype=np.uint8)
-    lo = e2m1_decode(q & np.uint8(0xF))
-    hi = e2m1_decode(q >> np.uint8(4))
-    vals = np.stack([lo, hi], axis=-1).reshape(*q.shape[:-1], q.shape[-1] * 2)
-    scale = np.repeat(e8m0_decode(s), 32, axis=-1)
+    # value pair of every byte: (low-nibble element, high-nibble element)
+    byte_vals = np.stack([e2m1_decode(np.arange(256) & 0xF), e2m1_decode(np.arange(256) >> 4)],
+                         axis=-1)
+    vals = byte_vals[q].reshape(*q.shape[:-1], q.shape[-1] // 16, 32)   # [..., N, K/32, 32]
     with np.errstate(invalid="ignore"):
-        return vals * scale
+        vals *= e8m0_decode(s)[..., None]
+    return vals.reshape(*q.shape[:-1], q.shape[-1] * 2)
 
 
 def bf16_to_f64(bits) -> np.ndarray:

@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+the header declares, and rejects bad arguments synchronously (before any CUDA
+call). None of these calls reaches a kernel launch: every case fails one
+host-side check, so they are safe with or without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mxfp4_routed_expert_04_b200 as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_mxfp4.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_function():
+    names = _declared_functions()
+    assert len(names) >= 12, names
+    lib = ctypes.CDLL(M.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _dims(**kw):
+    base = dict(T=4, H=256, I=128, E=16, k=2, I_shared=128, L=0, act_mode=0)
+    base.update(kw)
+    return M.MoeDims(**base)
+
+
+@pytest.mark.parametrize("kw,field", [
+    (dict(T=0), "T="), (dict(H=100), "H="), (dict(I=64), "I="), (dict(E=0), "E="),
+    (dict(k=17), "k="), (dict(k=33, E=64), "k="), (dict(L=96), "L="), (dict(I_shared=0), "I_shared="),
+    (dict(act_mode=7), "act_mode"), (dict(E=2048), "E="),
+])
+def test_invalid_dims_have_no_workspace(kw, field):
+    assert M.moe_workspace_size(_dims(**kw)) == 0
+    assert field in M._lib.moe_last_error().decode()
+
+
+def test_valid_dims_workspace_grows_with_tokens():
+    a = M.moe_workspace_size(_dims(T=4))
+    b = M.moe_workspace_size(_dims(T=64))
+    assert 0 < a < b and a % 256 == 0
+
+
+FAKE = 1 << 20          # 16-byte aligned fake address; never dereferenced (validation fails first)
+
+
+def _route(dims, x=FAKE, wr=FAKE, idx=FAKE, w=FAKE, logits=None, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = M.moe_workspace_size(dims)
+    return M._lib.moe_route(ctypes.byref(dims), x, wr, idx, w, logits, ws, ws_bytes, None)
+
+
+def test_null_pointer_is_invalid_arg():
+    assert _route(_dims(), x=None) == 1
+    assert "x is NULL" in M._lib.moe_last_error().decode()
+
+
+def test_misaligned_pointer_is_alignment_error():
+    assert _route(_dims(), wr=FAKE + 8) == 3
+    assert "w_router" in M._lib.moe_last_error().decode()
+
+
+def test_small_workspace_is_rejected():
+    d = _dims()
+    assert _route(d, ws_bytes=M.moe_workspace_size(d) - 256) == 4
+
+
+def test_bad_shape_is_rejected_before_pointers():
+    assert _route(_dims(H=200), x=None) == 2
+
+
+def test_null_dims():
+    assert M._lib.moe_route(None, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None) == 1
+
+
+def test_latent_down_needs_latent_dims():
+    d = _dims()
+    st = M._lib.moe_latent_down(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE,
+                                M.moe_workspace_size(d), None)
+    assert st == 1
+
+
+def test_combine_rejects_latent_weight_without_latent_width():
+    d = _dims()
+    st = M._lib.moe_combine(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                            FAKE, FAKE, FAKE, M.moe_workspace_size(d), None)
+    assert st == 1
+
+
+def test_status_strings():
+    assert M.moe_status_string(0) == "ok"
+    assert "workspace" in M.moe_status_string(4)
+    assert M.moe_status_string(99) == "unknown status"
+
+
+def test_x_op_size_by_mode():
+    d0, d1 = _dims(act_mode=0), _dims(act_mode=1)
+    # f16 rows + row scales vs packed E2M1 + E8M0 block scales
+    assert M.moe_x_op_size(d0) >= 4 * 256 * 2 + 16
+    assert M.moe_x_op_size(d1) >= 4 * 128 + 4 * 8
+    assert M.moe_x_op_size(d1) < M.moe_x_op_size(d0)

@@ -1,0 +1,209 @@
+"""GPU parity of the CUDA path against the fp64 oracle, stage by stage.
+
+Each workload runs through the C ABI (route -> [latent_down] -> permute ->
+expert_ffn -> combine, and the fused moe_layer) and is compared with the
+oracle on the same seeded inputs:
+
+* router logits within fp32 accumulation error; expert indices bit-exact
+  except tokens the oracle flags as near-ties (|l_k - l_k+1| < 1e-5), whose
+  GPU choice must be a valid top-k inside the tie window; weights to 2e-6;
+* permutation arrays bit-exact (integer work, given the same indices);
+* activation operand exact (bf16 -> f16 with a power-of-two row scale);
+* expert outputs, shared expert and the layer output: max |err| <= 1e-2 x RMS.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mxfp4_routed_expert_04_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+from parity_harness import (TOL, GpuRun, check_permutation, check_routing, check_x_op_f16,  # noqa: E402
+                            expert_getter, max_rel_err)
+
+MEDIUM = synth.MoeWorkload("medium_ragged", T=70, H=640, I=384, E=6, k=3, I_shared=256, seed=77)
+LATENT_SMALL = synth.MoeWorkload("latent_small", T=5, H=384, I=128, E=12, k=3, I_shared=128, L=256,
+                                 seed=78)
+
+CASES = [
+    (synth.WORKLOADS["tiny"], None),
+    (MEDIUM, None),
+    (LATENT_SMALL, None),
+    (synth.WORKLOADS["latent16"], None),
+    (synth.WORKLOADS["decode1"], None),
+    (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
+]
+
+
+def _free():
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@pytest.fixture(scope="module", params=CASES, ids=lambda c: c[0].name)
+def case(request):
+    w, sample = request.param
+    run = GpuRun(w)
+    gpu = run.run_stages()
+    yield w, sample, run, gpu
+    del run
+    _free()
+
+
+def test_routing_and_permutation(case):
+    w, sample, run, gpu = case
+    ref_logits = O.router_logits(run.dense["x"], run.dense["w_router"])
+    check_routing(gpu, ref_logits, w.k)
+    check_permutation(gpu, w.E)
+
+
+def test_activation_operand(case):
+    w, sample, run, gpu = case
+    x_in = gpu["x_lat"] if w.L else run.dense["x"]
+    check_x_op_f16(gpu["x_op"], x_in, w.T, w.W)
+
+
+def test_latent_projection(case):
+    w, sample, run, gpu = case
+    if not w.L:
+        pytest.skip("not a latent layer")
+    ref = O.latent_down(run.dense["x"], run.dense["w_lat_down"])
+    a = gpu["x_lat"].astype(np.int32)
+    b = ref.astype(np.int32)
+    # both sides round to bf16; fp32 vs fp64 sums may straddle a rounding boundary
+    assert np.max(np.abs(a - b)) <= 1
+    assert np.mean(a != b) < 0.01
+
+
+def test_expert_rows(case):
+    """y_perm rows of (a sample of) the permuted (token, slot) pairs."""
+    w, sample, run, gpu = case
+    get = expert_getter(w)
+    x_in = O.bf16_to_f64(gpu["x_lat"] if w.L else run.dense["x"])
+    rows = np.arange(w.T * w.k)
+    if sample is not None:
+        rows = np.concatenate([gpu["slot_row"][t] for t in sample])
+    off = gpu["offsets"]
+    got, want = [], []
+    for r in rows:
+        e = int(np.searchsorted(off, r, side="right") - 1)
+        wg_q, wg_s, wu_q, wu_s, wd_q, wd_s = get(e)
+        y, _ = O.expert_ffn(x_in[gpu["row_token"][r]][None], O.mxfp4_dequant(wg_q, wg_s),
+                            O.mxfp4_dequant(wu_q, wu_s), O.mxfp4_dequant(wd_q, wd_s))
+        want.append(y[0])
+        got.append(gpu["y_perm"][r])
+    err, rms = max_rel_err(np.array(got), np.array(want))
+    assert err <= TOL, (err, rms)
+
+
+def test_shared_expert_alone(case):
+    w, sample, run, gpu = case
+    d = run.dense
+    ref, _ = O.shared_expert(d["x"], d["ws_gate"], d["ws_up"], d["ws_down"], d["w_sgate"])
+    if w.L:
+        pytest.skip("latent layers add the up-projection of the routed sum before the shared part")
+    got = run.shared_only()
+    err, rms = max_rel_err(got, ref)
+    assert err <= TOL, (err, rms)
+
+
+def test_layer_output(case):
+    w, sample, run, gpu = case
+    d = run.dense
+    tokens = np.arange(w.T) if sample is None else np.array(sample)
+    flagged = O.topk_route(O.router_logits(d["x"][tokens], d["w_router"]), w.k)[2]
+    sub = dict(d, x=d["x"][tokens])
+    override = gpu["idx"][tokens] if np.any(flagged) else None
+    ref = O.moe_layer(sub, w.k, expert_getter(w), idx_override=override)
+    err, rms = max_rel_err(gpu["y"][tokens], ref["y"])
+    assert err <= TOL, (err, rms)
+
+
+def test_fused_layer_matches_stages_bitwise(case):
+    w, sample, run, gpu = case
+    y = run.run_layer()
+    np.testing.assert_array_equal(y, gpu["y"])
+    y2 = run.run_layer()
+    np.testing.assert_array_equal(y2, y)
+
+
+# ---------------------------------------------------------------------------
+# edge cases on small shapes
+# ---------------------------------------------------------------------------
+
+def _small(T=6, E=8, k=3, **kw):
+    return synth.MoeWorkload("edge", T=T, H=256, I=128, E=E, k=k, I_shared=128, seed=91, **kw)
+
+
+def test_zero_input_ties_go_to_lowest_index():
+    w = _small()
+    d = synth.dense_inputs(w)
+    d["x"] = np.zeros_like(d["x"])
+    run = GpuRun(w, dense=d)
+    gpu = run.run_stages()
+    assert np.all(gpu["logits"] == 0)
+    np.testing.assert_array_equal(gpu["idx"], np.tile(np.arange(w.k), (w.T, 1)))
+    np.testing.assert_allclose(gpu["w"], 1.0 / w.k, rtol=1e-6)
+    # x = 0: every expert output and the shared expert are exactly 0
+    assert np.all(gpu["y"] == 0)
+
+
+def test_all_experts_selected():
+    w = _small(T=3, E=4, k=4)
+    run = GpuRun(w)
+    gpu = run.run_stages()
+    assert np.all(gpu["counts"] == 3)
+    ref = O.moe_layer(run.dense, w.k, expert_getter(w))
+    err, _ = max_rel_err(gpu["y"], ref["y"])
+    assert err <= TOL
+
+
+def test_single_token_single_expert():
+    w = _small(T=1, E=1, k=1)
+    run = GpuRun(w)
+    gpu = run.run_stages()
+    ref = O.moe_layer(run.dense, 1, expert_getter(w))
+    assert gpu["w"][0, 0] == 1.0
+    err, _ = max_rel_err(gpu["y"], ref["y"])
+    assert err <= TOL
+
+
+def test_nan_scale_poisons_only_its_outputs():
+    w = _small(T=4, E=2, k=1)
+    run = GpuRun(w)
+    gpu0 = run.run_stages()
+    e = int(gpu0["idx"][0, 0])
+    # E8M0 code 255 (NaN) in one scale of one gate row of expert e
+    run.dev["wg_s"][e, 5, 3] = 255
+    gpu = run.run_stages()
+    rows_e = gpu["row_token"][gpu["offsets"][e]:gpu["offsets"][e + 1]]
+    for t in range(w.T):
+        r = gpu["slot_row"][t, 0]
+        if t in rows_e:
+            assert np.all(np.isnan(gpu["y_perm"][r]))      # h[5] is NaN and feeds every output
+        else:
+            assert np.all(np.isfinite(gpu["y_perm"][r]))
+
+
+def test_invalid_expert_index_sets_status_and_empties_routing():
+    import mxfp4_routed_expert_04_b200 as M
+    w = _small(T=4, E=8, k=2)
+    run = GpuRun(w)
+    L = run.layer
+    M.moe_workspace_init(run.dims, L.ws)
+    bad = torch.tensor([[0, 1], [2, 8], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
+    M.moe_permute(run.dims, bad, run.dev["x"], L.counts, L.offsets, L.row_token, L.row_slot,
+                  L.slot_row, L.x_op, L.ws)
+    assert M.moe_device_status(L.ws) & 1
+    assert int(L.counts.sum()) == 0 and int(L.offsets.abs().sum()) == 0
+    M.moe_workspace_init(run.dims, L.ws)
+    rep = torch.tensor([[0, 1], [2, 2], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
+    M.moe_permute(run.dims, rep, run.dev["x"], L.counts, L.offsets, L.row_token, L.row_slot,
+                  L.slot_row, L.x_op, L.ws)
+    assert M.moe_device_status(L.ws) & 2
+    M.moe_workspace_init(run.dims, L.ws)
+    assert M.moe_device_status(L.ws) == 0
