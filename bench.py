@@ -224,7 +224,7 @@ def run_ours(args, w):
 
     # dominant call alone: moe_expert_ffn on the routing of the captured step
     def ffn():
-        M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.row_token, dev["wg_q"],
+        M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.expert_list, layer.row_token, dev["wg_q"],
                          dev["wg_s"], dev["wu_q"], dev["wu_s"], dev["wd_q"], dev["wd_s"],
                          layer.y_perm, layer.ws, stream)
     timed(ffn, 3)

@@ -43,9 +43,9 @@
  *   produces empty routing (all counts 0) instead of touching memory out of
  *   range. Read it with moe_device_status().
  *
- * Supported shapes: 1 <= T <= 65536; H, I, I_shared, L multiples of 64;
- * 1 <= k <= min(E, 32); 1 <= E <= 4096. act_mode MOE_ACT_MXFP4 further needs
- * W and I multiples of 128.
+ * Supported shapes: 1 <= T <= 65536; H, I, I_shared and L (when non-zero)
+ * multiples of 128 in [128, 65536]; 1 <= E <= 1024; 1 <= k <= min(E, 32);
+ * T*k <= 2^24.
  */
 #ifndef MOE_MXFP4_H
 #define MOE_MXFP4_H
@@ -70,9 +70,9 @@ typedef enum {
 
 /* How the routed experts receive their activations. */
 typedef enum {
-  /* bf16 activations. x is carried exactly (as f16 scaled by a power of two
-   * per 32-element block); h = silu(g)*u enters the down projection as f16
-   * with a power-of-two scale per 32-element block (relative rounding
+  /* bf16 activations. x is carried exactly (as f16 times one power-of-two
+   * scale per token row); h = silu(g)*u enters the down projection as f16
+   * with a power-of-two scale per group of 16 elements (relative rounding
    * <= 2^-11). Decode path: a tensor-core grouped GEMV. */
   MOE_ACT_BF16 = 0,
   /* MXFP4 activations: x rows and h are quantised to OCP MXFP4 (32-element
@@ -133,20 +133,25 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
 /* --- a3-a4: permutation ----------------------------------------------------
  * Groups the T*k (token, slot) pairs by expert: counts[e] pairs per expert,
  * offsets = exclusive prefix sum (E+1 entries), permuted rows ordered by
- * expert and, inside an expert, by ascending token. row_token[r] / row_slot[r]
+ * expert and, inside an expert, by ascending token; expert_list[0] = number
+ * of experts with at least one pair, expert_list[1..] = those experts in
+ * ascending order (the work list of the expert kernels). row_token[r] / row_slot[r]
  * give the pair at permuted row r; slot_row[t, j] the row of pair (t, j).
  * It also writes the activation operand x_op from x_in ([T, W] bf16: x, or
  * x_lat for latent layers), ONE ROW PER TOKEN; the expert kernels gather the
  * rows they need through row_token, so no duplicated [T*k, W] copy is made.
- *   x_op format, MOE_ACT_BF16: f16 values [T, W], then fp32 block scales
- *     [T, W/32] (value = f16 * scale, scale a power of two per 32 elements).
+ *   x_op format, MOE_ACT_BF16: f16 values [T, W], then (at the next 256-byte
+ *     boundary) fp32 row scales [T]: value = f16 * scale, the scale a power of
+ *     two that maps the row's largest magnitude into [2^14, 2^15).
  *   x_op format, MOE_ACT_MXFP4: codes [T, W/2] uint8 (low nibble first), then
- *     E8M0 scale codes [T, W/32] uint8 (OCP MX v1.0 conversion, ties to even).
- *   topk_idx [T, k] int32; counts [E], offsets [E+1], row_token [T*k],
- *   row_slot [T*k], slot_row [T, k] int32 (out); x_op moe_x_op_size() bytes (out)
+ *     (at the next 256-byte boundary) E8M0 scale codes [T, W/32] uint8 (OCP MX
+ *     v1.0 conversion, ties to even).
+ *   topk_idx [T, k] int32; counts [E], offsets [E+1], expert_list [E+1],
+ *   row_token [T*k], row_slot [T*k], slot_row [T, k] int32 (out);
+ *   x_op moe_x_op_size() bytes (out)
  */
 moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
-                       int32_t* counts, int32_t* offsets, int32_t* row_token,
+                       int32_t* counts, int32_t* offsets, int32_t* expert_list, int32_t* row_token,
                        int32_t* row_slot, int32_t* slot_row, void* x_op,
                        void* ws, size_t ws_bytes, void* stream);
 
@@ -156,10 +161,11 @@ moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint
  *   y_perm[r] = Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) )      [W] fp32
  * Weights in the canonical MXFP4 layout above, decoded exactly (E2M1 value x
  * E8M0 scale); products accumulate in fp32.
- *   x_op, offsets, row_token as written by moe_permute; y_perm [T*k, W] fp32 (out)
+ *   x_op, offsets, expert_list, row_token as written by moe_permute;
+ *   y_perm [T*k, W] fp32 (out)
  */
 moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t* offsets,
-                          const int32_t* row_token,
+                          const int32_t* expert_list, const int32_t* row_token,
                           const uint8_t* wg_q, const uint8_t* wg_s,
                           const uint8_t* wu_q, const uint8_t* wu_s,
                           const uint8_t* wd_q, const uint8_t* wd_s,
@@ -200,7 +206,7 @@ typedef struct {
   /* outputs and intermediates (all caller-owned) */
   int32_t* topk_idx;   /* [T, k] */
   float* topk_w;       /* [T, k] */
-  int32_t *counts, *offsets, *row_token, *row_slot, *slot_row;
+  int32_t *counts, *offsets, *expert_list, *row_token, *row_slot, *slot_row;
   uint16_t* x_lat;     /* [T, L], NULL unless L > 0 */
   void* x_op;          /* moe_x_op_size() bytes */
   float* y_perm;       /* [T*k, W] */

@@ -58,7 +58,8 @@ class MoeLayerArgs(ctypes.Structure):
     _fields_ = [(n, _P) for n in (
         "x", "w_router", "wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s", "w_sgate",
         "ws_gate", "ws_up", "ws_down", "w_lat_down", "w_lat_up", "topk_idx", "topk_w",
-        "counts", "offsets", "row_token", "row_slot", "slot_row", "x_lat", "x_op", "y_perm", "y")]
+        "counts", "offsets", "expert_list", "row_token", "row_slot", "slot_row", "x_lat", "x_op",
+        "y_perm", "y")]
 
 
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -74,8 +75,8 @@ _sigs = {
     "moe_workspace_init": [_D, _P, _Z, _P],
     "moe_device_status": [_P, ctypes.POINTER(ctypes.c_int32), _P],
     "moe_route": [_D, _P, _P, _P, _P, _P, _P, _Z, _P],
-    "moe_permute": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
-    "moe_expert_ffn": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
+    "moe_permute": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
+    "moe_expert_ffn": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_combine": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_latent_down": [_D, _P, _P, _P, _P, _Z, _P],
     "moe_layer": [_D, ctypes.POINTER(MoeLayerArgs), _P, _Z, _P],
@@ -147,18 +148,19 @@ def moe_route(dims, x, w_router, topk_idx, topk_w, logits, ws, stream=None):
                           _ptr(topk_w), _ptr(logits), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
-def moe_permute(dims, topk_idx, x_in, counts, offsets, row_token, row_slot, slot_row, x_op, ws,
-                stream=None):
+def moe_permute(dims, topk_idx, x_in, counts, offsets, expert_list, row_token, row_slot, slot_row,
+                x_op, ws, stream=None):
     _check(_lib.moe_permute(ctypes.byref(dims), _ptr(topk_idx), _ptr(x_in), _ptr(counts),
-                            _ptr(offsets), _ptr(row_token), _ptr(row_slot), _ptr(slot_row),
-                            _ptr(x_op), _ptr(ws), _nbytes(ws), _stream(stream)))
+                            _ptr(offsets), _ptr(expert_list), _ptr(row_token), _ptr(row_slot),
+                            _ptr(slot_row), _ptr(x_op), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
-def moe_expert_ffn(dims, x_op, offsets, row_token, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws,
-                   stream=None):
-    _check(_lib.moe_expert_ffn(ctypes.byref(dims), _ptr(x_op), _ptr(offsets), _ptr(row_token),
-                               _ptr(wg_q), _ptr(wg_s), _ptr(wu_q), _ptr(wu_s), _ptr(wd_q),
-                               _ptr(wd_s), _ptr(y_perm), _ptr(ws), _nbytes(ws), _stream(stream)))
+def moe_expert_ffn(dims, x_op, offsets, expert_list, row_token, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s,
+                   y_perm, ws, stream=None):
+    _check(_lib.moe_expert_ffn(ctypes.byref(dims), _ptr(x_op), _ptr(offsets), _ptr(expert_list),
+                               _ptr(row_token), _ptr(wg_q), _ptr(wg_s), _ptr(wu_q), _ptr(wu_s),
+                               _ptr(wd_q), _ptr(wd_s), _ptr(y_perm), _ptr(ws), _nbytes(ws),
+                               _stream(stream)))
 
 
 def moe_combine(dims, y_perm, slot_row, topk_w, x, w_sgate, ws_gate, ws_up, ws_down, w_lat_up, y,
@@ -210,6 +212,7 @@ class MoeLayer:
         self.logits = torch.empty(T, d.E, **f32)
         self.counts = torch.empty(d.E, **i32)
         self.offsets = torch.empty(d.E + 1, **i32)
+        self.expert_list = torch.empty(d.E + 1, **i32)
         self.row_token = torch.empty(R, **i32)
         self.row_slot = torch.empty(R, **i32)
         self.slot_row = torch.empty(T, k, **i32)
@@ -227,6 +230,7 @@ class MoeLayer:
             ws_gate=g("ws_gate"), ws_up=g("ws_up"), ws_down=g("ws_down"),
             w_lat_down=g("w_lat_down"), w_lat_up=g("w_lat_up"), topk_idx=_ptr(self.topk_idx),
             topk_w=_ptr(self.topk_w), counts=_ptr(self.counts), offsets=_ptr(self.offsets),
+            expert_list=_ptr(self.expert_list),
             row_token=_ptr(self.row_token), row_slot=_ptr(self.row_slot),
             slot_row=_ptr(self.slot_row), x_lat=_ptr(self.x_lat), x_op=_ptr(self.x_op),
             y_perm=_ptr(self.y_perm), y=_ptr(self.y))
@@ -245,9 +249,9 @@ class MoeLayer:
         if d.L:
             moe_latent_down(d, x, w["w_lat_down"], self.x_lat, self.ws, stream)
             xin = self.x_lat
-        moe_permute(d, self.topk_idx, xin, self.counts, self.offsets, self.row_token,
-                    self.row_slot, self.slot_row, self.x_op, self.ws, stream)
-        moe_expert_ffn(d, self.x_op, self.offsets, self.row_token, w["wg_q"], w["wg_s"],
+        moe_permute(d, self.topk_idx, xin, self.counts, self.offsets, self.expert_list,
+                    self.row_token, self.row_slot, self.slot_row, self.x_op, self.ws, stream)
+        moe_expert_ffn(d, self.x_op, self.offsets, self.expert_list, self.row_token, w["wg_q"], w["wg_s"],
                        w["wu_q"], w["wu_s"], w["wd_q"], w["wd_s"], self.y_perm, self.ws, stream)
         moe_combine(d, self.y_perm, self.slot_row, self.topk_w, x, w["w_sgate"], w["ws_gate"],
                     w["ws_up"], w["ws_down"], w.get("w_lat_up"), self.y, self.ws, stream)

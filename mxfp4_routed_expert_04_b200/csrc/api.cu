@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/moe_mxfp4.h"
@@ -134,6 +135,8 @@ moe_status launched(const char* what) {
 // per-device one-time setup: kernel attributes, the side stream and events of moe_layer
 struct DeviceState {
   bool ready = false;
+  int num_sms = 0;
+  int gemv_ctas_per_sm = 0;
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_lat = nullptr, ev_shared = nullptr;
 };
@@ -149,6 +152,11 @@ moe_status device_state(DeviceState** out) {
   if (!s.ready) {
     cudaError_t e = cudaFuncSetAttribute(moe::k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)moe::permute_smem_bytes(1024));
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.gemv_ctas_per_sm, moe::k_gateup_mxfp4, 32,
+                                                        moe::gemv_mxfp4_smem_bytes());
+    if (e == cudaSuccess && s.gemv_ctas_per_sm < 1) s.gemv_ctas_per_sm = 1;
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s.side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_lat, cudaEventDisableTiming);
@@ -189,10 +197,11 @@ moe_status do_route(const Plan& p, const uint16_t* x, const uint16_t* wr, int32_
 }
 
 moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, int32_t* counts,
-                      int32_t* offsets, int32_t* row_token, int32_t* row_slot, int32_t* slot_row,
-                      void* x_op, void* ws, cudaStream_t st) {
+                      int32_t* offsets, int32_t* expert_list, int32_t* row_token, int32_t* row_slot,
+                      int32_t* slot_row, void* x_op, void* ws, cudaStream_t st) {
   moe::k_permute<<<1, 1024, moe::permute_smem_bytes(p.E), st>>>(
-      idx, p.T, p.k, p.E, counts, offsets, row_token, row_slot, slot_row, at<int32_t>(ws, p.off_status));
+      idx, p.T, p.k, p.E, counts, offsets, expert_list, row_token, row_slot, slot_row,
+      at<int32_t>(ws, p.off_status));
   moe_status s = launched("permute");
   if (s != MOE_OK) return s;
   if (p.mode == MOE_ACT_BF16) {
@@ -205,30 +214,34 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
   return launched("activation operand");
 }
 
-moe_status do_expert_ffn(const Plan& p, const void* x_op, const int32_t* offsets,
+moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
+                         const int32_t* offsets, const int32_t* expert_list,
                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
                          const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
   if (p.mode != MOE_ACT_BF16)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "act_mode MOE_ACT_MXFP4 expert GEMM is not available");
-  const int ny = p.E < p.R ? p.E : p.R;
+  const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
   moe::GateUpArgs g;
   g.x16 = static_cast<const __half*>(x_op);
   g.xscale = reinterpret_cast<const float*>(static_cast<const char*>(x_op) + p.xop_scale_off);
-  g.offsets = offsets; g.row_token = row_token;
+  g.offsets = offsets; g.expert_list = expert_list; g.row_token = row_token;
   g.wg_q = wg_q; g.wg_s = wg_s; g.wu_q = wu_q; g.wu_s = wu_s;
   g.h16 = at<__half>(ws, p.off_h16);
   g.hscale = at<float>(ws, p.off_hscale);
   g.W = p.W; g.I = p.I; g.E = p.E; g.R = p.R;
   const size_t smem = moe::gemv_mxfp4_smem_bytes();
-  moe::k_gateup_mxfp4<<<dim3(p.I / 16, ny), 32, smem, st>>>(g);
+  const long slots = (long)ds.num_sms * ds.gemv_ctas_per_sm;
+  const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
+  moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
   moe_status s = launched("expert gate/up");
   if (s != MOE_OK) return s;
   moe::DownArgs d;
-  d.h16 = g.h16; d.hscale = g.hscale; d.offsets = offsets;
+  d.h16 = g.h16; d.hscale = g.hscale; d.offsets = offsets; d.expert_list = expert_list;
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
-  moe::k_down_mxfp4<<<dim3(p.W / 32, ny), 32, smem, st>>>(d);
+  const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
+  moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
   return launched("expert down");
 }
 
@@ -349,34 +362,38 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
 }
 
 moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
-                       int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* row_slot,
-                       int32_t* slot_row, void* x_op, void* ws, size_t ws_bytes, void* stream) {
+                       int32_t* counts, int32_t* offsets, int32_t* expert_list, int32_t* row_token,
+                       int32_t* row_slot, int32_t* slot_row, void* x_op, void* ws, size_t ws_bytes,
+                       void* stream) {
   Plan p;
   moe_status s = make_plan(dims, p);
   if (s != MOE_OK) return s;
   CHECK_PTR(topk_idx); CHECK_PTR(x_in); CHECK_PTR(counts); CHECK_PTR(offsets);
-  CHECK_PTR(row_token); CHECK_PTR(row_slot); CHECK_PTR(slot_row); CHECK_PTR(x_op);
+  CHECK_PTR(expert_list); CHECK_PTR(row_token); CHECK_PTR(row_slot); CHECK_PTR(slot_row); CHECK_PTR(x_op);
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
   DeviceState* ds;
   if ((s = device_state(&ds)) != MOE_OK) return s;
-  return do_permute(p, topk_idx, x_in, counts, offsets, row_token, row_slot, slot_row, x_op, ws,
-                    (cudaStream_t)stream);
+  return do_permute(p, topk_idx, x_in, counts, offsets, expert_list, row_token, row_slot, slot_row,
+                    x_op, ws, (cudaStream_t)stream);
 }
 
 moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t* offsets,
-                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
+                          const int32_t* expert_list, const int32_t* row_token,
+                          const uint8_t* wg_q, const uint8_t* wg_s,
                           const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
                           const uint8_t* wd_s, float* y_perm, void* ws, size_t ws_bytes,
                           void* stream) {
   Plan p;
   moe_status s = make_plan(dims, p);
   if (s != MOE_OK) return s;
-  CHECK_PTR(x_op); CHECK_PTR(offsets); CHECK_PTR(row_token);
+  CHECK_PTR(x_op); CHECK_PTR(offsets); CHECK_PTR(expert_list); CHECK_PTR(row_token);
   CHECK_PTR(wg_q); CHECK_PTR(wg_s); CHECK_PTR(wu_q); CHECK_PTR(wu_s); CHECK_PTR(wd_q); CHECK_PTR(wd_s);
   CHECK_PTR(y_perm);
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
-  return do_expert_ffn(p, x_op, offsets, row_token, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws,
-                       (cudaStream_t)stream);
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  return do_expert_ffn(p, *ds, x_op, offsets, expert_list, row_token, wg_q, wg_s, wu_q, wu_s, wd_q,
+                       wd_s, y_perm, ws, (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* slot_row,
@@ -418,6 +435,7 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   CHECK_PTR(a->wd_q); CHECK_PTR(a->wd_s);
   CHECK_PTR(a->w_sgate); CHECK_PTR(a->ws_gate); CHECK_PTR(a->ws_up); CHECK_PTR(a->ws_down);
   CHECK_PTR(a->topk_idx); CHECK_PTR(a->topk_w); CHECK_PTR(a->counts); CHECK_PTR(a->offsets);
+  CHECK_PTR(a->expert_list);
   CHECK_PTR(a->row_token); CHECK_PTR(a->row_slot); CHECK_PTR(a->slot_row); CHECK_PTR(a->x_op);
   CHECK_PTR(a->y_perm); CHECK_PTR(a->y);
   if (p.L) { CHECK_PTR(a->w_lat_down); CHECK_PTR(a->w_lat_up); CHECK_PTR(a->x_lat); }
@@ -443,11 +461,12 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if ((s = do_route(p, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st)) != MOE_OK) return s;
   if (p.L && (e = cudaStreamWaitEvent(st, ds->ev_lat, 0)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
-  if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets, a->row_token,
-                      a->row_slot, a->slot_row, a->x_op, ws, st)) != MOE_OK)
+  if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets,
+                      a->expert_list, a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) !=
+      MOE_OK)
     return s;
-  if ((s = do_expert_ffn(p, a->x_op, a->offsets, a->row_token, a->wg_q, a->wg_s, a->wu_q, a->wu_s,
-                         a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
+  if ((s = do_expert_ffn(p, *ds, a->x_op, a->offsets, a->expert_list, a->row_token, a->wg_q,
+                         a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
     return s;
   if ((e = cudaStreamWaitEvent(st, ds->ev_shared, 0)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));

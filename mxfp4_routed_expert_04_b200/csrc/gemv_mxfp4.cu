@@ -6,9 +6,9 @@
 // one E8M0 scale per 32 elements of a row), read once from HBM.
 //
 // Design (B200, memory-bound):
-// * one warp per CTA and per work item: a 16-row tile of one expert's
-//   matrices over the full K; grid = tiles x active experts, so a 1-token
-//   decode step spreads 1280 gate/up items over the 148 SMs;
+// * one warp per CTA; persistent CTAs walk the work items (active expert from
+//   the permutation's expert list, 16-row tile of its matrices, full K), so a
+//   1-token decode step spreads 1280 gate/up items over the 148 SMs;
 // * each warp streams its rows through a private 4-stage cp.async ring in
 //   shared memory (128 B of every row per stage = 8 scale blocks, stored with
 //   the 128-byte XOR swizzle so ldmatrix is conflict-free);
@@ -19,7 +19,8 @@
 //   fp32 MMA result;
 // * E2M1 pairs become f16x2 with one cvt.rn.f16x2.e2m1x2 each (exact);
 // * activations enter as f16: x with one power-of-two scale per token row
-//   (exact for bf16 x), h with one power-of-two scale per 16 elements.
+//   (exact for bf16 x), h with one power-of-two scale per group of 16
+//   elements that one MMA of the down projection consumes.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -34,17 +35,25 @@ constexpr int kStageWBytes = kRowsPerStage * kRowBytes;
 constexpr int kStageSBytes = kRowsPerStage * 8;    // 8 E8M0 codes per row
 constexpr int kStageBytes = kStageWBytes + kStageSBytes;
 
-// Issue the cp.async copies of one stage: rows 0..15 from (q0, s0), rows 16..31
-// from (q1, s1); `kb` = first K element of the slab, `nblk` = 4 or 8 blocks.
+// Global row (relative to the tile base) of tile-local row r (0..15). A gate/up
+// tile takes the interleaved set {8a + j : a = 0..3, j = 0..3} of its 32-row
+// block (its partner tile, based 4 rows further, takes j = 4..7): exactly the
+// K elements one mma.m16n8k16 of the down projection covers in a 32-element
+// block, so the power-of-two scale of each 16-element h group is per MMA.
+MOE_DEV int tile_row(int r, bool interleaved) { return interleaved ? 8 * (r >> 2) + (r & 3) : r; }
+
+// Issue the cp.async copies of one stage: tile rows 0..15 from (q0, s0), rows
+// 16..31 from (q1, s1); `kb` = first K element of the slab, `nblk` = 4 or 8 blocks.
 MOE_DEV void issue_stage(uint8_t* st, const uint8_t* __restrict__ q0, const uint8_t* __restrict__ s0,
                          const uint8_t* __restrict__ q1, const uint8_t* __restrict__ s1,
-                         size_t qrow, size_t srow, int kb, int nblk, int lane) {
+                         size_t qrow, size_t srow, int kb, int nblk, bool interleaved, int lane) {
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     const int idx = lane + 32 * m;
     const int row = idx >> 3, c = idx & 7;
     if (c < nblk) {
-      const uint8_t* src = (row < 16 ? q0 + row * qrow : q1 + (row - 16) * qrow) + (kb >> 1) + c * 16;
+      const int gr = tile_row(row & 15, interleaved);
+      const uint8_t* src = (row < 16 ? q0 : q1) + gr * qrow + (kb >> 1) + c * 16;
       cp_async_16(smem_u32(st + row * kRowBytes + ((c ^ (row & 7)) << 4)), src);
     }
   }
@@ -53,7 +62,8 @@ MOE_DEV void issue_stage(uint8_t* st, const uint8_t* __restrict__ q0, const uint
     const int idx = lane + 32 * m;
     const int row = idx >> 1, wd = idx & 1;
     if (wd * 4 < nblk) {
-      const uint8_t* src = (row < 16 ? s0 + row * srow : s1 + (row - 16) * srow) + (kb >> 5) + wd * 4;
+      const int gr = tile_row(row & 15, interleaved);
+      const uint8_t* src = (row < 16 ? s0 : s1) + gr * srow + (kb >> 5) + wd * 4;
       cp_async_4(smem_u32(st + kStageWBytes + row * 8 + wd * 4), src);
     }
   }
@@ -90,17 +100,22 @@ MOE_DEV void f16_block_scale(float m, float& scale, float& inv) {
 
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU
-// grid (I/16, min(E, R)), block 32, dynamic smem kStages*kStageBytes
+// persistent grid, block 32, dynamic smem kStages*kStageBytes; work item =
+// (active expert, 16-row tile), item = ai * (I/16) + tile
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
-  const int e = nth_active_expert(a.offsets, a.E, blockIdx.y, lane);
-  if (e < 0) return;
+  const int tiles = a.I >> 4;
+  const int items = __ldg(a.expert_list) * tiles;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+  const int ai = item / tiles, tile = item - ai * tiles;
+  const int e = __ldg(a.expert_list + 1 + ai);
   const int r0 = __ldg(a.offsets + e);
   const int n_all = __ldg(a.offsets + e + 1) - r0;
-  const int i0 = blockIdx.x * 16;
+  // tile q covers rows {32*(q/2) + 4*(q%2) + 8a + j : a, j = 0..3}; its h group is q
+  const int i0 = 32 * (tile >> 1) + 4 * (tile & 1);
   const size_t qrow = (size_t)a.W / 2, srow = (size_t)a.W / 32;
   const uint8_t* gq = a.wg_q + ((size_t)e * a.I + i0) * qrow;
   const uint8_t* gs = a.wg_s + ((size_t)e * a.I + i0) * srow;
@@ -127,7 +142,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
     for (int s = 0; s < kStages - 1; ++s) {
       if (s < nslab)
         issue_stage(smem + s * kStageBytes, gq, gs, uq, us, qrow, srow, s * 256,
-                    min(8, (a.W - s * 256) >> 5), lane);
+                    min(8, (a.W - s * 256) >> 5), true, lane);
       cp_async_commit();
     }
     for (int slab = 0; slab < nslab; ++slab) {
@@ -137,7 +152,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
         const int nx = slab + kStages - 1;
         if (nx < nslab)
           issue_stage(smem + (nx % kStages) * kStageBytes, gq, gs, uq, us, qrow, srow, nx * 256,
-                      min(8, (a.W - nx * 256) >> 5), lane);
+                      min(8, (a.W - nx * 256) >> 5), true, lane);
         cp_async_commit();
       }
       const uint8_t* st = smem + (slab % kStages) * kStageBytes;
@@ -217,7 +232,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
         for (int j = 0; j < 4; ++j) {
           const int col = gi * 8 + 2 * t + (j & 1);
           if (col < n) {
-            const int row = g + 8 * (j >> 1);
+            const int row = tile_row(g + 8 * (j >> 1), true);
             a.h16[(size_t)(r0 + c0 + col) * a.I + i0 + row] = __float2half_rn(h[j] * inv[j & 1]);
           }
         }
@@ -225,27 +240,32 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int col = gi * 8 + 2 * t + c;
-            if (col < n) a.hscale[(size_t)(i0 >> 4) * a.R + r0 + c0 + col] = sc[c];
+            if (col < n) a.hscale[(size_t)tile * a.R + r0 + c0 + col] = sc[c];
           }
         }
       }
     }
   }
+  }  // items
 }
 
 // ---------------------------------------------------------------------------
 // down projection
-// grid (W/32, min(E, R)), block 32, dynamic smem kStages*kStageBytes
+// persistent grid, block 32, dynamic smem kStages*kStageBytes; work item =
+// (active expert, 32-row tile of W), item = ai * (W/32) + tile
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
-  const int e = nth_active_expert(a.offsets, a.E, blockIdx.y, lane);
-  if (e < 0) return;
+  const int tiles = a.W >> 5;
+  const int items = __ldg(a.expert_list) * tiles;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+  const int ai = item / tiles, tile = item - ai * tiles;
+  const int e = __ldg(a.expert_list + 1 + ai);
   const int r0 = __ldg(a.offsets + e);
   const int n_all = __ldg(a.offsets + e + 1) - r0;
-  const int n0 = blockIdx.x * 32;
+  const int n0 = tile * 32;
   const size_t qrow = (size_t)a.I / 2, srow = (size_t)a.I / 32;
   const uint8_t* dq = a.wd_q + ((size_t)e * a.W + n0) * qrow;
   const uint8_t* ds = a.wd_s + ((size_t)e * a.W + n0) * srow;
@@ -272,7 +292,7 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
     for (int s = 0; s < kStages - 1; ++s) {
       if (s < nslab)
         issue_stage(smem + s * kStageBytes, dq, ds, dq + 16 * qrow, ds + 16 * srow, qrow, srow,
-                    s * 256, min(8, (a.I - s * 256) >> 5), lane);
+                    s * 256, min(8, (a.I - s * 256) >> 5), false, lane);
       cp_async_commit();
     }
     for (int slab = 0; slab < nslab; ++slab) {
@@ -282,7 +302,7 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
         const int nx = slab + kStages - 1;
         if (nx < nslab)
           issue_stage(smem + (nx % kStages) * kStageBytes, dq, ds, dq + 16 * qrow, ds + 16 * srow,
-                      qrow, srow, nx * 256, min(8, (a.I - nx * 256) >> 5), lane);
+                      qrow, srow, nx * 256, min(8, (a.I - nx * 256) >> 5), false, lane);
         cp_async_commit();
       }
       const uint8_t* st = smem + (slab % kStages) * kStageBytes;
@@ -306,7 +326,7 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
             ws[0][1] = e8m0_to_f32(ss[(g + 8) * 8 + b]);
             ws[1][0] = e8m0_to_f32(ss[(g + 16) * 8 + b]);
             ws[1][1] = e8m0_to_f32(ss[(g + 24) * 8 + b]);
-            const int hb16 = (kb >> 4) + 2 * b;     // 16-element h block of the first k half
+            const int hb16 = 2 * ((kb >> 5) + b);   // h group of the first MMA of this block
 #pragma unroll
             for (int gi = 0; gi < 4; ++gi) {
               if (gi < ng) {
@@ -355,6 +375,7 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
       }
     }
   }
+  }  // items
 }
 
 size_t gemv_mxfp4_smem_bytes() { return (size_t)kStages * kStageBytes; }

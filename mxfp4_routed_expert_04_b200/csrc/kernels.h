@@ -13,6 +13,7 @@ struct GateUpArgs {
   const __half* x16;         // [T, W] f16 activation rows (one per token)
   const float* xscale;       // [T] power-of-two row scales
   const int32_t* offsets;    // [E+1]
+  const int32_t* expert_list;  // [E+1]: count, then active experts
   const int32_t* row_token;  // [R]
   const uint8_t *wg_q, *wg_s, *wu_q, *wu_s;
   __half* h16;               // [R, I]
@@ -24,6 +25,7 @@ struct DownArgs {
   const __half* h16;
   const float* hscale;
   const int32_t* offsets;
+  const int32_t* expert_list;
   const uint8_t *wd_q, *wd_s;
   float* y_perm;             // [R, W]
   int W, I, E, R;
@@ -52,8 +54,8 @@ __global__ void k_topk(const float* part, int S, int T, int E, int k, int32_t* i
 
 // --- permutation and activation operands ------------------------------------
 __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
-                          int32_t* offsets, int32_t* row_token, int32_t* row_slot,
-                          int32_t* slot_row, int32_t* status);
+                          int32_t* offsets, int32_t* expert_list, int32_t* row_token,
+                          int32_t* row_slot, int32_t* slot_row, int32_t* status);
 size_t permute_smem_bytes(int E);
 __global__ void k_act_to_f16(const uint16_t* x, int W, __half* x16, float* xscale);
 __global__ void k_act_to_mxfp4(const uint16_t* x, int W, uint8_t* q, uint8_t* s);

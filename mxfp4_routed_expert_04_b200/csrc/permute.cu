@@ -32,6 +32,7 @@ size_t permute_smem_bytes(int E) {
 __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restrict__ idx, int T, int k,
                                                         int E, int32_t* __restrict__ counts,
                                                         int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ expert_list,
                                                         int32_t* __restrict__ row_token,
                                                         int32_t* __restrict__ row_slot,
                                                         int32_t* __restrict__ slot_row,
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
   if (bad) {
     for (int e = tid; e < E; e += kPermThreads) counts[e] = 0;
     for (int e = tid; e <= E; e += kPermThreads) offsets[e] = 0;
+    if (tid == 0) expert_list[0] = 0;
     if (tid == 0) atomicOr(status, bad);
     return;
   }
@@ -98,6 +100,15 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
       cnt[e] = excl;         // cursor
     }
     if (e == E - 1) offsets[E] = excl + c;
+    // compact list of the experts that received pairs, ascending
+    const unsigned act = __ballot_sync(0xFFFFFFFFu, c > 0);
+    __syncthreads();
+    if (lane == 0) wsum[warp] = __popc(act);
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (c > 0) expert_list[1 + before + __popc(act & ((1u << lane) - 1u))] = e;
+    if (tid == kPermThreads - 1) expert_list[0] = before + __popc(act);
   }
   __syncthreads();
 

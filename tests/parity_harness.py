@@ -35,6 +35,7 @@ class GpuRun:
             logits=L.logits.cpu().numpy().astype(np.float64),
             idx=L.topk_idx.cpu().numpy(), w=L.topk_w.cpu().numpy().astype(np.float64),
             counts=L.counts.cpu().numpy(), offsets=L.offsets.cpu().numpy(),
+            expert_list=L.expert_list.cpu().numpy(),
             row_token=L.row_token.cpu().numpy(), row_slot=L.row_slot.cpu().numpy(),
             slot_row=L.slot_row.cpu().numpy(), y_perm=L.y_perm.cpu().numpy().astype(np.float64),
             y=y.cpu().numpy().astype(np.float64), x_op=L.x_op.cpu().numpy())
@@ -100,6 +101,9 @@ def check_permutation(gpu, E):
     np.testing.assert_array_equal(gpu["row_token"], row_token)
     np.testing.assert_array_equal(gpu["row_slot"], row_slot)
     np.testing.assert_array_equal(gpu["slot_row"], slot_row)
+    active = np.nonzero(counts)[0]
+    assert gpu["expert_list"][0] == len(active)
+    np.testing.assert_array_equal(gpu["expert_list"][1:1 + len(active)], active)
 
 
 def check_x_op_f16(x_op, x_bits, T, W):

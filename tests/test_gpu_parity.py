@@ -196,14 +196,15 @@ def test_invalid_expert_index_sets_status_and_empties_routing():
     L = run.layer
     M.moe_workspace_init(run.dims, L.ws)
     bad = torch.tensor([[0, 1], [2, 8], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
-    M.moe_permute(run.dims, bad, run.dev["x"], L.counts, L.offsets, L.row_token, L.row_slot,
-                  L.slot_row, L.x_op, L.ws)
+    M.moe_permute(run.dims, bad, run.dev["x"], L.counts, L.offsets, L.expert_list, L.row_token,
+                  L.row_slot, L.slot_row, L.x_op, L.ws)
     assert M.moe_device_status(L.ws) & 1
     assert int(L.counts.sum()) == 0 and int(L.offsets.abs().sum()) == 0
+    assert int(L.expert_list[0]) == 0
     M.moe_workspace_init(run.dims, L.ws)
     rep = torch.tensor([[0, 1], [2, 2], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
-    M.moe_permute(run.dims, rep, run.dev["x"], L.counts, L.offsets, L.row_token, L.row_slot,
-                  L.slot_row, L.x_op, L.ws)
+    M.moe_permute(run.dims, rep, run.dev["x"], L.counts, L.offsets, L.expert_list, L.row_token,
+                  L.row_slot, L.slot_row, L.x_op, L.ws)
     assert M.moe_device_status(L.ws) & 2
     M.moe_workspace_init(run.dims, L.ws)
     assert M.moe_device_status(L.ws) == 0
