@@ -29,17 +29,18 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Number of K splits of a dense GEMV: enough warps to cover the GPU, each split
-// a whole number of 32-element steps and at least 4 of them.
+// Number of K splits of a dense GEMV: enough warps to cover the GPU (about 4
+// per SM), each split a whole number of 32-element steps and at least 8 of
+// them, at most 16 splits.
 int dense_splits(int N, int T, int K) {
   const long warps = (long)((N + 15) / 16) * ((T + 31) / 32);
   const int ksteps = K / 32;
   int S = 1;
-  for (int c = 1; c <= ksteps; ++c) {
+  for (int c = 1; c <= ksteps && c <= 16; ++c) {
     if (ksteps % c) continue;
-    if (ksteps / c < 4) break;
+    if (ksteps / c < 8) break;
     S = c;
-    if (warps * c >= (long)kNumSMs * 8) break;
+    if (warps * c >= (long)kNumSMs * 4) break;
   }
   return S;
 }
@@ -192,7 +193,7 @@ moe_status do_route(const Plan& p, const uint16_t* x, const uint16_t* wr, int32_
   moe_status s = launch_dense(wr, p.E, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H,
                               p.S_router, st, "router gemv");
   if (s != MOE_OK) return s;
-  moe::k_topk<<<(p.T + 7) / 8, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
+  moe::k_topk<<<p.T, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
   return launched("top-k");
 }
 
@@ -214,6 +215,46 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
   return launched("activation operand");
 }
 
+// threads of a CUDA-core GEMV CTA for K elements: every thread owns BPT
+// 32-element blocks (BPT = 2 from 64 blocks up), rounded up to whole warps.
+int fma_bpt(int K) { return (K / 32) >= 64 ? 2 : 1; }
+int fma_threads(int K) {
+  const int kb = K / 32, bpt = fma_bpt(K);
+  const int t = (kb + bpt - 1) / bpt;
+  return (t + 31) / 32 * 32;
+}
+// the CUDA-core path serves single-token experts when both K fit one CTA
+bool fma_path(const Plan& p) {
+  return fma_threads(p.W) <= moe::kFmaMaxThreads && fma_threads(p.I) <= moe::kFmaMaxThreads;
+}
+
+template <typename Kern, typename Args>
+moe_status launch_persistent(const DeviceState& ds, Kern kern, const Args& args, int threads,
+                             long max_items, cudaStream_t st, const char* what) {
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s occupancy: %s", what, cudaGetErrorString(e));
+  const long grid = std::max<long>(1, std::min<long>(max_items, (long)ds.num_sms * std::max(1, per_sm)));
+  kern<<<(int)grid, threads, 0, st>>>(args);
+  return launched(what);
+}
+
+moe_status launch_fma_gateup(const DeviceState& ds, const moe::GateUpArgs& g, long max_items,
+                             cudaStream_t st) {
+  const int thr = fma_threads(g.W);
+  if (fma_bpt(g.W) == 2)
+    return launch_persistent(ds, moe::k_gateup_fma<2>, g, thr, max_items, st, "expert gate/up (fma)");
+  return launch_persistent(ds, moe::k_gateup_fma<1>, g, thr, max_items, st, "expert gate/up (fma)");
+}
+
+moe_status launch_fma_down(const DeviceState& ds, const moe::DownArgs& d, long max_items,
+                           cudaStream_t st) {
+  const int thr = fma_threads(d.I);
+  if (fma_bpt(d.I) == 2)
+    return launch_persistent(ds, moe::k_down_fma<2>, d, thr, max_items, st, "expert down (fma)");
+  return launch_persistent(ds, moe::k_down_fma<1>, d, thr, max_items, st, "expert down (fma)");
+}
+
 moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const int32_t* offsets, const int32_t* expert_list,
                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
@@ -232,14 +273,21 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   g.W = p.W; g.I = p.I; g.E = p.E; g.R = p.R;
   const size_t smem = moe::gemv_mxfp4_smem_bytes();
   const long slots = (long)ds.num_sms * ds.gemv_ctas_per_sm;
+  // single-token experts on the CUDA cores
+  const bool fma = fma_path(p);
+  g.min_tokens = fma ? 2 : 1;
+  moe_status s = MOE_OK;
+  if (fma && (s = launch_fma_gateup(ds, g, ny * (p.I / 16), st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
   moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
-  moe_status s = launched("expert gate/up");
+  s = launched("expert gate/up");
   if (s != MOE_OK) return s;
   moe::DownArgs d;
   d.h16 = g.h16; d.hscale = g.hscale; d.offsets = offsets; d.expert_list = expert_list;
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
+  d.min_tokens = g.min_tokens;
+  if (fma && (s = launch_fma_down(ds, d, ny * (p.W / 32), st)) != MOE_OK) return s;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
   return launched("expert down");

@@ -138,3 +138,62 @@ MOE_DEV int nth_active_expert(const int32_t* __restrict__ offsets, int E, int a,
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// acc + a * b with f16 a, b (the two halves of the f16x2 words wa, wb) and an
+// fp32 accumulator; the product of two f16 values is exact in fp32.
+MOE_DEV float fma_f16lo(uint32_t wa, uint32_t wb, float acc) {
+  float d;
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}"
+      : "=f"(d) : "r"(wa), "r"(wb), "f"(acc));
+  return d;
+}
+MOE_DEV float fma_f16hi(uint32_t wa, uint32_t wb, float acc) {
+  float d;
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a1, b1, %3;\n\t}"
+      : "=f"(d) : "r"(wa), "r"(wb), "f"(acc));
+  return d;
+}
+
+// Dot product of one 32-element MXFP4 block (16 packed bytes) with 32 f16
+// activations (16 f16x2 words), fp32 accumulation, block scale not applied.
+MOE_DEV float dot_block_e2m1_f16(uint4 w, const uint32_t (&x)[16]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t h[4];
+    e2m1x8_to_f16x8(words[q], h);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a0 = fma_f16lo(h[j], x[4 * q + j], a0);
+      a1 = fma_f16hi(h[j], x[4 * q + j], a1);
+    }
+  }
+  return a0 + a1;
+}
+
+// Warp reduce-scatter of 32 values per lane: afterwards lane l holds the sum
+// over the warp of v[l] (v[0] on return).
+MOE_DEV float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+    }
+  }
+  return v[0];
+}
+
+}  // namespace moe

@@ -1,4 +1,5 @@
-// Grouped MXFP4 GEMV for the routed experts (decode: a few tokens per expert).
+// Grouped MXFP4 GEMV for the routed experts that received 2 or more tokens
+// (decode batches); single-token experts take the CUDA-core path (gemv_fma.cu).
 //
 // The "expert matmul" of the rabbit README phase breakdown: for every active
 // expert e and its n_e tokens, gate/up projections with a fused SwiGLU
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
   const int e = __ldg(a.expert_list + 1 + ai);
   const int r0 = __ldg(a.offsets + e);
   const int n_all = __ldg(a.offsets + e + 1) - r0;
+  if (n_all < a.min_tokens) continue;          // single-token experts: CUDA-core path
   // tile q covers rows {32*(q/2) + 4*(q%2) + 8a + j : a, j = 0..3}; its h group is q
   const int i0 = 32 * (tile >> 1) + 4 * (tile & 1);
   const size_t qrow = (size_t)a.W / 2, srow = (size_t)a.W / 32;
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
   const int e = __ldg(a.expert_list + 1 + ai);
   const int r0 = __ldg(a.offsets + e);
   const int n_all = __ldg(a.offsets + e + 1) - r0;
+  if (n_all < a.min_tokens) continue;          // single-token experts: CUDA-core path
   const int n0 = tile * 32;
   const size_t qrow = (size_t)a.I / 2, srow = (size_t)a.I / 32;
   const uint8_t* dq = a.wd_q + ((size_t)e * a.W + n0) * qrow;

@@ -19,6 +19,7 @@ struct GateUpArgs {
   __half* h16;               // [R, I]
   float* hscale;             // [I/16, R]
   int W, I, E, R;
+  int min_tokens;            // experts with fewer tokens are left to the CUDA-core path
 };
 
 struct DownArgs {
@@ -29,11 +30,18 @@ struct DownArgs {
   const uint8_t *wd_q, *wd_s;
   float* y_perm;             // [R, W]
   int W, I, E, R;
+  int min_tokens;
 };
 
+// tensor-core path: experts with >= 2 tokens
 __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
+// CUDA-core path: experts with exactly 1 token; BPT = K blocks per thread,
+// at most kFmaMaxThreads threads (K <= kFmaMaxThreads * 2 * 32)
+constexpr int kFmaMaxThreads = 256;
+template <int BPT> __global__ void k_gateup_fma(GateUpArgs a);
+template <int BPT> __global__ void k_down_fma(DownArgs a);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {

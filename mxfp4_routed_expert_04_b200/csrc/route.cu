@@ -1,7 +1,7 @@
 // Router tail: softmax top-k with renormalised weights (rabbit README, model
 // table row "MoE routing": softmax top-10 of 512).
 //
-// One warp per token. The router logits arrive as split-K partial sums
+// One CTA per token. The router logits arrive as split-K partial sums
 // [S, T, E] from k_dense_gemv and are summed in a fixed order (s = 0..S-1),
 // so the logits, and with them the selection, are reproducible run to run.
 // Selection ranks by fp32 logit (the softmax is monotone); equal logits go to
@@ -16,29 +16,39 @@ namespace moe {
 
 constexpr int kMaxPerLane = 32;   // E <= 1024
 
-// grid ceil(T/8), block 256 (8 warps, one token each)
+// grid T, block 256: the CTA sums the S partial logits of its token (all
+// threads, independent loads), then warp 0 selects the top k.
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, int S, int T, int E,
                                               int k, int32_t* __restrict__ idx,
                                               float* __restrict__ w, float* __restrict__ logits) {
-  const int lane = threadIdx.x & 31;
-  const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (tok >= T) return;
+  __shared__ float lg[1024];
+  const int tok = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += 256) {
+    const float* p = part + (size_t)tok * E + e;
+    const size_t stride = (size_t)T * E;
+    float acc = 0.0f;
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {                // fixed summation order s = 0, 1, 2, ...
+      const float v0 = __ldg(p + (s + 0) * stride), v1 = __ldg(p + (s + 1) * stride);
+      const float v2 = __ldg(p + (s + 2) * stride), v3 = __ldg(p + (s + 3) * stride);
+      acc += v0; acc += v1; acc += v2; acc += v3;
+    }
+    for (; s < S; ++s) acc += __ldg(p + s * stride);
+    if (logits) logits[(size_t)tok * E + e] = acc;
+    lg[e] = isnan(acc) ? -INFINITY : acc;      // a NaN logit never wins
+  }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
   float v[kMaxPerLane];
 #pragma unroll
   for (int j = 0; j < kMaxPerLane; ++j) {
     const int e = lane + 32 * j;
-    float acc = -INFINITY;
-    if (e < E) {
-      acc = 0.0f;
-      for (int s = 0; s < S; ++s) acc += __ldg(part + ((size_t)s * T + tok) * E + e);
-      if (logits) logits[(size_t)tok * E + e] = acc;
-      if (isnan(acc)) acc = -INFINITY;      // a NaN logit never wins
-    }
-    v[j] = acc;
+    v[j] = (e < E) ? lg[e] : -INFINITY;
   }
   uint32_t taken = 0;
-  float selv[32];
-  int sele[32];
+  float selv = 0.0f;     // lane r keeps the r-th selection
+  int sele = 0;
   for (int r = 0; r < k; ++r) {
     float bv = -INFINITY;
     int be = 0x7FFFFFFF;
@@ -56,17 +66,16 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, in
       if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
     }
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    selv[r] = bv;
-    sele[r] = be;
+    if (lane == r) { selv = bv; sele = be; }
   }
-  if (lane == 0) {
-    const float m = selv[0];
-    float den = 0.0f;
-    for (int r = 0; r < k; ++r) den += expf(selv[r] - m);
-    for (int r = 0; r < k; ++r) {
-      idx[(size_t)tok * k + r] = sele[r];
-      w[(size_t)tok * k + r] = expf(selv[r] - m) / den;
-    }
+  const float m = __shfl_sync(0xFFFFFFFFu, selv, 0);
+  const float ex = (lane < k) ? expf(selv - m) : 0.0f;
+  float den = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, off);
+  if (lane < k) {
+    idx[(size_t)tok * k + lane] = sele;
+    w[(size_t)tok * k + lane] = ex / den;
   }
 }
 
