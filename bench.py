@@ -179,7 +179,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     n_active = int((layer.counts > 0).sum())
 
-    launches_per_step = 10 + (3 if w.L else 0)
+    launches_per_step = 12 + (4 if w.L else 0)   # kernels enqueued by one moe_layer call
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

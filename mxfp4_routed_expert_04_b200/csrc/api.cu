@@ -215,44 +215,52 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
   return launched("activation operand");
 }
 
-// threads of a CUDA-core GEMV CTA for K elements: every thread owns BPT
-// 32-element blocks (BPT = 2 from 64 blocks up), rounded up to whole warps.
-int fma_bpt(int K) { return (K / 32) >= 64 ? 2 : 1; }
-int fma_threads(int K) {
-  const int kb = K / 32, bpt = fma_bpt(K);
-  const int t = (kb + bpt - 1) / bpt;
-  return (t + 31) / 32 * 32;
+// CUDA-core GEMV geometry for a reduction length K: every thread owns BPT
+// 32-element blocks (BPT = 2 from 256 blocks up), rounded up to whole warps;
+// a ring stage holds RPS rows (a power of two <= 16, about 8 KB of codes,
+// with the stage's E8M0 bytes a multiple of 16 for the bulk copy).
+struct FmaGeom {
+  int bpt = 0, threads = 0, rps = 0;
+  bool ok = false;
+};
+FmaGeom fma_geom(int K) {
+  FmaGeom g;
+  const int kb = K / 32;
+  g.bpt = kb >= 256 ? 2 : 1;
+  g.threads = ((kb + g.bpt - 1) / g.bpt + 31) / 32 * 32;
+  const int qrow = K / 2, srow = K / 32;
+  for (int r = 1; r <= 16; r *= 2) {
+    if ((r * srow) % 16 != 0) continue;
+    g.rps = r;
+    if ((long)r * qrow >= 8192) break;
+  }
+  g.ok = g.rps > 0 && g.threads <= moe::kFmaMaxThreads &&
+         moe::fma_smem_bytes(K, g.rps) <= 160 * 1024;
+  return g;
 }
-// the CUDA-core path serves single-token experts when both K fit one CTA
-bool fma_path(const Plan& p) {
-  return fma_threads(p.W) <= moe::kFmaMaxThreads && fma_threads(p.I) <= moe::kFmaMaxThreads;
-}
+// the CUDA-core path serves single-token experts when both projections fit it
+bool fma_path(const Plan& p) { return fma_geom(p.W).ok && fma_geom(p.I).ok; }
 
-template <typename Kern, typename Args>
-moe_status launch_persistent(const DeviceState& ds, Kern kern, const Args& args, int threads,
-                             long max_items, cudaStream_t st, const char* what) {
+template <bool kGateUp>
+moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, int K, long max_items,
+                      cudaStream_t st) {
+  const FmaGeom g = fma_geom(K);
+  const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
+  void (*kern)(moe::FmaArgs) = nullptr;
+#define MOE_PICK(B, R) if (g.bpt == B && g.rps == R) kern = moe::k_fma_gemv<B, R, kGateUp>;
+  MOE_PICK(1, 1) MOE_PICK(1, 2) MOE_PICK(1, 4) MOE_PICK(1, 8) MOE_PICK(1, 16)
+  MOE_PICK(2, 1) MOE_PICK(2, 2) MOE_PICK(2, 4) MOE_PICK(2, 8) MOE_PICK(2, 16)
+#undef MOE_PICK
+  if (!kern) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
+  const size_t smem = moe::fma_smem_bytes(K, g.rps);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
-  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s occupancy: %s", what, cudaGetErrorString(e));
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, smem);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
   const long grid = std::max<long>(1, std::min<long>(max_items, (long)ds.num_sms * std::max(1, per_sm)));
-  kern<<<(int)grid, threads, 0, st>>>(args);
+  kern<<<(int)grid, g.threads, smem, st>>>(a);
   return launched(what);
-}
-
-moe_status launch_fma_gateup(const DeviceState& ds, const moe::GateUpArgs& g, long max_items,
-                             cudaStream_t st) {
-  const int thr = fma_threads(g.W);
-  if (fma_bpt(g.W) == 2)
-    return launch_persistent(ds, moe::k_gateup_fma<2>, g, thr, max_items, st, "expert gate/up (fma)");
-  return launch_persistent(ds, moe::k_gateup_fma<1>, g, thr, max_items, st, "expert gate/up (fma)");
-}
-
-moe_status launch_fma_down(const DeviceState& ds, const moe::DownArgs& d, long max_items,
-                           cudaStream_t st) {
-  const int thr = fma_threads(d.I);
-  if (fma_bpt(d.I) == 2)
-    return launch_persistent(ds, moe::k_down_fma<2>, d, thr, max_items, st, "expert down (fma)");
-  return launch_persistent(ds, moe::k_down_fma<1>, d, thr, max_items, st, "expert down (fma)");
 }
 
 moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
@@ -275,9 +283,16 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   const long slots = (long)ds.num_sms * ds.gemv_ctas_per_sm;
   // single-token experts on the CUDA cores
   const bool fma = fma_path(p);
+  moe::FmaArgs f;
+  f.x16 = g.x16; f.xscale = g.xscale; f.h16 = g.h16; f.hscale = g.hscale;
+  f.offsets = offsets; f.expert_list = expert_list; f.row_token = row_token;
+  f.wg_q = wg_q; f.wg_s = wg_s; f.wu_q = wu_q; f.wu_s = wu_s; f.wd_q = wd_q; f.wd_s = wd_s;
+  f.h16_out = g.h16; f.hscale_out = g.hscale; f.y_perm = y_perm;
+  f.status = at<int32_t>(ws, p.off_status);
+  f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
   g.min_tokens = fma ? 2 : 1;
   moe_status s = MOE_OK;
-  if (fma && (s = launch_fma_gateup(ds, g, ny * (p.I / 16), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<true>(ds, f, p.W, ny * (p.I / 16), st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
   moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
   s = launched("expert gate/up");
@@ -287,7 +302,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
   d.min_tokens = g.min_tokens;
-  if (fma && (s = launch_fma_down(ds, d, ny * (p.W / 32), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<false>(ds, f, p.I, ny * (p.W / 32), st)) != MOE_OK) return s;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
   return launched("expert down");

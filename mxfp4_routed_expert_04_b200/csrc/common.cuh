@@ -197,3 +197,46 @@ MOE_DEV float warp_reduce_scatter32(float (&v)[32], int lane) {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk-copy (TMA, non-tensor) helpers
+// ---------------------------------------------------------------------------
+enum : int32_t { kStatusWaitTimeout = 4 };   // a bounded device wait gave up
+
+MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+MOE_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::); }
+MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::); }
+
+MOE_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;\n"
+               ::"r"(smem_u32(bar)), "r"(bytes));
+}
+
+// Bounded wait for phase `parity` of `bar`: false when it did not complete
+// within the iteration limit (the caller reports it and leaves).
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t it = 0; it < (1u << 26); ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(a), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// Bulk global -> shared copy completing on `bar` (16-byte aligned, bytes % 16 == 0).
+MOE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+}  // namespace moe

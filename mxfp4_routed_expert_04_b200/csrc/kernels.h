@@ -38,10 +38,30 @@ __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
 // CUDA-core path: experts with exactly 1 token; BPT = K blocks per thread,
-// at most kFmaMaxThreads threads (K <= kFmaMaxThreads * 2 * 32)
+// RPS = weight rows per ring stage; at most kFmaMaxThreads threads
 constexpr int kFmaMaxThreads = 256;
-template <int BPT> __global__ void k_gateup_fma(GateUpArgs a);
-template <int BPT> __global__ void k_down_fma(DownArgs a);
+struct FmaArgs {
+  // activations
+  const __half* x16;         // gate/up: [T, W] f16 rows, xscale [T]
+  const float* xscale;
+  const __half* h16;         // down: [R, I] f16 rows, hscale [I/16, R]
+  const float* hscale;
+  // routing
+  const int32_t* offsets;
+  const int32_t* expert_list;
+  const int32_t* row_token;
+  // weights
+  const uint8_t *wg_q, *wg_s, *wu_q, *wu_s, *wd_q, *wd_s;
+  // outputs
+  __half* h16_out;           // gate/up writes h here (same buffer as h16)
+  float* hscale_out;
+  float* y_perm;             // down: [R, W]
+  int32_t* status;           // device status word
+  int W, I, E, R;
+};
+template <int BPT, int RPS, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a);
+size_t fma_stage_bytes(int K, int rps);
+size_t fma_smem_bytes(int K, int rps);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {
