@@ -91,7 +91,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_status = take(256);
   p.off_router = take((size_t)p.S_router * p.T * p.E * 4);
   p.off_h16 = take((size_t)p.R * p.I * 2);
-  p.off_hscale = take((size_t)(p.I / 16) * p.R * 4);
+  p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
   p.off_sgu = take((size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
   p.off_hs = take((size_t)p.T * p.Is * 4);
   p.off_gl = take((size_t)p.T * 4);
@@ -215,51 +215,44 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
   return launched("activation operand");
 }
 
-// CUDA-core GEMV geometry for a reduction length K: every thread owns BPT
-// 32-element blocks (BPT = 2 from 256 blocks up), rounded up to whole warps;
-// a ring stage holds RPS rows (a power of two <= 16, about 8 KB of codes,
-// with the stage's E8M0 bytes a multiple of 16 for the bulk copy).
-struct FmaGeom {
-  int bpt = 0, threads = 0, rps = 0;
-  bool ok = false;
+// CUDA-core GEMV launch shape for reduction length K: 256 consumer threads
+// (64 for K < 2048), one 32-element block per thread per row (2 beyond 8192),
+// shared memory for two CTAs per SM (four with 64 consumer threads).
+struct FmaPlan {
+  int nt = 0, bpt = 0;
+  moe::FmaGeometry g{};
 };
-FmaGeom fma_geom(int K) {
-  FmaGeom g;
+FmaPlan fma_plan(int K, bool gate_up) {
+  FmaPlan f;
   const int kb = K / 32;
-  g.bpt = kb >= 256 ? 2 : 1;
-  g.threads = ((kb + g.bpt - 1) / g.bpt + 31) / 32 * 32;
-  const int qrow = K / 2, srow = K / 32;
-  for (int r = 1; r <= 16; r *= 2) {
-    if ((r * srow) % 16 != 0) continue;
-    g.rps = r;
-    if ((long)r * qrow >= 8192) break;
-  }
-  g.ok = g.rps > 0 && g.threads <= moe::kFmaMaxThreads &&
-         moe::fma_smem_bytes(K, g.rps) <= 160 * 1024;
-  return g;
+  f.nt = kb >= 64 ? 256 : 64;
+  f.bpt = kb > 256 ? 2 : 1;
+  if (kb > 512) return f;                      // g.ok == 0: tensor-core path only
+  f.g = moe::fma_geometry(K, gate_up, f.nt, f.bpt, (f.nt == 256 ? 110 : 54) * 1024);
+  return f;
 }
 // the CUDA-core path serves single-token experts when both projections fit it
-bool fma_path(const Plan& p) { return fma_geom(p.W).ok && fma_geom(p.I).ok; }
+bool fma_path(const Plan& p) { return fma_plan(p.W, true).g.ok && fma_plan(p.I, false).g.ok; }
 
 template <bool kGateUp>
-moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, int K, long max_items,
-                      cudaStream_t st) {
-  const FmaGeom g = fma_geom(K);
+moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, long max_items, cudaStream_t st) {
+  const int K = kGateUp ? a.W : a.I;
+  const FmaPlan f = fma_plan(K, kGateUp);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
-  void (*kern)(moe::FmaArgs) = nullptr;
-#define MOE_PICK(B, R) if (g.bpt == B && g.rps == R) kern = moe::k_fma_gemv<B, R, kGateUp>;
-  MOE_PICK(1, 1) MOE_PICK(1, 2) MOE_PICK(1, 4) MOE_PICK(1, 8) MOE_PICK(1, 16)
-  MOE_PICK(2, 1) MOE_PICK(2, 2) MOE_PICK(2, 4) MOE_PICK(2, 8) MOE_PICK(2, 16)
-#undef MOE_PICK
-  if (!kern) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
-  const size_t smem = moe::fma_smem_bytes(K, g.rps);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
+  if (f.nt == 64 && f.bpt == 1) kern = moe::k_fma_gemv<64, 1, kGateUp>;
+  if (f.nt == 256 && f.bpt == 1) kern = moe::k_fma_gemv<256, 1, kGateUp>;
+  if (f.nt == 256 && f.bpt == 2) kern = moe::k_fma_gemv<256, 2, kGateUp>;
+  if (!kern || !f.g.ok) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
+  const int threads = f.nt + 32;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)f.g.smem_bytes);
   int per_sm = 0;
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.threads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, f.g.smem_bytes);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
   const long grid = std::max<long>(1, std::min<long>(max_items, (long)ds.num_sms * std::max(1, per_sm)));
-  kern<<<(int)grid, g.threads, smem, st>>>(a);
+  kern<<<(int)grid, threads, f.g.smem_bytes, st>>>(a, f.g);
   return launched(what);
 }
 
@@ -292,7 +285,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
   g.min_tokens = fma ? 2 : 1;
   moe_status s = MOE_OK;
-  if (fma && (s = launch_fma<true>(ds, f, p.W, ny * (p.I / 16), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<true>(ds, f, ny * (p.I / 16), st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
   moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
   s = launched("expert gate/up");
@@ -302,7 +295,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
   d.min_tokens = g.min_tokens;
-  if (fma && (s = launch_fma<false>(ds, f, p.I, ny * (p.W / 32), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<false>(ds, f, ny * (p.W / 32), st)) != MOE_OK) return s;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
   return launched("expert down");

@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int col = gi * 8 + 2 * t + c;
-            if (col < n) a.hscale[(size_t)tile * a.R + r0 + c0 + col] = sc[c];
+            if (col < n) a.hscale[(size_t)(r0 + c0 + col) * (a.I >> 4) + tile] = sc[c];
           }
         }
       }
@@ -339,8 +339,9 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
                 for (int c = 0; c < 2; ++c) {
                   const int col = gi * 8 + 2 * t + c;
                   const bool ok = col < n;
-                  hs0[c] = ok ? __ldg(a.hscale + (size_t)hb16 * a.R + r0 + c0 + col) : 0.0f;
-                  hs1[c] = ok ? __ldg(a.hscale + (size_t)(hb16 + 1) * a.R + r0 + c0 + col) : 0.0f;
+                  const float* hsr = a.hscale + (size_t)(r0 + c0 + col) * (a.I >> 4) + hb16;
+                  hs0[c] = ok ? __ldg(hsr) : 0.0f;
+                  hs1[c] = ok ? __ldg(hsr + 1) : 0.0f;
                 }
                 float c00[4] = {0.f, 0.f, 0.f, 0.f}, c01[4] = {0.f, 0.f, 0.f, 0.f};
                 float c10[4] = {0.f, 0.f, 0.f, 0.f}, c11[4] = {0.f, 0.f, 0.f, 0.f};

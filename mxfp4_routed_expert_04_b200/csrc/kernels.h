@@ -17,7 +17,7 @@ struct GateUpArgs {
   const int32_t* row_token;  // [R]
   const uint8_t *wg_q, *wg_s, *wu_q, *wu_s;
   __half* h16;               // [R, I]
-  float* hscale;             // [I/16, R]
+  float* hscale;             // [R, I/16]
   int W, I, E, R;
   int min_tokens;            // experts with fewer tokens are left to the CUDA-core path
 };
@@ -37,14 +37,12 @@ struct DownArgs {
 __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
-// CUDA-core path: experts with exactly 1 token; BPT = K blocks per thread,
-// RPS = weight rows per ring stage; at most kFmaMaxThreads threads
-constexpr int kFmaMaxThreads = 256;
+// CUDA-core path: experts with exactly 1 token (gemv_fma.cu)
 struct FmaArgs {
   // activations
   const __half* x16;         // gate/up: [T, W] f16 rows, xscale [T]
   const float* xscale;
-  const __half* h16;         // down: [R, I] f16 rows, hscale [I/16, R]
+  const __half* h16;         // down: [R, I] f16 rows, hscale [R, I/16]
   const float* hscale;
   // routing
   const int32_t* offsets;
@@ -59,9 +57,14 @@ struct FmaArgs {
   int32_t* status;           // device status word
   int W, I, E, R;
 };
-template <int BPT, int RPS, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a);
-size_t fma_stage_bytes(int K, int rps);
-size_t fma_smem_bytes(int K, int rps);
+// Launch geometry: tpr threads per weight row (a power of two), rps rows per
+// ring stage, nslot ring slots, shared-memory offsets.
+struct FmaGeometry {
+  int ok, tpr, rps, nslot;
+  uint32_t stage_bytes, x_bytes, off_x, off_part, off_rsum, off_bar, smem_bytes;
+};
+FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget);
+template <int NT, int BPT, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {
