@@ -48,20 +48,24 @@ def _inputs_digest() -> str:
     return h.hexdigest()
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None) -> str:
-    """Compile every .cu under csrc/ for sm_100a and link the shared library."""
-    digest = _inputs_digest()
-    stamp = LIB + ".sha256"
-    if not force and os.path.exists(LIB) and os.path.exists(stamp):
+def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None,
+          out: str | None = None, defines: tuple = ()) -> str:
+    """Compile every .cu under csrc/ for sm_100a and link the shared library
+    (``out`` and ``defines`` build a variant elsewhere, e.g. for a tuning sweep)."""
+    lib = out or LIB
+    digest = _inputs_digest() + ",".join(defines)
+    stamp = lib + ".sha256"
+    if not force and os.path.exists(lib) and os.path.exists(stamp):
         with open(stamp) as f:
             if f.read().strip() == digest:
                 return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    bdir = BUILD if out is None else out + ".objs"
+    os.makedirs(bdir, exist_ok=True)
     nvcc = _nvcc()
-    extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra = (["-Xptxas", "-v"] if ptxas_verbose else []) + [f"-D{d}" for d in defines]
     procs, objs = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", CSRC, "-c", src, "-o", obj]
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
@@ -76,13 +80,13 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = N
             sys.stdout.write(text)
     if failed:
         raise RuntimeError("nvcc failed")
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     subprocess.check_call([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                            "-o", tmp, *objs])
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     with open(stamp, "w") as f:
         f.write(digest)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":

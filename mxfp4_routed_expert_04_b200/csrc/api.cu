@@ -217,7 +217,14 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
 
 // CUDA-core GEMV launch shape for reduction length K: 256 consumer threads
 // (64 for K < 2048), one 32-element block per thread per row (2 beyond 8192),
-// shared memory for two CTAs per SM (four with 64 consumer threads).
+// shared memory for MOE_FMA_CTAS CTAs per SM (twice as many with 64 consumer
+// threads), ring stages of about MOE_FMA_STAGE_KB KB of codes.
+#ifndef MOE_FMA_CTAS
+#define MOE_FMA_CTAS 2
+#endif
+#ifndef MOE_FMA_STAGE_KB
+#define MOE_FMA_STAGE_KB 8
+#endif
 struct FmaPlan {
   int nt = 0, bpt = 0;
   moe::FmaGeometry g{};
@@ -228,7 +235,8 @@ FmaPlan fma_plan(int K, bool gate_up) {
   f.nt = kb >= 64 ? 256 : 64;
   f.bpt = kb > 256 ? 2 : 1;
   if (kb > 512) return f;                      // g.ok == 0: tensor-core path only
-  f.g = moe::fma_geometry(K, gate_up, f.nt, f.bpt, (f.nt == 256 ? 110 : 54) * 1024);
+  const size_t budget = (220 * 1024) / (f.nt == 256 ? MOE_FMA_CTAS : 2 * MOE_FMA_CTAS);
+  f.g = moe::fma_geometry(K, gate_up, f.nt, f.bpt, budget, MOE_FMA_STAGE_KB * 1024);
   return f;
 }
 // the CUDA-core path serves single-token experts when both projections fit it

@@ -128,6 +128,9 @@ __global__ void __launch_bounds__(NT + 32) k_fma_gemv(FmaArgs a, FmaGeometry g) 
         if (!*abort_flag) timed_out();
         return;
       }
+      // the consumers' generic-proxy reads of this buffer (ordered by the
+      // mbarrier) must precede the bulk copy's async-proxy writes
+      fence_proxy_async_smem();
       uint8_t* xb = xbuf + p * g.x_bytes;
       if (kGateUp) {
         const int tok = __ldg(a.row_token + r0);
@@ -146,6 +149,7 @@ __global__ void __launch_bounds__(NT + 32) k_fma_gemv(FmaArgs a, FmaGeometry g) 
           if (!*abort_flag) timed_out();
           return;
         }
+        fence_proxy_async_smem();
         size_t row;
         const uint8_t *q, *s;
         if (kGateUp) {
@@ -267,7 +271,8 @@ __global__ void __launch_bounds__(NT + 32) k_fma_gemv(FmaArgs a, FmaGeometry g) 
 
 // Geometry of one launch for reduction length K (host side). A gate/up
 // stage never spans the gate and up rows (at most 16 rows).
-FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget) {
+FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget,
+                         size_t stage_target) {
   FmaGeometry g{};
   const int kb = K / 32;
   const int need = (kb + bpt - 1) / bpt;               // threads per row
@@ -277,14 +282,14 @@ FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budge
   g.tpr = tpr;
   const int rp = nt / tpr;
   const size_t qrow = K / 2, srow = K / 32;
-  // rows per stage: a power of two, multiple of rp, <= 32, codes >= ~8 KB,
+  // rows per stage: a power of two, multiple of rp, <= 32, codes >= stage_target,
   // E8M0 bytes a multiple of 16 (bulk-copy size rule)
   int rps = 0;
   for (int r = 1; r <= (gate_up ? 16 : kItemRows); r *= 2) {
     if (r % rp) continue;
     if ((r * srow) % 16) continue;
     rps = r;
-    if ((size_t)r * qrow >= 8192) break;
+    if ((size_t)r * qrow >= stage_target) break;
   }
   if (!rps) return g;
   g.rps = rps;
@@ -293,7 +298,7 @@ FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budge
   const size_t fixed = 2 * (size_t)g.x_bytes + (size_t)kItemRows * tpr * 4 + kItemRows * 4 + 1024;
   int nslot = (int)((smem_budget - fixed) / g.stage_bytes);
   if (nslot < 2) return g;
-  g.nslot = nslot > 16 ? 16 : nslot;
+  g.nslot = nslot > 32 ? 32 : nslot;
   g.off_x = (uint32_t)g.nslot * g.stage_bytes;
   g.off_part = g.off_x + 2 * g.x_bytes;
   g.off_rsum = g.off_part + (uint32_t)(kItemRows * tpr * 4);

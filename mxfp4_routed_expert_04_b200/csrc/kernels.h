@@ -63,7 +63,8 @@ struct FmaGeometry {
   int ok, tpr, rps, nslot;
   uint32_t stage_bytes, x_bytes, off_x, off_part, off_rsum, off_bar, smem_bytes;
 };
-FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget);
+FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget,
+                         size_t stage_target);
 template <int NT, int BPT, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
