@@ -48,7 +48,7 @@ int dense_splits(int N, int T, int K) {
 struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   int S_router, S_sgu, S_sd, S_ld, S_lu;
-  size_t off_status, off_router, off_h16, off_hscale, off_sgu, off_hs, off_gl, off_sd, off_ld,
+  size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_hs, off_gl, off_sd, off_ld,
       off_ylat, off_lu, total;
   size_t xop_bytes, xop_scale_off;
 };
@@ -92,6 +92,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_router = take((size_t)p.S_router * p.T * p.E * 4);
   p.off_h16 = take((size_t)p.R * p.I * 2);
   p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
+  p.off_h32 = take((size_t)p.R * p.I * 4);
   p.off_sgu = take((size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
   p.off_hs = take((size_t)p.T * p.Is * 4);
   p.off_gl = take((size_t)p.T * 4);
@@ -215,52 +216,58 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
   return launched("activation operand");
 }
 
-// CUDA-core GEMV launch shape for reduction length K: 256 consumer threads
-// (64 for K < 2048), one 32-element block per thread per row (2 beyond 8192),
-// shared memory for MOE_FMA_CTAS CTAs per SM (twice as many with 64 consumer
-// threads), ring stages of about MOE_FMA_STAGE_KB KB of codes.
+// CUDA-core GEMV launch shape for reduction length K (up to 8192): lanes own
+// BPL = ceil(K/1024) blocks; work items of MOE_FMA_RT rows per side; shared
+// memory for MOE_FMA_CTAS CTAs per SM; ring stages of about MOE_FMA_STAGE_KB
+// KB of codes.
 #ifndef MOE_FMA_CTAS
-#define MOE_FMA_CTAS 2
+#define MOE_FMA_CTAS 3
 #endif
 #ifndef MOE_FMA_STAGE_KB
-#define MOE_FMA_STAGE_KB 8
+#define MOE_FMA_STAGE_KB 4
+#endif
+#ifndef MOE_FMA_RT
+#define MOE_FMA_RT 8
 #endif
 struct FmaPlan {
-  int nt = 0, bpt = 0;
+  int bpl = 0;
   moe::FmaGeometry g{};
 };
-FmaPlan fma_plan(int K, bool gate_up) {
+FmaPlan fma_plan(int K, int rows) {
   FmaPlan f;
   const int kb = K / 32;
-  f.nt = kb >= 64 ? 256 : 64;
-  f.bpt = kb > 256 ? 2 : 1;
-  if (kb > 512) return f;                      // g.ok == 0: tensor-core path only
-  const size_t budget = (220 * 1024) / (f.nt == 256 ? MOE_FMA_CTAS : 2 * MOE_FMA_CTAS);
-  f.g = moe::fma_geometry(K, gate_up, f.nt, f.bpt, budget, MOE_FMA_STAGE_KB * 1024);
+  f.bpl = kb <= 32 ? 1 : kb <= 64 ? 2 : kb <= 128 ? 4 : kb <= 256 ? 8 : 0;
+  int rt = MOE_FMA_RT;
+  while (rt > 1 && rows % rt) rt /= 2;
+  if (!f.bpl || rows % rt) return f;
+  f.g = moe::fma_geometry(K, rt, (220 * 1024) / MOE_FMA_CTAS, MOE_FMA_STAGE_KB * 1024);
   return f;
 }
 // the CUDA-core path serves single-token experts when both projections fit it
-bool fma_path(const Plan& p) { return fma_plan(p.W, true).g.ok && fma_plan(p.I, false).g.ok; }
+bool fma_path(const Plan& p) { return fma_plan(p.W, p.I).g.ok && fma_plan(p.I, p.W).g.ok; }
 
 template <bool kGateUp>
-moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, long max_items, cudaStream_t st) {
-  const int K = kGateUp ? a.W : a.I;
-  const FmaPlan f = fma_plan(K, kGateUp);
+moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t st) {
+  const int K = kGateUp ? a.W : a.I, rows = kGateUp ? a.I : a.W;
+  const FmaPlan f = fma_plan(K, rows);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
   void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
-  if (f.nt == 64 && f.bpt == 1) kern = moe::k_fma_gemv<64, 1, kGateUp>;
-  if (f.nt == 256 && f.bpt == 1) kern = moe::k_fma_gemv<256, 1, kGateUp>;
-  if (f.nt == 256 && f.bpt == 2) kern = moe::k_fma_gemv<256, 2, kGateUp>;
+  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp>;
+  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp>;
+  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp>;
+  if (f.bpl == 8) kern = moe::k_fma_gemv<8, kGateUp>;
   if (!kern || !f.g.ok) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
-  const int threads = f.nt + 32;
+  const int threads = 32 * moe::kFmaWarps;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)f.g.smem_bytes);
   int per_sm = 0;
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, f.g.smem_bytes);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
-  const long grid = std::max<long>(1, std::min<long>(max_items, (long)ds.num_sms * std::max(1, per_sm)));
-  kern<<<(int)grid, threads, f.g.smem_bytes, st>>>(a, f.g);
+  const long items = (long)std::min(a.E, a.R) * (rows / f.g.rt);
+  const long warps = std::max<long>(1, std::min<long>(items, (long)ds.num_sms * std::max(1, per_sm) * moe::kFmaWarps));
+  const int grid = (int)((warps + moe::kFmaWarps - 1) / moe::kFmaWarps);
+  kern<<<grid, threads, f.g.smem_bytes, st>>>(a, f.g);
   return launched(what);
 }
 
@@ -285,15 +292,15 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   // single-token experts on the CUDA cores
   const bool fma = fma_path(p);
   moe::FmaArgs f;
-  f.x16 = g.x16; f.xscale = g.xscale; f.h16 = g.h16; f.hscale = g.hscale;
+  f.x16 = g.x16; f.xscale = g.xscale; f.h32 = at<float>(ws, p.off_h32);
   f.offsets = offsets; f.expert_list = expert_list; f.row_token = row_token;
   f.wg_q = wg_q; f.wg_s = wg_s; f.wu_q = wu_q; f.wu_s = wu_s; f.wd_q = wd_q; f.wd_s = wd_s;
-  f.h16_out = g.h16; f.hscale_out = g.hscale; f.y_perm = y_perm;
+  f.y_perm = y_perm;
   f.status = at<int32_t>(ws, p.off_status);
   f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
   g.min_tokens = fma ? 2 : 1;
   moe_status s = MOE_OK;
-  if (fma && (s = launch_fma<true>(ds, f, ny * (p.I / 16), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<true>(ds, f, st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
   moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
   s = launched("expert gate/up");
@@ -303,7 +310,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
   d.min_tokens = g.min_tokens;
-  if (fma && (s = launch_fma<false>(ds, f, ny * (p.W / 32), st)) != MOE_OK) return s;
+  if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
   return launched("expert down");

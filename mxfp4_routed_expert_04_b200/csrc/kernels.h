@@ -38,34 +38,27 @@ __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
 // CUDA-core path: experts with exactly 1 token (gemv_fma.cu)
+constexpr int kFmaWarps = 4;     // independent warps per CTA
 struct FmaArgs {
-  // activations
   const __half* x16;         // gate/up: [T, W] f16 rows, xscale [T]
   const float* xscale;
-  const __half* h16;         // down: [R, I] f16 rows, hscale [R, I/16]
-  const float* hscale;
-  // routing
+  float* h32;                // gate/up writes, down reads: [R, I] fp32
   const int32_t* offsets;
   const int32_t* expert_list;
   const int32_t* row_token;
-  // weights
   const uint8_t *wg_q, *wg_s, *wu_q, *wu_s, *wd_q, *wd_s;
-  // outputs
-  __half* h16_out;           // gate/up writes h here (same buffer as h16)
-  float* hscale_out;
   float* y_perm;             // down: [R, W]
   int32_t* status;           // device status word
   int W, I, E, R;
 };
-// Launch geometry: tpr threads per weight row (a power of two), rps rows per
-// ring stage, nslot ring slots, shared-memory offsets.
+// Launch geometry: rt rows per item side, rps rows per ring stage, nst ring
+// stages per warp.
 struct FmaGeometry {
-  int ok, tpr, rps, nslot;
-  uint32_t stage_bytes, x_bytes, off_x, off_part, off_rsum, off_bar, smem_bytes;
+  int ok, rt, rps, nst;
+  uint32_t stage_bytes, smem_bytes;
 };
-FmaGeometry fma_geometry(int K, bool gate_up, int nt, int bpt, size_t smem_budget,
-                         size_t stage_target);
-template <int NT, int BPT, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
+FmaGeometry fma_geometry(int K, int rt, size_t smem_budget, size_t stage_target);
+template <int BPL, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {
