@@ -217,39 +217,33 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
 }
 
 // CUDA-core GEMV launch shape for reduction length K (up to 8192): lanes own
-// BPL = ceil(K/1024) blocks; work items of MOE_FMA_RT rows per side; shared
-// memory for MOE_FMA_CTAS CTAs per SM; ring stages of about MOE_FMA_STAGE_KB
-// KB of codes.
+// BPL = ceil(K/1024) blocks; shared memory for MOE_FMA_CTAS CTAs per SM;
+// down-projection stages of about MOE_FMA_STAGE_KB KB of codes.
 #ifndef MOE_FMA_CTAS
 #define MOE_FMA_CTAS 3
 #endif
 #ifndef MOE_FMA_STAGE_KB
 #define MOE_FMA_STAGE_KB 4
 #endif
-#ifndef MOE_FMA_RT
-#define MOE_FMA_RT 8
-#endif
 struct FmaPlan {
   int bpl = 0;
   moe::FmaGeometry g{};
 };
-FmaPlan fma_plan(int K, int rows) {
+FmaPlan fma_plan(int K, bool gate_up) {
   FmaPlan f;
   const int kb = K / 32;
   f.bpl = kb <= 32 ? 1 : kb <= 64 ? 2 : kb <= 128 ? 4 : kb <= 256 ? 8 : 0;
-  int rt = MOE_FMA_RT;
-  while (rt > 1 && rows % rt) rt /= 2;
-  if (!f.bpl || rows % rt) return f;
-  f.g = moe::fma_geometry(K, rt, (220 * 1024) / MOE_FMA_CTAS, MOE_FMA_STAGE_KB * 1024);
+  if (!f.bpl) return f;
+  f.g = moe::fma_geometry(K, gate_up, (216 * 1024) / MOE_FMA_CTAS, MOE_FMA_STAGE_KB * 1024);
   return f;
 }
 // the CUDA-core path serves single-token experts when both projections fit it
-bool fma_path(const Plan& p) { return fma_plan(p.W, p.I).g.ok && fma_plan(p.I, p.W).g.ok; }
+bool fma_path(const Plan& p) { return fma_plan(p.W, true).g.ok && fma_plan(p.I, false).g.ok; }
 
 template <bool kGateUp>
 moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t st) {
-  const int K = kGateUp ? a.W : a.I, rows = kGateUp ? a.I : a.W;
-  const FmaPlan f = fma_plan(K, rows);
+  const int K = kGateUp ? a.W : a.I;
+  const FmaPlan f = fma_plan(K, kGateUp);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
   void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
   if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp>;
@@ -264,10 +258,11 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, f.g.smem_bytes);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
-  const long items = (long)std::min(a.E, a.R) * (rows / f.g.rt);
-  const long warps = std::max<long>(1, std::min<long>(items, (long)ds.num_sms * std::max(1, per_sm) * moe::kFmaWarps));
-  const int grid = (int)((warps + moe::kFmaWarps - 1) / moe::kFmaWarps);
-  kern<<<grid, threads, f.g.smem_bytes, st>>>(a, f.g);
+  // every warp takes an equal share of the rows of the single-token experts
+  const long rows = (long)std::min(a.E, a.R) * (kGateUp ? a.I : a.W);
+  const long ctas = std::max<long>(1, std::min<long>((rows + moe::kFmaWarps - 1) / moe::kFmaWarps,
+                                                     (long)ds.num_sms * std::max(1, per_sm)));
+  kern<<<(int)ctas, threads, f.g.smem_bytes, st>>>(a, f.g);
   return launched(what);
 }
 

@@ -51,13 +51,14 @@ struct FmaArgs {
   int32_t* status;           // device status word
   int W, I, E, R;
 };
-// Launch geometry: rt rows per item side, rps rows per ring stage, nst ring
+// Launch geometry: rps rows per down-projection ring stage (gate/up stages
+// hold one row), sbuf_off = offset of the E8M0 span inside a stage, nst ring
 // stages per warp.
 struct FmaGeometry {
-  int ok, rt, rps, nst;
-  uint32_t stage_bytes, smem_bytes;
+  int ok, rps, nst;
+  uint32_t sbuf_off, stage_bytes, smem_bytes;
 };
-FmaGeometry fma_geometry(int K, int rt, size_t smem_budget, size_t stage_target);
+FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, size_t stage_target);
 template <int BPL, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
