@@ -61,15 +61,6 @@ MOE_DEV float warp_max(float v) {
   return v;
 }
 
-// One ring stage: `n` consecutive rows of one weight matrix.
-struct StageDesc {
-  const uint8_t* q;        // codes of the first row
-  const uint8_t* s;        // first byte of the copied E8M0 span
-  uint32_t n;              // rows
-  uint32_t soff;           // offset of the first row's E8M0 codes inside the span
-  uint32_t sbytes;         // bytes of the span (multiple of 16)
-};
-
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -77,7 +68,7 @@ struct StageDesc {
 // shared memory = kFmaWarps * g.nst * (g.stage_bytes + 8)
 // ---------------------------------------------------------------------------
 template <int BPL, bool kGateUp>
-__global__ void __launch_bounds__(32 * kFmaWarps) k_fma_gemv(FmaArgs a, FmaGeometry g) {
+__global__ void __launch_bounds__(32 * kFmaWarps, 3) k_fma_gemv(FmaArgs a, FmaGeometry g) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
   __shared__ int s_wsum[kFmaWarps];
@@ -109,11 +100,12 @@ __global__ void __launch_bounds__(32 * kFmaWarps) k_fma_gemv(FmaArgs a, FmaGeome
   }
 
   // 2) this warp's share of the units (gate/up: row pairs; down: rows)
-  const long total = (long)n_single * N;
-  const long nwarps = (long)gridDim.x * kFmaWarps;
-  const long gw = (long)blockIdx.x * kFmaWarps + warp;
-  const long lo = total * gw / nwarps, hi = total * (gw + 1) / nwarps;
+  const int total = n_single * N;                        // < 2^27
+  const int nwarps = gridDim.x * kFmaWarps;
+  const int gw = blockIdx.x * kFmaWarps + warp;
+  const int lo = (int)((long)total * gw / nwarps), hi = (int)((long)total * (gw + 1) / nwarps);
   if (lo >= hi) return;
+  const int hi_si = hi / N, hi_r = hi - hi_si * N;       // end of the range as (expert, row)
 
   uint8_t* ring = smem + (size_t)warp * g.nst * g.stage_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kFmaWarps * g.nst * g.stage_bytes) +
@@ -124,69 +116,60 @@ __global__ void __launch_bounds__(32 * kFmaWarps) k_fma_gemv(FmaArgs a, FmaGeome
   }
   __syncwarp();
 
-  // stage sequence: gate/up -> per unit the gate row, then the up row;
-  // down -> up to g.rps rows of one expert per stage
-  auto stage_of = [&](long u, int half, StageDesc& d) -> long {   // returns units consumed
-    const int si = (int)(u / N), r = (int)(u - (long)si * N);
-    const int e = s_list[si];
-    long take;
-    size_t row;
-    const uint8_t *q, *s;
-    if (kGateUp) {
-      take = half;                               // the pair is done after its up row
-      row = (size_t)e * N + r;
-      q = half ? a.wu_q : a.wg_q;
-      s = half ? a.wu_s : a.wg_s;
-      d.n = 1;
-    } else {
-      take = min((long)g.rps, min(hi - u, (long)(N - r)));
-      row = (size_t)e * N + r;
-      q = a.wd_q;
-      s = a.wd_s;
-      d.n = (uint32_t)take;
-    }
-    d.q = q + row * qrow;
-    const size_t s0 = row * srow, s1 = (row + d.n) * srow;
-    const size_t a0 = s0 & ~(size_t)15, a1 = min((s1 + 15) & ~(size_t)15, s_total);
-    d.s = s + a0;
-    d.soff = (uint32_t)(s0 - a0);
-    d.sbytes = (uint32_t)(a1 - a0);
-    return take;
+  // A cursor walks the stage sequence: gate/up -> for each row pair the gate
+  // row, then the up row; down -> up to g.rps rows of one expert per stage.
+  struct Cursor { int si, r, half; };
+  auto rows_in_stage = [&](const Cursor& c) -> int {
+    if (kGateUp) return 1;
+    const int left = (c.si == hi_si) ? hi_r - c.r : N - c.r;
+    return min(g.rps, left);
   };
+  auto advance = [&](Cursor& c, int n) {
+    if (kGateUp) {
+      c.half ^= 1;
+      if (c.half) return;
+      n = 1;
+    }
+    c.r += n;
+    if (c.r == N) { c.r = 0; ++c.si; }
+  };
+  auto done = [&](const Cursor& c) { return c.si > hi_si || (c.si == hi_si && c.r >= hi_r); };
 
-  // producer state (lane 0): next unit and half to copy
-  long p_u = lo;
-  int p_half = 0, p_v = 0;
+  // producer (lane 0): stage copies, g.nst ahead of the consumer
+  Cursor pc{lo / N, lo - (lo / N) * N, 0};
+  int p_v = 0;
   auto issue_next = [&]() {
-    if (p_u >= hi) return;
-    StageDesc d;
-    const long took = stage_of(p_u, p_half, d);
+    if (done(pc)) return;
+    const int n = rows_in_stage(pc);
+    const int e = s_list[pc.si];
+    const size_t row = (size_t)e * N + pc.r;
+    const uint8_t* q = kGateUp ? (pc.half ? a.wu_q : a.wg_q) : a.wd_q;
+    const uint8_t* sp = kGateUp ? (pc.half ? a.wu_s : a.wg_s) : a.wd_s;
+    const size_t s0 = row * srow, s1 = (row + n) * srow;
+    const size_t a0 = s0 & ~(size_t)15, a1 = min((s1 + 15) & ~(size_t)15, s_total);
     const int slot = p_v % g.nst;
     uint8_t* dst = ring + (size_t)slot * g.stage_bytes;
-    const uint32_t cb = (uint32_t)(d.n * qrow);
+    const uint32_t cb = (uint32_t)(n * qrow);
     fence_proxy_async_smem();            // earlier generic reads of the slot come first
-    mbar_expect_tx(&bars[slot], cb + d.sbytes);
-    bulk_g2s(dst, d.q, cb, &bars[slot]);
-    bulk_g2s(dst + g.sbuf_off, d.s, d.sbytes, &bars[slot]);
+    mbar_expect_tx(&bars[slot], cb + (uint32_t)(a1 - a0));
+    bulk_g2s(dst, q + row * qrow, cb, &bars[slot]);
+    bulk_g2s(dst + g.sbuf_off, sp + a0, (uint32_t)(a1 - a0), &bars[slot]);
     ++p_v;
-    if (kGateUp) { p_u += took; p_half ^= 1; }
-    else p_u += took;
+    advance(pc, n);
   };
   if (lane == 0)
     for (int i = 0; i < g.nst; ++i) issue_next();
 
   bool dead = false;
-  int v = 0;
+  int v = 0, slot = 0, phase = 0;
   int cur_si = -1, r0 = 0;
   uint32_t xr[BPL][16];
   float xs = 1.0f, gsum = 0.0f;
-  long u = lo;
-  int half = 0;
-  while (u < hi) {
-    const int si = (int)(u / N);
-    if (si != cur_si) {                   // new expert: load its activation row
-      cur_si = si;
-      const int e = s_list[si];
+  Cursor c{lo / N, lo - (lo / N) * N, 0};
+  while (!done(c)) {
+    if (c.si != cur_si) {                 // new expert: load its activation row
+      cur_si = c.si;
+      const int e = s_list[c.si];
       r0 = __ldg(a.offsets + e);
       if (kGateUp) {
         const int tok = __ldg(a.row_token + r0);
@@ -240,17 +223,15 @@ __global__ void __launch_bounds__(32 * kFmaWarps) k_fma_gemv(FmaArgs a, FmaGeome
         }
       }
     }
-    StageDesc d;
-    const long took = stage_of(u, half, d);
-    const int slot = v % g.nst;
-    if (!dead && !mbar_wait(&bars[slot], (uint32_t)(v / g.nst) & 1u)) {
+    const int n = rows_in_stage(c);
+    if (!dead && !mbar_wait(&bars[slot], (uint32_t)phase)) {
       dead = true;
       if (lane == 0) atomicOr(a.status, kStatusWaitTimeout);
     }
     const uint8_t* stg = ring + (size_t)slot * g.stage_bytes;
-    const uint8_t* ssc = stg + g.sbuf_off + d.soff;
-    const int r = (int)(u - (long)si * N);
-    for (uint32_t rr = 0; rr < d.n; ++rr) {
+    const int e = s_list[c.si];
+    const uint8_t* ssc = stg + g.sbuf_off + ((((size_t)e * N + c.r) * srow) & 15);
+    for (int rr = 0; rr < n; ++rr) {
       float acc = 0.0f;
 #pragma unroll
       for (int j = 0; j < BPL; ++j) {
@@ -262,17 +243,17 @@ __global__ void __launch_bounds__(32 * kFmaWarps) k_fma_gemv(FmaArgs a, FmaGeome
       }
       const float sum = warp_sum(acc);
       if (kGateUp) {
-        if (!half) gsum = sum;
-        else if (lane == 0) a.h32[(size_t)r0 * a.I + r] = silu_f32(gsum * xs) * (sum * xs);
+        if (!c.half) gsum = sum;
+        else if (lane == 0) a.h32[(size_t)r0 * a.I + c.r] = silu_f32(gsum * xs) * (sum * xs);
       } else if (lane == 0) {
-        a.y_perm[(size_t)r0 * a.W + r + rr] = sum * xs;
+        a.y_perm[(size_t)r0 * a.W + c.r + rr] = sum * xs;
       }
     }
     __syncwarp();
     ++v;
+    if (++slot == g.nst) { slot = 0; phase ^= 1; }
     if (lane == 0 && !dead) issue_next();  // refill the slot just consumed
-    if (kGateUp) { u += took; half ^= 1; }
-    else u += took;
+    advance(c, n);
   }
 }
 
