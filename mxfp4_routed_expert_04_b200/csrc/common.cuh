@@ -217,16 +217,18 @@ MOE_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 }
 
 // Bounded wait for phase `parity` of `bar`: false when it did not complete
-// within the iteration limit (the caller reports it and leaves).
+// within the iteration limit (the caller reports it and leaves). Each
+// try_wait may suspend the thread for up to 20 us until the phase completes,
+// so a waiting warp does not spin on the issue slots; the bound is about 5 s.
 MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0; it < (1u << 26); ++it) {
+  for (uint32_t it = 0; it < (1u << 18); ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        : "=r"(done) : "r"(a), "r"(parity), "r"(20000u) : "memory");
     if (done) return true;
   }
   return false;

@@ -36,18 +36,35 @@ namespace {
 // scale not applied).
 MOE_DEV float dot_block(uint4 w, const uint32_t (&x)[16]) {
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t h[4];
     e2m1x8_to_f16x8(words[q], h);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      a[2 * (j & 1)] = fma_f16lo(h[j], x[4 * q + j], a[2 * (j & 1)]);
-      a[2 * (j & 1) + 1] = fma_f16hi(h[j], x[4 * q + j], a[2 * (j & 1) + 1]);
+      a0 = fma_f16lo(h[j], x[4 * q + j], a0);
+      a1 = fma_f16hi(h[j], x[4 * q + j], a1);
     }
   }
-  return (a[0] + a[1]) + (a[2] + a[3]);
+  return a0 + a1;
+}
+
+// E8M0 code -> fp32 scale for codes 1..254 (one shift); codes 0 and 255 go
+// through e8m0_to_f32 (a stage holding either takes the exact path).
+MOE_DEV float e8m0_fast(uint32_t c) { return __uint_as_float(c << 23); }
+
+// true when any of the n bytes at p (16-byte aligned span) is 0x00 or 0xFF;
+// every lane checks 16-byte pieces, the warp votes
+MOE_DEV bool span_has_special(const uint8_t* p, int n, int lane) {
+  bool any = false;
+  for (int i = lane * 16; i < n; i += 32 * 16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) any |= (__vcmpeq4(w[k], 0u) | __vcmpeq4(w[k], 0xFFFFFFFFu)) != 0u;
+  }
+  return __any_sync(0xFFFFFFFFu, any);
 }
 
 MOE_DEV float warp_sum(float v) {
@@ -230,7 +247,10 @@ __global__ void __launch_bounds__(32 * kFmaWarps, 3) k_fma_gemv(FmaArgs a, FmaGe
     }
     const uint8_t* stg = ring + (size_t)slot * g.stage_bytes;
     const int e = s_list[c.si];
-    const uint8_t* ssc = stg + g.sbuf_off + ((((size_t)e * N + c.r) * srow) & 15);
+    const uint32_t soff = (uint32_t)((((size_t)e * N + c.r) * srow) & 15);
+    const uint8_t* ssc = stg + g.sbuf_off + soff;
+    // the span copied with the stage is scanned once: codes 0 / 255 are rare
+    const bool special = span_has_special(stg + g.sbuf_off, (int)((soff + n * srow + 15) & ~15u), lane);
     for (int rr = 0; rr < n; ++rr) {
       float acc = 0.0f;
 #pragma unroll
@@ -238,7 +258,8 @@ __global__ void __launch_bounds__(32 * kFmaWarps, 3) k_fma_gemv(FmaArgs a, FmaGe
         const int b = lane + 32 * j;
         if (b < KB) {
           const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * qrow + b * 16);
-          acc = fmaf(dot_block(w, xr[j]), e8m0_to_f32(ssc[rr * srow + b]), acc);
+          const uint32_t code = ssc[rr * srow + b];
+          acc = fmaf(dot_block(w, xr[j]), special ? e8m0_to_f32(code) : e8m0_fast(code), acc);
         }
       }
       const float sum = warp_sum(acc);
