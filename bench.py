@@ -76,6 +76,29 @@ def layer_flops(w):
     return f
 
 
+def _csrc_digest():
+    import hashlib
+    d = os.path.join(ROOT, "mxfp4_routed_expert_04_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload):
+    """DRAM bytes per moe_expert_ffn call from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        if t.get("csrc_sha") == _csrc_digest() and workload in t.get("bytes_per_call", {}):
+            return t["bytes_per_call"][workload]
+    except Exception:
+        pass
+    return None
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -277,7 +300,8 @@ def run_ours(args, w):
         "roofline": {"kernel": "moe_expert_ffn (k_gateup_mxfp4 + k_down_mxfp4)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "bytes_per_launch": fb, "ms_per_launch": ffn_ms, "traffic": None},
+                     "bytes_per_launch": fb, "ms_per_launch": ffn_ms,
+                     "traffic": _traffic(w.name)},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
@@ -383,9 +407,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling case: keep only this many experts resident (same shapes "
+                         "and top-k); the line is then not the workload's metric")
     args = ap.parse_args()
+    import dataclasses
+
     from mxfp4_routed_expert_04_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.experts:
+        w = dataclasses.replace(w, E=args.experts, name=f"{w.name}-E{args.experts}")
     res = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if res is not None:
         print(json.dumps(res), flush=True)
