@@ -130,6 +130,21 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
                      int32_t* topk_idx, float* topk_w, float* logits,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* --- router without a workspace ---------------------------------------------
+ * (No counterpart in the pages: an interface convenience of this library.)
+ * The same computation and outputs as moe_route, for callers that cannot
+ * supply device scratch memory (a plug-in given only its input and output
+ * tensors, or a runtime whose memory plan allows no extra buffer): the
+ * split-K partial sums go to a 4 MiB device array built into the library.
+ * Shapes needing more than 4 MiB of partials (S * T * E fp32 values, S the
+ * K-split count of moe_route) return MOE_ERR_UNSUPPORTED_SHAPE. The array is
+ * shared by every call on a device: calls that overlap on the GPU race on
+ * it. The first call on each device looks up the array's address; make it
+ * before capturing a stream into a CUDA graph. Nothing is allocated.
+ */
+moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
+                             int32_t* topk_idx, float* topk_w, float* logits, void* stream);
+
 /* --- a3-a4: permutation ----------------------------------------------------
  * Groups the T*k (token, slot) pairs by expert: counts[e] pairs per expert,
  * offsets = exclusive prefix sum (E+1 entries), permuted rows ordered by

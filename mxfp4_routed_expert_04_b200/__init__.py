@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "MoeError", "MoeDims", "MoeLayerArgs", "ACT_BF16", "ACT_MXFP4", "library_path",
     "moe_status_string", "moe_workspace_size", "moe_x_op_size", "moe_workspace_init",
-    "moe_device_status", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+    "moe_device_status", "moe_route", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_latent_down", "moe_layer", "MoeLayer",
 ]
 
@@ -34,7 +34,7 @@ def _load():
     path = library_path()
     if not os.path.exists(path):
         raise ImportError(
-            f"{path} is missing: build it with `python -m mxfp4_routed_expert_04_b200.build` "
+            f"{path} is missing: build it with `python mxfp4_routed_expert_04_b200/build.py` "
             "(there is no fallback implementation)")
     return ctypes.CDLL(path)
 
@@ -75,6 +75,7 @@ _sigs = {
     "moe_workspace_init": [_D, _P, _Z, _P],
     "moe_device_status": [_P, ctypes.POINTER(ctypes.c_int32), _P],
     "moe_route": [_D, _P, _P, _P, _P, _P, _P, _Z, _P],
+    "moe_route_noalloc": [_D, _P, _P, _P, _P, _P, _P],
     "moe_permute": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_expert_ffn": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_combine": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
@@ -146,6 +147,12 @@ def _nbytes(t):
 def moe_route(dims, x, w_router, topk_idx, topk_w, logits, ws, stream=None):
     _check(_lib.moe_route(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(topk_idx),
                           _ptr(topk_w), _ptr(logits), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def moe_route_noalloc(dims, x, w_router, topk_idx, topk_w, logits, stream=None):
+    """moe_route without a workspace (partials in the library's static device array)."""
+    _check(_lib.moe_route_noalloc(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(topk_idx),
+                                  _ptr(topk_w), _ptr(logits), _stream(stream)))
 
 
 def moe_permute(dims, topk_idx, x_in, counts, offsets, expert_list, row_token, row_slot, slot_row,

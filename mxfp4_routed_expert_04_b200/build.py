@@ -1,6 +1,6 @@
 """Build the CUDA library (sm_100a) in-tree: mxfp4_routed_expert_04_b200/libmoe_mxfp4.so.
 
-Usage: python -m mxfp4_routed_expert_04_b200.build [--verbose-ptxas]
+Usage: python mxfp4_routed_expert_04_b200/build.py [--force] [--verbose-ptxas]
 """
 from __future__ import annotations
 

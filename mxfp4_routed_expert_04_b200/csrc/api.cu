@@ -365,6 +365,12 @@ moe_status do_latent_down(const Plan& p, const uint16_t* x, const uint16_t* w_ld
 
 }  // namespace
 
+namespace moe {
+// Record a status and its one-line reason for moe_last_error() (used by the
+// entry points that live in other translation units).
+moe_status record_error(moe_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace moe
+
 // ===========================================================================
 // C ABI
 // ===========================================================================

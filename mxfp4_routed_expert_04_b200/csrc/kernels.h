@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe_mxfp4.h"
+
 namespace moe {
 
 // --- grouped MXFP4 GEMV (decode) -------------------------------------------
@@ -105,5 +107,8 @@ struct CombineArgs {
   int T, width;
 };
 __global__ void k_combine(CombineArgs a);
+
+// one-line reason for moe_last_error() (defined with the C ABI in api.cu)
+moe_status record_error(moe_status s, const char* msg);
 
 }  // namespace moe
