@@ -151,6 +151,17 @@ def topk_route(logits, k: int, near_tie: float = 1e-5):
     return idx, w, flagged
 
 
+def selection_weights(logits, idx):
+    """Renormalised softmax weights of a GIVEN selection idx [T, k] (the weight
+    rule of topk_route applied to another valid choice, e.g. the GPU's choice
+    at a near-tie token): w[t, j] = exp(l_j - m) / sum_j' exp(l_j' - m), m the
+    largest selected logit."""
+    logits = np.asarray(logits, dtype=np.float64)
+    sel = np.take_along_axis(logits, np.asarray(idx, dtype=np.int64), axis=1)
+    ex = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return ex / ex.sum(axis=1, keepdims=True)
+
+
 # ---------------------------------------------------------------------------
 # a3: permutation (token -> expert dispatch)
 # ---------------------------------------------------------------------------
@@ -361,9 +372,7 @@ def moe_layer(inp: dict, k: int, experts, act: str = "exact", idx_override=None,
     idx, w, flagged = topk_route(logits, k, near_tie)
     if idx_override is not None:
         idx = np.asarray(idx_override, dtype=np.int32)
-        sel = np.take_along_axis(logits, idx.astype(np.int64), axis=1)
-        ex = np.exp(sel - sel.max(axis=1, keepdims=True))
-        w = ex / ex.sum(axis=1, keepdims=True)
+        w = selection_weights(logits, idx)
     counts, offsets, row_token, row_slot, slot_row = permute(idx, E)
     latent = "w_lat_down" in inp
     if latent:
