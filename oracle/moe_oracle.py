@@ -39,7 +39,8 @@ import numpy as np
 
 __all__ = [
     "E2M1_MAGNITUDES", "e2m1_decode", "e8m0_decode", "mxfp4_dequant", "bf16_to_f64",
-    "round_to_bf16_bits", "router_logits", "topk_route", "permute", "mxfp4_quantize",
+    "round_to_bf16_bits", "router_logits", "topk_route", "selection_weights", "permute",
+    "mxfp4_quantize",
     "silu", "sigmoid", "expert_ffn", "shared_expert", "combine", "latent_down", "moe_layer",
 ]
 

@@ -195,6 +195,17 @@ def test_topk_weights_equal_renormalised_full_softmax():
     assert np.all(np.diff(w, axis=1) <= 0)      # slots in descending weight
 
 
+def test_selection_weights_of_any_choice_equal_renormalised_full_softmax():
+    # any k distinct experts, not only the top k (the weight rule of a near-tie choice)
+    rng = np.random.default_rng(9)
+    logits = rng.standard_normal((20, 48)) * 1.8
+    idx = np.stack([rng.permutation(48)[:6] for _ in range(20)]).astype(np.int32)
+    p = scipy.special.softmax(logits, axis=1)
+    sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(O.selection_weights(logits, idx), sel / sel.sum(axis=1, keepdims=True),
+                               rtol=1e-13)
+
+
 def test_topk_near_tie_flag():
     logits = np.array([[3.0, 2.0, 1.0, 1.0 - 5e-6, 0.0],
                        [3.0, 2.0, 1.0, 0.5, 0.0],
