@@ -186,6 +186,18 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
                           const uint8_t* wd_q, const uint8_t* wd_s,
                           float* y_perm, void* ws, size_t ws_bytes, void* stream);
 
+/* --- inspection of the intermediate activation h ----------------------------
+ * (No counterpart in the pages: a test and debugging aid of this library.)
+ * Byte offsets inside the workspace where moe_expert_ffn leaves, for
+ * MOE_ACT_MXFP4, the MXFP4 encoding of h = silu(Wg x) * (Wu x) exactly as the
+ * down projection consumed it: codes [T*k, I/2] uint8 (low nibble = even
+ * element) at *codes_off and E8M0 scale codes [T*k, I/32] uint8 at
+ * *scales_off, rows in permuted order. Valid until the next call that uses
+ * the workspace. MOE_ACT_BF16 keeps h in an internal form and returns
+ * MOE_ERR_UNSUPPORTED_SHAPE; NULL outputs return MOE_ERR_INVALID_ARG.
+ */
+moe_status moe_h_operand_offsets(const moe_dims* dims, size_t* codes_off, size_t* scales_off);
+
 /* --- a8-a9 (+a10 up): shared expert and combine ------------------------------
  *   s_t = sigmoid(w_sgate . x_t) * Ws_down (silu(Ws_gate x_t) * (Ws_up x_t))
  *   y_t = [W_lu] (sum_j topk_w[t, j] * y_perm[slot_row[t, j]]) + s_t

@@ -17,7 +17,7 @@ __all__ = [
     "MoeError", "MoeDims", "MoeLayerArgs", "ACT_BF16", "ACT_MXFP4", "library_path",
     "moe_status_string", "moe_workspace_size", "moe_x_op_size", "moe_workspace_init",
     "moe_device_status", "moe_route", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
-    "moe_latent_down", "moe_layer", "MoeLayer",
+    "moe_latent_down", "moe_layer", "moe_h_operand_offsets", "MoeLayer",
 ]
 
 ACT_BF16 = 0
@@ -81,6 +81,7 @@ _sigs = {
     "moe_combine": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_latent_down": [_D, _P, _P, _P, _P, _Z, _P],
     "moe_layer": [_D, ctypes.POINTER(MoeLayerArgs), _P, _Z, _P],
+    "moe_h_operand_offsets": [_D, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)],
 }
 for _n, _a in _sigs.items():
     getattr(_lib, _n).argtypes = _a
@@ -124,6 +125,13 @@ def moe_workspace_size(dims: MoeDims) -> int:
 
 def moe_x_op_size(dims: MoeDims) -> int:
     return _lib.moe_x_op_size(ctypes.byref(dims))
+
+
+def moe_h_operand_offsets(dims) -> tuple:
+    """Workspace byte offsets of the MXFP4 h operand (codes, scales); MOE_ACT_MXFP4 only."""
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.moe_h_operand_offsets(ctypes.byref(dims), ctypes.byref(c), ctypes.byref(s)))
+    return c.value, s.value
 
 
 def moe_workspace_init(dims, ws, stream=None):

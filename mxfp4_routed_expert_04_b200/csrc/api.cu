@@ -1,5 +1,7 @@
 // C ABI of the routed MXFP4 MoE layer: validation, workspace plan, launch
 // order. Declared in include/moe_mxfp4.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -49,7 +51,8 @@ struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   int S_router, S_sgu, S_sd, S_ld, S_lu;
   size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_hs, off_gl, off_sd, off_ld,
-      off_ylat, off_lu, total;
+      off_ylat, off_lu, off_tiles, off_ntiles, total;
+  int max_tiles;
   size_t xop_bytes, xop_scale_off;
 };
 
@@ -100,6 +103,11 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
   p.off_ylat = take(p.L ? (size_t)p.T * p.L * 4 : 0);
   p.off_lu = take(p.L ? (size_t)p.S_lu * p.T * p.H * 4 : 0);
+  // MXFP4 activations: tile list of the tensor-core GEMM (h codes and scales
+  // reuse the h16 / hscale regions, which are larger)
+  p.max_tiles = p.mode == MOE_ACT_MXFP4 ? p.R / 128 + std::min(p.E, p.R) + 1 : 0;
+  p.off_tiles = take((size_t)p.max_tiles * 16);
+  p.off_ntiles = take(p.mode == MOE_ACT_MXFP4 ? 16 : 0);
   p.total = o;
   if (p.mode == MOE_ACT_BF16) {
     p.xop_scale_off = align_up((size_t)p.T * p.W * 2, 256);
@@ -154,6 +162,12 @@ moe_status device_state(DeviceState** out) {
   if (!s.ready) {
     cudaError_t e = cudaFuncSetAttribute(moe::k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)moe::permute_smem_bytes(1024));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_mxf4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)moe::mxf4_gemm_smem_bytes(true));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_mxf4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)moe::mxf4_gemm_smem_bytes(false));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.gemv_ctas_per_sm, moe::k_gateup_mxfp4, 32,
@@ -266,13 +280,92 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   return launched(what);
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links no driver stub).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D map over a [rows, row_bytes] uint8 matrix read in boxes of 128 rows x
+// 128 bytes with the 128-byte swizzle (row_bytes a multiple of 64).
+moe_status weight_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
+                      const char* what) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
+  return MOE_OK;
+}
+
+// MXFP4 activations: tile list, then gate/up (+ SwiGLU, h quantised to MXFP4)
+// and down on the tensor cores, one persistent CTA per SM each.
+moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* x_op,
+                              const int32_t* offsets, const int32_t* expert_list,
+                              const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
+                              const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
+                              const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
+  int4* tiles = at<int4>(ws, p.off_tiles);
+  int32_t* n_tiles = at<int32_t>(ws, p.off_ntiles);
+  moe::k_tile_list<<<1, 1024, 0, st>>>(offsets, expert_list, tiles, n_tiles);
+  moe_status s = launched("tile list");
+  if (s != MOE_OK) return s;
+  uint8_t* hq = at<uint8_t>(ws, p.off_h16);
+  uint8_t* hs = at<uint8_t>(ws, p.off_hscale);
+  moe::Mxf4GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  if ((s = weight_map(&g.map_a0, wg_q, (uint64_t)p.E * p.I, p.W / 2, "gate weights")) != MOE_OK ||
+      (s = weight_map(&g.map_a1, wu_q, (uint64_t)p.E * p.I, p.W / 2, "up weights")) != MOE_OK)
+    return s;
+  g.sa0 = wg_s; g.sa1 = wu_s;
+  g.bq = static_cast<const uint8_t*>(x_op);
+  g.bs = static_cast<const uint8_t*>(x_op) + p.xop_scale_off;
+  g.row_token = row_token;
+  g.tiles = tiles; g.n_tiles = n_tiles;
+  g.hq = hq; g.hs = hs;
+  g.status = at<int32_t>(ws, p.off_status);
+  g.K = p.W; g.M = p.I;
+  moe::k_mxf4_gemm<true><<<ds.num_sms, 256, moe::mxf4_gemm_smem_bytes(true), st>>>(g);
+  if ((s = launched("expert gate/up (tcgen05)")) != MOE_OK) return s;
+  moe::Mxf4GemmArgs d;
+  memset(&d, 0, sizeof(d));
+  if ((s = weight_map(&d.map_a0, wd_q, (uint64_t)p.E * p.W, p.I / 2, "down weights")) != MOE_OK)
+    return s;
+  d.map_a1 = d.map_a0;
+  d.sa0 = wd_s; d.sa1 = wd_s;
+  d.bq = hq; d.bs = hs;
+  d.row_token = nullptr;
+  d.tiles = tiles; d.n_tiles = n_tiles;
+  d.y = y_perm;
+  d.status = g.status;
+  d.K = p.I; d.M = p.W;
+  moe::k_mxf4_gemm<false><<<ds.num_sms, 256, moe::mxf4_gemm_smem_bytes(false), st>>>(d);
+  return launched("expert down (tcgen05)");
+}
+
 moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const int32_t* offsets, const int32_t* expert_list,
                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
                          const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
-  if (p.mode != MOE_ACT_BF16)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "act_mode MOE_ACT_MXFP4 expert GEMM is not available");
+  if (p.mode == MOE_ACT_MXFP4)
+    return do_expert_ffn_mxf4(p, ds, x_op, offsets, expert_list, row_token, wg_q, wg_s, wu_q, wu_s,
+                              wd_q, wd_s, y_perm, ws, st);
   const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
   moe::GateUpArgs g;
   g.x16 = static_cast<const __half*>(x_op);
@@ -399,6 +492,18 @@ size_t moe_workspace_size(const moe_dims* dims) {
 size_t moe_x_op_size(const moe_dims* dims) {
   Plan p;
   return make_plan(dims, p) == MOE_OK ? p.xop_bytes : 0;
+}
+
+moe_status moe_h_operand_offsets(const moe_dims* dims, size_t* codes_off, size_t* scales_off) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if (!codes_off || !scales_off) return fail(MOE_ERR_INVALID_ARG, "output pointer is NULL");
+  if (p.mode != MOE_ACT_MXFP4)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "h is exposed only for MOE_ACT_MXFP4");
+  *codes_off = p.off_h16;
+  *scales_off = p.off_hscale;
+  return MOE_OK;
 }
 
 moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream) {

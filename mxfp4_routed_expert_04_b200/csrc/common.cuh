@@ -58,6 +58,15 @@ MOE_DEV void e2m1x8_to_f16x8(uint32_t w, uint32_t (&out)[4]) {
       : "r"(w));
 }
 
+// E2M1 code (0..7 magnitude) of a non-negative value already divided by the
+// block scale: nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even code
+// (the OCP MX v1.0 conversion to E2M1).
+MOE_DEV uint32_t e2m1_magnitude_code(float s) {
+  return (uint32_t)(s > 0.25f) + (uint32_t)(s >= 0.75f) + (uint32_t)(s > 1.25f) +
+         (uint32_t)(s >= 1.75f) + (uint32_t)(s > 2.5f) + (uint32_t)(s >= 3.5f) +
+         (uint32_t)(s > 5.0f);
+}
+
 // ---------------------------------------------------------------------------
 // tensor-core MMA (warp-level m16n8k16, fp32 accumulate)
 // ---------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 // Internal kernel interfaces of the MoE layer library (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -62,6 +63,31 @@ struct FmaGeometry {
 };
 FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, size_t stage_target);
 template <int BPL, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
+
+// --- grouped MXFP4 GEMM on tcgen05 (many tokens per expert) ----------------
+// Weight operands are read through 2-D tensor maps over [E*M, K/2] bytes
+// (boxes of 128 rows x 128 bytes, 128-byte swizzle); their E8M0 scales are
+// [E*M, K/32]. B rows (tokens) are codes [*, K/2] and scales [*, K/32].
+struct Mxf4GemmArgs {
+  CUtensorMap map_a0;        // gate/up: gate weights; down: down weights
+  CUtensorMap map_a1;        // gate/up: up weights
+  const uint8_t* sa0;
+  const uint8_t* sa1;
+  const uint8_t* bq;         // B codes: x_op codes [T, K/2] (gate/up) or h codes [R, K/2] (down)
+  const uint8_t* bs;         // B scales
+  const int32_t* row_token;  // gate/up: B row of permuted row r; down: NULL (B row = r)
+  const int4* tiles;         // k_tile_list output
+  const int32_t* n_tiles;
+  uint8_t* hq;               // gate/up out: h codes [R, M/2]
+  uint8_t* hs;               // gate/up out: h scales [R, M/32]
+  float* y;                  // down out: y_perm [R, M]
+  int32_t* status;           // device status word
+  int K, M;                  // reduction length; weight rows per expert (a multiple of 128)
+};
+__global__ void k_tile_list(const int32_t* offsets, const int32_t* expert_list, int4* tiles,
+                            int32_t* n_tiles);
+template <bool kGateUp> __global__ void k_mxf4_gemm(const __grid_constant__ Mxf4GemmArgs a);
+size_t mxf4_gemm_smem_bytes(bool gate_up);
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {

@@ -196,14 +196,6 @@ __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__
   if (threadIdx.x == 0) xscale[tok] = scale;
 }
 
-// E2M1 code (0..7 magnitude) of a non-negative value already divided by the
-// block scale: nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even code.
-MOE_DEV uint32_t e2m1_magnitude_code(float s) {
-  return (uint32_t)(s > 0.25f) + (uint32_t)(s >= 0.75f) + (uint32_t)(s > 1.25f) +
-         (uint32_t)(s >= 1.75f) + (uint32_t)(s > 2.5f) + (uint32_t)(s >= 3.5f) +
-         (uint32_t)(s > 5.0f);
-}
-
 // grid T, block 256; W a multiple of 32. Each 4 consecutive threads own one
 // 32-element block (8 elements each).
 __global__ void __launch_bounds__(256) k_act_to_mxfp4(const uint16_t* __restrict__ x, int W,

@@ -108,3 +108,15 @@ def test_x_op_size_by_mode():
     assert M.moe_x_op_size(d0) >= 4 * 256 * 2 + 16
     assert M.moe_x_op_size(d1) >= 4 * 128 + 4 * 8
     assert M.moe_x_op_size(d1) < M.moe_x_op_size(d0)
+
+
+def test_h_operand_offsets_only_for_mxfp4_activations():
+    d0, d1 = _dims(act_mode=0), _dims(act_mode=1)
+    with pytest.raises(M.MoeError, match="MOE_ACT_MXFP4"):
+        M.moe_h_operand_offsets(d0)
+    c, s = M.moe_h_operand_offsets(d1)
+    R, I = d1.T * d1.k, d1.I
+    # both regions lie inside the workspace, 16-byte aligned, and do not overlap
+    assert c % 16 == 0 and s % 16 == 0
+    assert c + R * I // 2 <= M.moe_workspace_size(d1) and s + R * I // 32 <= M.moe_workspace_size(d1)
+    assert c + R * I // 2 <= s or s + R * I // 32 <= c
