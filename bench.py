@@ -11,9 +11,13 @@ replica of the layer (the layer does not shard: no collective on the data
 path); timing is the max over ranks and ``value`` counts the tokens of all
 ranks ("scaling": "weak").
 
-Extra keys: ``roofline`` for the routed-expert call (moe_expert_ffn: the
-gate/up and down grouped GEMVs), timed alone in its own loop with the same
-flushing; ``cpu_baseline`` (the fp64 oracle on the host cores, rank 0 only);
+Activations: decode workloads keep bf16 activations (exact f16 operand of the
+grouped GEMVs); prefill workloads quantise them to MXFP4 for the tcgen05
+block-scaled GEMMs (``--act`` overrides).
+
+Extra keys: ``roofline`` for the routed-expert call (moe_expert_ffn), timed
+alone in its own loop with the same flushing, against HBM bandwidth or, when
+its FLOPs take longer than its bytes at peak, the FP4 tensor peak; ``cpu_baseline`` (the fp64 oracle on the host cores, rank 0 only);
 ``e2e`` (the same metric through moe_layer with the step's x copied in from
 pinned host memory and y copied back, inside the timed region); ``clocks``
 (nvidia-smi samples taken during the timed region).
@@ -62,10 +66,20 @@ def layer_bytes(w, n_active):
     return n_active * expert_bytes(w) + dense_bytes(w) + w.T * w.H * 2 + w.T * w.H * 4
 
 
-def ffn_bytes(w, n_active):
-    """Algorithmic bytes of one moe_expert_ffn call: routed weights, x_op rows, y_perm rows."""
+def ffn_bytes(w, n_active, act="bf16"):
+    """Algorithmic bytes of one moe_expert_ffn call: routed weights read once,
+    the activation operand read once, y_perm written once; with MXFP4
+    activations also h (codes + scales) written by gate/up and read by down."""
     R = w.T * w.k
+    if act == "mxfp4":
+        return (n_active * expert_bytes(w) + w.T * w.W * 17 // 32 + R * w.W * 4
+                + 2 * R * w.I * 17 // 32)
     return n_active * expert_bytes(w) + w.T * w.W * 2 + R * w.W * 4
+
+
+def ffn_flops(w):
+    """Multiply-adds x 2 of the routed experts: gate, up and down for every (token, slot)."""
+    return 2 * w.T * w.k * 3 * w.I * w.W
 
 
 def layer_flops(w):
@@ -106,6 +120,25 @@ def _peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+FP4_PER_BF16 = 4.0      # nominal dense ratio: 9 PFLOP/s FP4 / 2.25 PFLOP/s bf16
+
+
+def _fp4_peak_tflops():
+    """FP4 dense tensor peak = measured cuBLAS bf16 burst x the nominal ratio."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]) * FP4_PER_BF16, "measured bf16 burst x 4 (nominal fp4/bf16)"
+    except Exception:
+        return 1590.0 * FP4_PER_BF16, "fallback bf16 x 4 (nominal fp4/bf16)"
+
+
+def default_act(w):
+    """Prefill-sized batches quantise activations to MXFP4 for the tcgen05 block-scaled
+    MMA; decode keeps bf16 activations (f16 operand, exact)."""
+    return "mxfp4" if w.name.startswith("prefill") else "bf16"
 
 
 class ClockSampler:
@@ -181,7 +214,8 @@ def run_ours(args, w):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = synth.to_device(w)
-    dims = M.MoeDims.of(w, M.ACT_BF16)
+    act = args.act or default_act(w)
+    dims = M.MoeDims.of(w, M.ACT_MXFP4 if act == "mxfp4" else M.ACT_BF16)
     layer = M.MoeLayer(dims, {k: v for k, v in dev.items() if k != "x"})
     x = dev["x"]
     stream = torch.cuda.Stream()
@@ -202,7 +236,10 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     n_active = int((layer.counts > 0).sum())
 
-    launches_per_step = 12 + (4 if w.L else 0)   # kernels enqueued by one moe_layer call
+    # kernels enqueued by one moe_layer call: router 2, permute 2, shared expert 3,
+    # combine 1, routed experts 4 (bf16: two GEMV pairs) or 3 (mxfp4: tile list +
+    # two tcgen05 GEMMs), latent projections 4
+    launches_per_step = 8 + (3 if act == "mxfp4" else 4) + (4 if w.L else 0)
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -274,9 +311,32 @@ def run_ours(args, w):
             dist.destroy_process_group()
         return None
     peak, peak_kind = _peaks()
-    fb = ffn_bytes(w, n_active)
-    achieved = fb / (ffn_ms * 1e-3) / 1e9
+    fb = ffn_bytes(w, n_active, act)
     lb = layer_bytes(w, n_active)
+    ff = ffn_flops(w)
+    hbm_gbs = fb / (ffn_ms * 1e-3) / 1e9
+    if act == "mxfp4":
+        tpeak, tkind = _fp4_peak_tflops()
+        tflops = ff / (ffn_ms * 1e-3) / 1e12
+        t_mem, t_tc = fb / (peak * 1e9), ff / (tpeak * 1e12)
+        kernel = "moe_expert_ffn (k_tile_list + k_mxf4_gemm<gate/up> + k_mxf4_gemm<down>)"
+        if t_tc > t_mem:
+            roof = {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": tflops / tpeak, "peak_kind": tkind}
+        else:
+            roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peak, "unit": "GB/s",
+                    "frac": hbm_gbs / peak, "peak_kind": peak_kind}
+        roof.update({"hbm_frac": hbm_gbs / peak, "tensor_frac": tflops / tpeak,
+                     "tensor_tflops": tflops, "fp4_peak_tflops": tpeak,
+                     "roofline_ms": max(t_mem, t_tc) * 1e3,
+                     "frac_of_roofline_time": max(t_mem, t_tc) / (ffn_ms * 1e-3)})
+    else:
+        kernel = "moe_expert_ffn (k_fma_gemv + k_gateup_mxfp4 + k_down_mxfp4)"
+        roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peak, "unit": "GB/s",
+                "frac": hbm_gbs / peak, "peak_kind": peak_kind}
+    roof = dict({"kernel": kernel}, **roof)
+    roof.update({"bytes_per_launch": fb, "flops_per_launch": ff, "ms_per_launch": ffn_ms,
+                 "traffic": _traffic(w.name)})
     tokens = w.T * world
     out = {
         "metric": METRIC,
@@ -289,19 +349,16 @@ def run_ours(args, w):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "mxfp4 weights x f16 activations, fp32 accumulate",
+        "dtype": ("mxfp4 weights x mxfp4 activations (tcgen05 kind::mxf4), fp32 accumulate"
+                  if act == "mxfp4" else "mxfp4 weights x f16 activations, fp32 accumulate"),
         "data": "synthetic (seeded; BASELINE distributions)",
         "config": {"workload": workload_label(w), "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB write, outside the events)",
-                   "act_mode": "bf16", "active_experts": n_active},
+                   "act_mode": act, "active_experts": n_active},
         "layer": {"algorithmic_bytes": lb, "hbm_gbs": lb / (step_ms * 1e-3) / 1e9,
                   "hbm_frac": lb / (step_ms * 1e-3) / 1e9 / peak,
                   "tflops": layer_flops(w) / (step_ms * 1e-3) / 1e12},
-        "roofline": {"kernel": "moe_expert_ffn (k_gateup_mxfp4 + k_down_mxfp4)",
-                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind,
-                     "bytes_per_launch": fb, "ms_per_launch": ffn_ms,
-                     "traffic": _traffic(w.name)},
+        "roofline": roof,
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
@@ -311,7 +368,7 @@ def run_ours(args, w):
                        "flushed step on either side",
     }
     if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w)
+        out["cpu_baseline"] = cpu_baseline(w, act=act)
     if world > 1:
         del graph
         dist.destroy_process_group()
@@ -327,13 +384,13 @@ def _oracle_threads():
         return 1
 
 
-def _oracle_token_pass(w, t, dense, getter):
+def _oracle_token_pass(w, t, dense, getter, act="bf16"):
     import oracle as O
     sub = dict(dense, x=dense["x"][t:t + 1])
-    return O.moe_layer(sub, w.k, getter)
+    return O.moe_layer(sub, w.k, getter, act="mxfp4" if act == "mxfp4" else "exact")
 
 
-def cpu_baseline(w, budget_s: float = 20.0):
+def cpu_baseline(w, budget_s: float = 20.0, act: str = "bf16"):
     """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
     tokens of the same batch, one at a time, until about ``budget_s`` seconds."""
     from mxfp4_routed_expert_04_b200 import synth
@@ -349,7 +406,7 @@ def cpu_baseline(w, budget_s: float = 20.0):
     t0 = time.perf_counter()
     n = 0
     while n < w.T and (n == 0 or time.perf_counter() - t0 < budget_s):
-        _oracle_token_pass(w, n, dense, getter)
+        _oracle_token_pass(w, n, dense, getter, act)
         n += 1
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": "tokens/s", "cores": _oracle_threads(), "kind": "oracle",
@@ -372,15 +429,16 @@ def run_reference(args, w):
                 + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
                 + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
 
+    act = args.act or default_act(w)
     # each step is one token's full layer pass; keep the whole run within a few minutes
     t0 = time.perf_counter()
-    _oracle_token_pass(w, 0, dense, getter)            # one warm-up pass (also sizes the run)
+    _oracle_token_pass(w, 0, dense, getter, act)       # one warm-up pass (also sizes the run)
     per = time.perf_counter() - t0
     steps = max(1, min(args.steps, int(200.0 / max(per, 1e-3))))
     times = []
     for i in range(steps):
         t0 = time.perf_counter()
-        _oracle_token_pass(w, i % w.T, dense, getter)
+        _oracle_token_pass(w, i % w.T, dense, getter, act)
         times.append(time.perf_counter() - t0)
     step = statistics.mean(times)
     v = 1.0 / step
@@ -390,7 +448,7 @@ def run_reference(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; BASELINE distributions)",
         "config": {"workload": workload_label(w), "parallelism": "host cores, rank 0",
-                   "step": "one token of the batch through the whole layer"},
+                   "act_mode": act, "step": "one token of the batch through the whole layer"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _oracle_threads(),
                          "kind": "oracle",
                          "sample": f"{steps} single-token layer passes of {w.name} "
@@ -407,6 +465,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--act", choices=["bf16", "mxfp4"], default=None,
+                    help="activation operand of the routed experts (default: mxfp4 for "
+                         "prefill workloads, bf16 otherwise)")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: keep only this many experts resident (same shapes "
                          "and top-k); the line is then not the workload's metric")
