@@ -283,9 +283,11 @@ def run_ours(args, w):
         step_ms = float(t.item())
 
     # dominant call alone: moe_expert_ffn on the routing of the captured step
+    lw = layer.w      # the layer's weights (tiled scales for mxfp4 activations)
+
     def ffn():
-        M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.expert_list, layer.row_token, dev["wg_q"],
-                         dev["wg_s"], dev["wu_q"], dev["wu_s"], dev["wd_q"], dev["wd_s"],
+        M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.expert_list, layer.row_token, lw["wg_q"],
+                         lw["wg_s"], lw["wu_q"], lw["wu_s"], lw["wd_q"], lw["wd_s"],
                          layer.y_perm, layer.ws, stream)
     timed(ffn, 3)
     ffn_ms = statistics.mean(timed(ffn, max(5, args.steps)))
@@ -471,6 +473,8 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: keep only this many experts resident (same shapes "
                          "and top-k); the line is then not the workload's metric")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling case: this many tokens instead of the workload's T")
     args = ap.parse_args()
     import dataclasses
 
@@ -478,6 +482,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.experts:
         w = dataclasses.replace(w, E=args.experts, name=f"{w.name}-E{args.experts}")
+    if args.tokens:
+        w = dataclasses.replace(w, T=args.tokens, name=f"{w.name}-T{args.tokens}")
     res = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if res is not None:
         print(json.dumps(res), flush=True)

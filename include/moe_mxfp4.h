@@ -153,14 +153,26 @@ moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const uint
  * ascending order (the work list of the expert kernels). row_token[r] / row_slot[r]
  * give the pair at permuted row r; slot_row[t, j] the row of pair (t, j).
  * It also writes the activation operand x_op from x_in ([T, W] bf16: x, or
- * x_lat for latent layers), ONE ROW PER TOKEN; the expert kernels gather the
- * rows they need through row_token, so no duplicated [T*k, W] copy is made.
- *   x_op format, MOE_ACT_BF16: f16 values [T, W], then (at the next 256-byte
+ * x_lat for latent layers).
+ *   x_op format, MOE_ACT_BF16: ONE ROW PER TOKEN (the grouped GEMVs gather
+ *     rows through row_token): f16 values [T, W], then (at the next 256-byte
  *     boundary) fp32 row scales [T]: value = f16 * scale, the scale a power of
  *     two that maps the row's largest magnitude into [2^14, 2^15).
- *   x_op format, MOE_ACT_MXFP4: codes [T, W/2] uint8 (low nibble first), then
- *     (at the next 256-byte boundary) E8M0 scale codes [T, W/32] uint8 (OCP MX
- *     v1.0 conversion, ties to even).
+ *   x_op format, MOE_ACT_MXFP4: ONE ROW PER PERMUTED ROW, ready for the tensor
+ *     cores (offsets of the parts from moe_mxf4_layout_of):
+ *       codes [T*k, W/2] uint8 (low nibble = even element; OCP MX v1.0
+ *         conversion of the token's bf16 row, ties to even), row r = token
+ *         row_token[r];
+ *       E8M0 scales in the TILED layout below, K = W;
+ *       the tile list: tiles[t] = {expert, first permuted row, rows, 0} int32x4,
+ *         each expert's rows cut into tiles of at most tile_rows consecutive
+ *         rows, experts in expert_list order; tile_base[e] int32 = the first
+ *         tile of active expert e; n_tiles int32 = number of tiles.
+ *   TILED scale layout (what tcgen05 block-scaled MMAs read): for row n of
+ *     tile t (0 <= n < 128) and K-block j (32 elements), the byte at
+ *     (t * K/128 + j/4) * 512 + 16*(n % 32) + 4*(n / 32) + j % 4. For weight
+ *     matrices the tiles are the 128-row blocks (t = row / 128, n = row % 128),
+ *     see moe_tile_scales.
  *   topk_idx [T, k] int32; counts [E], offsets [E+1], expert_list [E+1],
  *   row_token [T*k], row_slot [T*k], slot_row [T, k] int32 (out);
  *   x_op moe_x_op_size() bytes (out)
@@ -176,6 +188,10 @@ moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint
  *   y_perm[r] = Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) )      [W] fp32
  * Weights in the canonical MXFP4 layout above, decoded exactly (E2M1 value x
  * E8M0 scale); products accumulate in fp32.
+ * MOE_ACT_MXFP4 (tcgen05 block-scaled MMAs): x and h = silu(Wg x) * (Wu x)
+ * enter their products as MXFP4 (h quantised per 32-element block along I);
+ * wg_s, wu_s and wd_s must then be in the TILED layout (moe_tile_scales of the
+ * canonical [E*N, K/32] arrays); the codes keep the canonical layout.
  *   x_op, offsets, expert_list, row_token as written by moe_permute;
  *   y_perm [T*k, W] fp32 (out)
  */
@@ -186,17 +202,27 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
                           const uint8_t* wd_q, const uint8_t* wd_s,
                           float* y_perm, void* ws, size_t ws_bytes, void* stream);
 
-/* --- inspection of the intermediate activation h ----------------------------
- * (No counterpart in the pages: a test and debugging aid of this library.)
- * Byte offsets inside the workspace where moe_expert_ffn leaves, for
- * MOE_ACT_MXFP4, the MXFP4 encoding of h = silu(Wg x) * (Wu x) exactly as the
- * down projection consumed it: codes [T*k, I/2] uint8 (low nibble = even
- * element) at *codes_off and E8M0 scale codes [T*k, I/32] uint8 at
- * *scales_off, rows in permuted order. Valid until the next call that uses
- * the workspace. MOE_ACT_BF16 keeps h in an internal form and returns
- * MOE_ERR_UNSUPPORTED_SHAPE; NULL outputs return MOE_ERR_INVALID_ARG.
+/* --- MXFP4 tensor-core operands ----------------------------------------------
+ * (No counterpart in the pages: data layout of this library.)
+ * moe_tile_scales: canonical row-major E8M0 scales [rows, K/32] (src) -> the
+ * TILED layout with 128-row tiles (dst, the same rows*K/32 bytes), as
+ * moe_expert_ffn / moe_layer take them for MOE_ACT_MXFP4. rows and K
+ * multiples of 128; enqueued on `stream`; src and dst device pointers.
  */
-moe_status moe_h_operand_offsets(const moe_dims* dims, size_t* codes_off, size_t* scales_off);
+moe_status moe_tile_scales(const uint8_t* src, int64_t rows, int32_t K, uint8_t* dst, void* stream);
+
+/* Byte offsets of the MOE_ACT_MXFP4 operands, for inspection and tests:
+ * inside x_op: x_codes, x_scales (tiled), tiles, tile_base, n_tiles (see
+ * moe_permute); inside the workspace, where moe_expert_ffn leaves h exactly as
+ * the down projection consumed it: h_codes [T*k, I/2] uint8 and h_scales
+ * (tiled, K = I, tiles of the tile list). Valid until the next call that uses
+ * the buffer. MOE_ACT_BF16 returns MOE_ERR_UNSUPPORTED_SHAPE. */
+typedef struct {
+  size_t x_codes, x_scales, tiles, tile_base, n_tiles;   /* in x_op */
+  size_t h_codes, h_scales;                              /* in the workspace */
+  int32_t max_tiles, tile_rows;
+} moe_mxf4_layout;
+moe_status moe_mxf4_layout_of(const moe_dims* dims, moe_mxf4_layout* out);
 
 /* --- a8-a9 (+a10 up): shared expert and combine ------------------------------
  *   s_t = sigmoid(w_sgate . x_t) * Ws_down (silu(Ws_gate x_t) * (Ws_up x_t))

@@ -17,7 +17,7 @@ __all__ = [
     "MoeError", "MoeDims", "MoeLayerArgs", "ACT_BF16", "ACT_MXFP4", "library_path",
     "moe_status_string", "moe_workspace_size", "moe_x_op_size", "moe_workspace_init",
     "moe_device_status", "moe_route", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
-    "moe_latent_down", "moe_layer", "moe_h_operand_offsets", "MoeLayer",
+    "moe_latent_down", "moe_layer", "moe_mxf4_layout_of", "moe_tile_scales", "MoeLayer",
 ]
 
 ACT_BF16 = 0
@@ -81,7 +81,8 @@ _sigs = {
     "moe_combine": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_latent_down": [_D, _P, _P, _P, _P, _Z, _P],
     "moe_layer": [_D, ctypes.POINTER(MoeLayerArgs), _P, _Z, _P],
-    "moe_h_operand_offsets": [_D, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)],
+    "moe_mxf4_layout_of": [_D, ctypes.c_void_p],
+    "moe_tile_scales": [_P, ctypes.c_int64, ctypes.c_int32, _P, _P],
 }
 for _n, _a in _sigs.items():
     getattr(_lib, _n).argtypes = _a
@@ -127,11 +128,24 @@ def moe_x_op_size(dims: MoeDims) -> int:
     return _lib.moe_x_op_size(ctypes.byref(dims))
 
 
-def moe_h_operand_offsets(dims) -> tuple:
-    """Workspace byte offsets of the MXFP4 h operand (codes, scales); MOE_ACT_MXFP4 only."""
-    c, s = ctypes.c_size_t(), ctypes.c_size_t()
-    _check(_lib.moe_h_operand_offsets(ctypes.byref(dims), ctypes.byref(c), ctypes.byref(s)))
-    return c.value, s.value
+class MoeMxf4Layout(ctypes.Structure):
+    _fields_ = [("x_codes", ctypes.c_size_t), ("x_scales", ctypes.c_size_t),
+                ("tiles", ctypes.c_size_t), ("tile_base", ctypes.c_size_t),
+                ("n_tiles", ctypes.c_size_t), ("h_codes", ctypes.c_size_t),
+                ("h_scales", ctypes.c_size_t), ("max_tiles", ctypes.c_int32),
+                ("tile_rows", ctypes.c_int32)]
+
+
+def moe_mxf4_layout_of(dims) -> MoeMxf4Layout:
+    """Byte offsets of the MOE_ACT_MXFP4 operands inside x_op and the workspace."""
+    out = MoeMxf4Layout()
+    _check(_lib.moe_mxf4_layout_of(ctypes.byref(dims), ctypes.addressof(out)))
+    return out
+
+
+def moe_tile_scales(src, rows: int, K: int, dst, stream=None):
+    """Canonical E8M0 scales [rows, K/32] -> the tiled layout of the tensor-core path."""
+    _check(_lib.moe_tile_scales(_ptr(src), int(rows), int(K), _ptr(dst), _stream(stream)))
 
 
 def moe_workspace_init(dims, ws, stream=None):
@@ -205,15 +219,23 @@ class MoeLayer:
     ``weights``: dict of device tensors (x excluded) named like the C ABI
     (w_router, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, w_sgate, ws_gate, ws_up,
     ws_down and, for latent layers, w_lat_down, w_lat_up); bf16 tensors as
-    int16/uint16 bit patterns or torch.bfloat16.
+    int16/uint16 bit patterns or torch.bfloat16. Scales in the canonical
+    layout; for ACT_MXFP4 the layer keeps tiled copies (moe_tile_scales) in
+    ``self.w``, the weights every call uses.
     """
 
     def __init__(self, dims: MoeDims, weights: dict, device="cuda"):
         self.dims = dims
-        self.w = weights
         d, T, k = dims, dims.T, dims.k
         W = d.L if d.L else d.H
         R = T * k
+        self.w = dict(weights)
+        if d.act_mode == ACT_MXFP4:
+            for name, rows, K in (("wg_s", d.E * d.I, W), ("wu_s", d.E * d.I, W),
+                                  ("wd_s", d.E * W, d.I)):
+                tiled = torch.empty_like(weights[name])
+                moe_tile_scales(weights[name], rows, K, tiled)
+                self.w[name] = tiled
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
         f32 = dict(dtype=torch.float32, device=dev)

@@ -51,9 +51,9 @@ struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   int S_router, S_sgu, S_sd, S_ld, S_lu;
   size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_hs, off_gl, off_sd, off_ld,
-      off_ylat, off_lu, off_tiles, off_ntiles, total;
+      off_ylat, off_lu, off_hsf, total;
   int max_tiles;
-  size_t xop_bytes, xop_scale_off;
+  size_t xop_bytes, xop_scale_off, xop_tiles_off, xop_tbase_off, xop_ntiles_off;
 };
 
 moe_status check_dims(const moe_dims* d) {
@@ -103,18 +103,22 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
   p.off_ylat = take(p.L ? (size_t)p.T * p.L * 4 : 0);
   p.off_lu = take(p.L ? (size_t)p.S_lu * p.T * p.H * 4 : 0);
-  // MXFP4 activations: tile list of the tensor-core GEMM (h codes and scales
-  // reuse the h16 / hscale regions, which are larger)
-  p.max_tiles = p.mode == MOE_ACT_MXFP4 ? p.R / 128 + std::min(p.E, p.R) + 1 : 0;
-  p.off_tiles = take((size_t)p.max_tiles * 16);
-  p.off_ntiles = take(p.mode == MOE_ACT_MXFP4 ? 16 : 0);
+  // MXFP4 activations: tiles of at most kTileRows rows of one expert; the sum
+  // over experts of ceil(rows / kTileRows) is below R / kTileRows + (experts) + 1.
+  // h codes reuse the h16 region (larger); h scales are tiled.
+  p.max_tiles = p.mode == MOE_ACT_MXFP4 ? p.R / moe::kTileRows + std::min(p.E, p.R) + 1 : 0;
+  p.off_hsf = take((size_t)p.max_tiles * (p.I / 128) * 512);
   p.total = o;
   if (p.mode == MOE_ACT_BF16) {
     p.xop_scale_off = align_up((size_t)p.T * p.W * 2, 256);
     p.xop_bytes = p.xop_scale_off + (size_t)p.T * 4;
+    p.xop_tiles_off = p.xop_tbase_off = p.xop_ntiles_off = 0;
   } else {
-    p.xop_scale_off = align_up((size_t)p.T * p.W / 2, 256);
-    p.xop_bytes = p.xop_scale_off + (size_t)p.T * (p.W / 32);
+    p.xop_scale_off = align_up((size_t)p.R * p.W / 2, 256);
+    p.xop_tiles_off = align_up(p.xop_scale_off + (size_t)p.max_tiles * (p.W / 128) * 512, 256);
+    p.xop_tbase_off = align_up(p.xop_tiles_off + (size_t)p.max_tiles * 16, 256);
+    p.xop_ntiles_off = align_up(p.xop_tbase_off + (size_t)p.E * 4, 256);
+    p.xop_bytes = p.xop_ntiles_off + 16;
   }
   return MOE_OK;
 }
@@ -224,8 +228,13 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
     moe::k_act_to_f16<<<p.T, 256, 0, st>>>(xin, p.W, static_cast<__half*>(x_op),
                                             at<float>(x_op, p.xop_scale_off));
   } else {
-    moe::k_act_to_mxfp4<<<p.T, 256, 0, st>>>(xin, p.W, static_cast<uint8_t*>(x_op),
-                                              at<uint8_t>(x_op, p.xop_scale_off));
+    moe::k_tile_list<<<1, 1024, 0, st>>>(offsets, expert_list, at<int4>(x_op, p.xop_tiles_off),
+                                         at<int32_t>(x_op, p.xop_tbase_off),
+                                         at<int32_t>(x_op, p.xop_ntiles_off));
+    if ((s = launched("tile list")) != MOE_OK) return s;
+    moe::k_act_to_mxfp4_perm<<<p.T, 256, 0, st>>>(
+        xin, p.W, p.k, idx, slot_row, offsets, expert_list, at<int32_t>(x_op, p.xop_tbase_off),
+        static_cast<uint8_t*>(x_op), at<uint8_t>(x_op, p.xop_scale_off));
   }
   return launched("activation operand");
 }
@@ -295,15 +304,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D map over a [rows, row_bytes] uint8 matrix read in boxes of 128 rows x
-// 128 bytes with the 128-byte swizzle (row_bytes a multiple of 64).
-moe_status weight_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
-                      const char* what) {
+// 2-D map over a [rows, row_bytes] uint8 matrix read in boxes of box_rows
+// rows x 128 bytes with the 128-byte swizzle (row_bytes a multiple of 64).
+moe_status code_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_rows, const char* what) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {row_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -313,48 +322,48 @@ moe_status weight_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64
   return MOE_OK;
 }
 
-// MXFP4 activations: tile list, then gate/up (+ SwiGLU, h quantised to MXFP4)
-// and down on the tensor cores, one persistent CTA per SM each.
+// MXFP4 activations: gate/up (+ SwiGLU, h quantised to MXFP4) and down on the
+// tensor cores, one persistent CTA per SM each; the tile list and the token
+// operand come from moe_permute (inside x_op), weight scales are tiled.
 moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* x_op,
-                              const int32_t* offsets, const int32_t* expert_list,
-                              const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
-                              const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
-                              const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
-  int4* tiles = at<int4>(ws, p.off_tiles);
-  int32_t* n_tiles = at<int32_t>(ws, p.off_ntiles);
-  moe::k_tile_list<<<1, 1024, 0, st>>>(offsets, expert_list, tiles, n_tiles);
-  moe_status s = launched("tile list");
-  if (s != MOE_OK) return s;
+                              const uint8_t* wg_q, const uint8_t* wg_s, const uint8_t* wu_q,
+                              const uint8_t* wu_s, const uint8_t* wd_q, const uint8_t* wd_s,
+                              float* y_perm, void* ws, cudaStream_t st) {
+  void* xop = const_cast<void*>(x_op);
+  const int4* tiles = at<int4>(xop, p.xop_tiles_off);
+  const int32_t* n_tiles = at<int32_t>(xop, p.xop_ntiles_off);
   uint8_t* hq = at<uint8_t>(ws, p.off_h16);
-  uint8_t* hs = at<uint8_t>(ws, p.off_hscale);
+  uint8_t* hs = at<uint8_t>(ws, p.off_hsf);
+  moe_status s;
   moe::Mxf4GemmArgs g;
   memset(&g, 0, sizeof(g));
-  if ((s = weight_map(&g.map_a0, wg_q, (uint64_t)p.E * p.I, p.W / 2, "gate weights")) != MOE_OK ||
-      (s = weight_map(&g.map_a1, wu_q, (uint64_t)p.E * p.I, p.W / 2, "up weights")) != MOE_OK)
+  if ((s = code_map(&g.map_a0, wg_q, (uint64_t)p.E * p.I, p.W / 2, 128, "gate weights")) != MOE_OK ||
+      (s = code_map(&g.map_a1, wu_q, (uint64_t)p.E * p.I, p.W / 2, 128, "up weights")) != MOE_OK ||
+      (s = code_map(&g.map_b, static_cast<const uint8_t*>(x_op), (uint64_t)p.R, p.W / 2,
+                    moe::kTileRows, "token codes")) != MOE_OK)
     return s;
   g.sa0 = wg_s; g.sa1 = wu_s;
-  g.bq = static_cast<const uint8_t*>(x_op);
-  g.bs = static_cast<const uint8_t*>(x_op) + p.xop_scale_off;
-  g.row_token = row_token;
+  g.bs = at<uint8_t>(xop, p.xop_scale_off);
   g.tiles = tiles; g.n_tiles = n_tiles;
   g.hq = hq; g.hs = hs;
   g.status = at<int32_t>(ws, p.off_status);
   g.K = p.W; g.M = p.I;
-  moe::k_mxf4_gemm<true><<<ds.num_sms, 256, moe::mxf4_gemm_smem_bytes(true), st>>>(g);
+  const int threads = moe::mxf4_gemm_threads();
+  moe::k_mxf4_gemm<true><<<ds.num_sms, threads, moe::mxf4_gemm_smem_bytes(true), st>>>(g);
   if ((s = launched("expert gate/up (tcgen05)")) != MOE_OK) return s;
   moe::Mxf4GemmArgs d;
   memset(&d, 0, sizeof(d));
-  if ((s = weight_map(&d.map_a0, wd_q, (uint64_t)p.E * p.W, p.I / 2, "down weights")) != MOE_OK)
+  if ((s = code_map(&d.map_a0, wd_q, (uint64_t)p.E * p.W, p.I / 2, 128, "down weights")) != MOE_OK ||
+      (s = code_map(&d.map_b, hq, (uint64_t)p.R, p.I / 2, moe::kTileRows, "h codes")) != MOE_OK)
     return s;
   d.map_a1 = d.map_a0;
   d.sa0 = wd_s; d.sa1 = wd_s;
-  d.bq = hq; d.bs = hs;
-  d.row_token = nullptr;
+  d.bs = hs;
   d.tiles = tiles; d.n_tiles = n_tiles;
   d.y = y_perm;
   d.status = g.status;
   d.K = p.I; d.M = p.W;
-  moe::k_mxf4_gemm<false><<<ds.num_sms, 256, moe::mxf4_gemm_smem_bytes(false), st>>>(d);
+  moe::k_mxf4_gemm<false><<<ds.num_sms, threads, moe::mxf4_gemm_smem_bytes(false), st>>>(d);
   return launched("expert down (tcgen05)");
 }
 
@@ -364,8 +373,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
                          const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
   if (p.mode == MOE_ACT_MXFP4)
-    return do_expert_ffn_mxf4(p, ds, x_op, offsets, expert_list, row_token, wg_q, wg_s, wu_q, wu_s,
-                              wd_q, wd_s, y_perm, ws, st);
+    return do_expert_ffn_mxf4(p, ds, x_op, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st);
   const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
   moe::GateUpArgs g;
   g.x16 = static_cast<const __half*>(x_op);
@@ -494,16 +502,36 @@ size_t moe_x_op_size(const moe_dims* dims) {
   return make_plan(dims, p) == MOE_OK ? p.xop_bytes : 0;
 }
 
-moe_status moe_h_operand_offsets(const moe_dims* dims, size_t* codes_off, size_t* scales_off) {
+moe_status moe_mxf4_layout_of(const moe_dims* dims, moe_mxf4_layout* out) {
   Plan p;
   moe_status s = make_plan(dims, p);
   if (s != MOE_OK) return s;
-  if (!codes_off || !scales_off) return fail(MOE_ERR_INVALID_ARG, "output pointer is NULL");
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
   if (p.mode != MOE_ACT_MXFP4)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "h is exposed only for MOE_ACT_MXFP4");
-  *codes_off = p.off_h16;
-  *scales_off = p.off_hscale;
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "the layout applies to MOE_ACT_MXFP4 only");
+  out->x_codes = 0;
+  out->x_scales = p.xop_scale_off;
+  out->tiles = p.xop_tiles_off;
+  out->tile_base = p.xop_tbase_off;
+  out->n_tiles = p.xop_ntiles_off;
+  out->h_codes = p.off_h16;
+  out->h_scales = p.off_hsf;
+  out->max_tiles = p.max_tiles;
+  out->tile_rows = moe::kTileRows;
   return MOE_OK;
+}
+
+moe_status moe_tile_scales(const uint8_t* src, int64_t rows, int32_t K, uint8_t* dst, void* stream) {
+  if (!src || !dst) return fail(MOE_ERR_INVALID_ARG, "src or dst is NULL");
+  if (!aligned16(src) || !aligned16(dst)) return fail(MOE_ERR_ALIGNMENT, "src or dst not 16-byte aligned");
+  if (rows < 128 || rows % 128 != 0 || K < 128 || K % 128 != 0 || K > (1 << 16) ||
+      rows > (1L << 31))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "rows=%lld, K=%d: rows and K must be multiples of 128",
+                (long long)rows, K);
+  const long n = rows * (K / 128);
+  const int blocks = (int)std::min<long>((n + 255) / 256, 148L * 16);
+  moe::k_tile_scales<<<blocks, 256, 0, (cudaStream_t)stream>>>(src, rows, K, dst);
+  return launched("tile scales");
 }
 
 moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream) {

@@ -67,6 +67,14 @@ MOE_DEV uint32_t e2m1_magnitude_code(float s) {
          (uint32_t)(s > 5.0f);
 }
 
+// Byte offset of scale j (K-block of 32 elements) of row n of tile `tile` in
+// the tiled scale layout read by the tcgen05 block-scaled MMAs: per tile and
+// per 128 elements of K one 512-byte block, row n at 16*(n%32) + 4*(n/32),
+// four consecutive K-blocks in four consecutive bytes.
+MOE_DEV size_t sf_tiled_offset(long tile, int k128, int n, int j) {
+  return ((size_t)tile * k128 + (j >> 2)) * 512 + 16 * (n & 31) + 4 * (n >> 5) + (j & 3);
+}
+
 // ---------------------------------------------------------------------------
 // tensor-core MMA (warp-level m16n8k16, fp32 accumulate)
 // ---------------------------------------------------------------------------

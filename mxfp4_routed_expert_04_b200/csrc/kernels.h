@@ -65,29 +65,34 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, size_t stage_t
 template <int BPL, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- grouped MXFP4 GEMM on tcgen05 (many tokens per expert) ----------------
-// Weight operands are read through 2-D tensor maps over [E*M, K/2] bytes
-// (boxes of 128 rows x 128 bytes, 128-byte swizzle); their E8M0 scales are
-// [E*M, K/32]. B rows (tokens) are codes [*, K/2] and scales [*, K/32].
+// Token rows are grouped in tiles of at most kTileRows consecutive permuted
+// rows of one expert (the MMA's N side). Weight codes are read through 2-D
+// tensor maps over [E*M, K/2] bytes (boxes of 128 rows x 128 bytes, 128-byte
+// swizzle), token codes through a map over [R, K/2] (boxes of kTileRows rows);
+// all scales are in the tiled layout of sf_tiled_offset (weights: 128-row
+// tiles; tokens: the tiles of the tile list).
+constexpr int kTileRows = 112;
 struct Mxf4GemmArgs {
   CUtensorMap map_a0;        // gate/up: gate weights; down: down weights
   CUtensorMap map_a1;        // gate/up: up weights
-  const uint8_t* sa0;
+  CUtensorMap map_b;         // token codes: x rows (gate/up) or h rows (down), [R, K/2]
+  const uint8_t* sa0;        // tiled weight scales
   const uint8_t* sa1;
-  const uint8_t* bq;         // B codes: x_op codes [T, K/2] (gate/up) or h codes [R, K/2] (down)
-  const uint8_t* bs;         // B scales
-  const int32_t* row_token;  // gate/up: B row of permuted row r; down: NULL (B row = r)
+  const uint8_t* bs;         // tiled token scales
   const int4* tiles;         // k_tile_list output
   const int32_t* n_tiles;
   uint8_t* hq;               // gate/up out: h codes [R, M/2]
-  uint8_t* hs;               // gate/up out: h scales [R, M/32]
+  uint8_t* hs;               // gate/up out: h scales, tiled (K = M)
   float* y;                  // down out: y_perm [R, M]
   int32_t* status;           // device status word
   int K, M;                  // reduction length; weight rows per expert (a multiple of 128)
 };
 __global__ void k_tile_list(const int32_t* offsets, const int32_t* expert_list, int4* tiles,
-                            int32_t* n_tiles);
+                            int32_t* tile_base, int32_t* n_tiles);
+__global__ void k_tile_scales(const uint8_t* src, long rows, int K, uint8_t* dst);
 template <bool kGateUp> __global__ void k_mxf4_gemm(const __grid_constant__ Mxf4GemmArgs a);
 size_t mxf4_gemm_smem_bytes(bool gate_up);
+int mxf4_gemm_threads();
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {
@@ -112,7 +117,10 @@ __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* coun
                           int32_t* row_slot, int32_t* slot_row, int32_t* status);
 size_t permute_smem_bytes(int E);
 __global__ void k_act_to_f16(const uint16_t* x, int W, __half* x16, float* xscale);
-__global__ void k_act_to_mxfp4(const uint16_t* x, int W, uint8_t* q, uint8_t* s);
+__global__ void k_act_to_mxfp4_perm(const uint16_t* x, int W, int k, const int32_t* idx,
+                                    const int32_t* slot_row, const int32_t* offsets,
+                                    const int32_t* expert_list, const int32_t* tile_base,
+                                    uint8_t* q, uint8_t* sf);
 
 // --- finalisers of split-K partials ----------------------------------------
 __global__ void k_shared_swiglu(const float* part, int S, int T, int Is, float* hs,

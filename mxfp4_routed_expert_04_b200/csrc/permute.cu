@@ -11,9 +11,10 @@
 // per row (the largest magnitude maps into [2^14, 2^15); bf16 values keep all
 // their bits down to 2^-29 of the row maximum).
 //
-// k_act_to_mxfp4: bf16 activation rows -> OCP MXFP4 (OCP MX v1.0 section 6.3
+// k_act_to_mxfp4_perm: bf16 activation rows -> OCP MXFP4 (the OCP MX v1.0
 // conversion: shared exponent floor(log2 amax) - 2, elements rounded to the
-// nearest E2M1 value with ties to the even code, saturating at 6).
+// nearest E2M1 value with ties to the even code, saturating at 6), written to
+// every permuted row of the token (the operand of the tensor-core path).
 #include <math.h>
 
 #include "common.cuh"
@@ -196,13 +197,33 @@ __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__
   if (threadIdx.x == 0) xscale[tok] = scale;
 }
 
-// grid T, block 256; W a multiple of 32. Each 4 consecutive threads own one
-// 32-element block (8 elements each).
-__global__ void __launch_bounds__(256) k_act_to_mxfp4(const uint16_t* __restrict__ x, int W,
-                                                    uint8_t* __restrict__ q,
-                                                    uint8_t* __restrict__ s) {
+// grid T, block 256; W a multiple of 128. MXFP4 activation operand of the
+// tensor-core path: token t's row quantised block by block (the conversion in
+// the file header) and written to each of its k permuted rows
+// r = slot_row[t, j]: codes to q[r] and scales into the tiled layout at
+// (tile, n) of row r (tile_base from k_tile_list, tiles of kTileRows
+// consecutive rows of one expert). Writes nothing when the permutation was
+// rejected (expert_list[0] == 0 then).
+__global__ void __launch_bounds__(256) k_act_to_mxfp4_perm(
+    const uint16_t* __restrict__ x, int W, int k, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ slot_row, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ expert_list, const int32_t* __restrict__ tile_base,
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  __shared__ int32_t s_row[32], s_tile[32], s_n[32];
+  if (__ldg(expert_list) == 0) return;
   const int tok = blockIdx.x;
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    const int e = __ldg(idx + (size_t)tok * k + j);
+    const int r = __ldg(slot_row + (size_t)tok * k + j);
+    const int local = r - __ldg(offsets + e);
+    s_row[j] = r;
+    s_tile[j] = __ldg(tile_base + e) + local / kTileRows;
+    s_n[j] = local % kTileRows;
+  }
+  __syncthreads();
   const uint16_t* row = x + (size_t)tok * W;
+  const int k128 = W / 128;
   for (int base = 0; base < W; base += 256 * 8) {      // uniform trip count: shuffles below
     const int i = base + threadIdx.x * 8;
     const bool ok = i < W;
@@ -231,8 +252,10 @@ __global__ void __launch_bounds__(256) k_act_to_mxfp4(const uint16_t* __restrict
       packed |= c << (4 * j);
     }
     if (ok) {
-      *reinterpret_cast<uint32_t*>(q + (size_t)tok * (W / 2) + i / 2) = packed;
-      if ((threadIdx.x & 3) == 0) s[(size_t)tok * (W / 32) + i / 32] = (uint8_t)code_s;
+      for (int j = 0; j < k; ++j) {
+        *reinterpret_cast<uint32_t*>(q + (size_t)s_row[j] * (W / 2) + i / 2) = packed;
+        if ((threadIdx.x & 3) == 0) sf[sf_tiled_offset(s_tile[j], k128, s_n[j], i / 32)] = (uint8_t)code_s;
+      }
     }
   }
 }

@@ -104,19 +104,39 @@ def test_status_strings():
 
 def test_x_op_size_by_mode():
     d0, d1 = _dims(act_mode=0), _dims(act_mode=1)
-    # f16 rows + row scales vs packed E2M1 + E8M0 block scales
+    # bf16 mode: f16 rows + row scales, one row per token (T=4, W=256)
     assert M.moe_x_op_size(d0) >= 4 * 256 * 2 + 16
-    assert M.moe_x_op_size(d1) >= 4 * 128 + 4 * 8
-    assert M.moe_x_op_size(d1) < M.moe_x_op_size(d0)
+    # mxfp4 mode: packed E2M1 + E8M0 scales, one row per permuted row (T*k = 8), + tile list
+    assert M.moe_x_op_size(d1) >= 8 * 128 + 8 * 8 + 16
 
 
-def test_h_operand_offsets_only_for_mxfp4_activations():
+def test_mxf4_layout_only_for_mxfp4_activations():
     d0, d1 = _dims(act_mode=0), _dims(act_mode=1)
     with pytest.raises(M.MoeError, match="MOE_ACT_MXFP4"):
-        M.moe_h_operand_offsets(d0)
-    c, s = M.moe_h_operand_offsets(d1)
-    R, I = d1.T * d1.k, d1.I
-    # both regions lie inside the workspace, 16-byte aligned, and do not overlap
-    assert c % 16 == 0 and s % 16 == 0
-    assert c + R * I // 2 <= M.moe_workspace_size(d1) and s + R * I // 32 <= M.moe_workspace_size(d1)
-    assert c + R * I // 2 <= s or s + R * I // 32 <= c
+        M.moe_mxf4_layout_of(d0)
+    lay = M.moe_mxf4_layout_of(d1)
+    R, W, I = d1.T * d1.k, d1.H, d1.I
+    assert lay.tile_rows == 112 and lay.max_tiles >= (R + lay.tile_rows - 1) // lay.tile_rows
+    # x_op parts in order, 256-byte aligned, inside moe_x_op_size
+    parts = [lay.x_codes, lay.x_scales, lay.tiles, lay.tile_base, lay.n_tiles]
+    assert parts == sorted(parts) and all(o % 256 == 0 for o in parts)
+    assert lay.x_scales >= R * W // 2
+    assert lay.tiles >= lay.x_scales + lay.max_tiles * (W // 128) * 512
+    assert lay.n_tiles + 4 <= M.moe_x_op_size(d1)
+    # h regions inside the workspace, disjoint
+    ws = M.moe_workspace_size(d1)
+    hc, hs = (lay.h_codes, R * I // 2), (lay.h_scales, lay.max_tiles * (I // 128) * 512)
+    assert hc[0] + hc[1] <= ws and hs[0] + hs[1] <= ws
+    assert hc[0] + hc[1] <= hs[0] or hs[0] + hs[1] <= hc[0]
+
+
+@pytest.mark.parametrize("rows,K", [(100, 256), (128, 96), (0, 128), (256, 130)])
+def test_tile_scales_rejects_bad_shapes(rows, K):
+    st = M._lib.moe_tile_scales(1 << 20, rows, K, 1 << 21, None)
+    assert st == 2
+    assert "multiples of 128" in M._lib.moe_last_error().decode()
+
+
+def test_tile_scales_rejects_null_and_misaligned():
+    assert M._lib.moe_tile_scales(None, 128, 128, 1 << 20, None) == 1
+    assert M._lib.moe_tile_scales((1 << 20) + 4, 128, 128, 1 << 20, None) == 3

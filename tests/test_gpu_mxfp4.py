@@ -50,14 +50,43 @@ def _free():
     torch.cuda.empty_cache()
 
 
-def _h_from_workspace(run):
+def _untile(buf, tiles, R, K):
+    """Canonical [R, K/32] scales from the tiled layout (the header's formula:
+    row n of tile t, K-block j at (t*K/128 + j/4)*512 + 16*(n%32) + 4*(n/32) + j%4)."""
+    out = np.zeros((R, K // 32), dtype=np.uint8)
+    j = np.arange(K // 32)[None, :]
+    for t, (e, row0, nrows, _) in enumerate(tiles):
+        n = np.arange(nrows)[:, None]
+        off = (t * (K // 128) + j // 4) * 512 + 16 * (n % 32) + 4 * (n // 32) + j % 4
+        out[row0:row0 + nrows] = buf[off]
+    return out
+
+
+def _tile_list_reference(offsets, expert_list, tile_rows):
+    tiles = []
+    for e in expert_list[1:1 + expert_list[0]]:
+        first, cnt = int(offsets[e]), int(offsets[e + 1] - offsets[e])
+        for j in range(0, cnt, tile_rows):
+            tiles.append((int(e), first + j, min(tile_rows, cnt - j), 0))
+    return np.array(tiles, dtype=np.int32).reshape(-1, 4)
+
+
+def _mxf4_operands(run, gpu):
+    """x operand, tile list and h operand of the MXFP4 path, in canonical form."""
     w, L = run.w, run.layer
-    co, so = M.moe_h_operand_offsets(run.dims)
+    lay = M.moe_mxf4_layout_of(run.dims)
     R = w.T * w.k
+    xo = gpu["x_op"]
+    n_tiles = int(xo[lay.n_tiles:lay.n_tiles + 4].view(np.int32)[0])
+    tiles = xo[lay.tiles:lay.tiles + 16 * n_tiles].view(np.int32).reshape(n_tiles, 4)
+    tile_base = xo[lay.tile_base:lay.tile_base + 4 * w.E].view(np.int32)
+    x_codes = xo[:R * w.W // 2].reshape(R, w.W // 2)
+    x_scales = _untile(xo[lay.x_scales:], tiles, R, w.W)
     ws = L.ws
-    codes = ws[co:co + R * w.I // 2].cpu().numpy().reshape(R, w.I // 2)
-    scales = ws[so:so + R * w.I // 32].cpu().numpy().reshape(R, w.I // 32)
-    return codes, scales
+    h_codes = ws[lay.h_codes:lay.h_codes + R * w.I // 2].cpu().numpy().reshape(R, w.I // 2)
+    h_buf = ws[lay.h_scales:lay.h_scales + lay.max_tiles * (w.I // 128) * 512].cpu().numpy()
+    return dict(tiles=tiles, tile_base=tile_base, tile_rows=lay.tile_rows, x_codes=x_codes,
+                x_scales=x_scales, h_codes=h_codes, h_scales=_untile(h_buf, tiles, R, w.I))
 
 
 def _unpack(packed):
@@ -73,7 +102,7 @@ def case(request):
     w, sample = request.param
     run = GpuRun(w, act_mode=M.ACT_MXFP4)
     gpu = run.run_stages()
-    gpu["h_codes"], gpu["h_scales"] = _h_from_workspace(run)
+    gpu.update(_mxf4_operands(run, gpu))
     assert M.moe_device_status(run.layer.ws) == 0
     yield w, sample, run, gpu
     del run
@@ -92,14 +121,24 @@ def test_routing_and_permutation(case):
     check_permutation(gpu, w.E)
 
 
+def test_tile_list(case):
+    w, sample, run, gpu = case
+    ref = _tile_list_reference(gpu["offsets"], gpu["expert_list"], gpu["tile_rows"])
+    np.testing.assert_array_equal(gpu["tiles"], ref)
+    firsts = {}
+    for t, (e, _, _, _) in enumerate(ref):
+        firsts.setdefault(e, t)
+    for e, t in firsts.items():
+        assert gpu["tile_base"][e] == t
+
+
 def test_x_operand_bit_exact(case):
+    """Every permuted row r holds the MXFP4 encoding of token row_token[r]."""
     w, sample, run, gpu = case
     codes, scales = O.mxfp4_quantize(O.bf16_to_f64(run.dense["x"]))
-    xo = gpu["x_op"]
-    nq = w.T * w.W // 2
-    off = (nq + 255) // 256 * 256
-    np.testing.assert_array_equal(xo[:nq].reshape(w.T, w.W // 2), O.mxfp4_pack(codes))
-    np.testing.assert_array_equal(xo[off:off + w.T * w.W // 32].reshape(w.T, w.W // 32), scales)
+    tok = gpu["row_token"]
+    np.testing.assert_array_equal(gpu["x_codes"], O.mxfp4_pack(codes)[tok])
+    np.testing.assert_array_equal(gpu["x_scales"], scales[tok])
 
 
 def _reference_h(h64, g_codes, g_scales):
@@ -214,3 +253,15 @@ def test_fused_layer_matches_stages_bitwise(case):
     w, sample, run, gpu = case
     y = run.run_layer()
     np.testing.assert_array_equal(y, gpu["y"])
+
+
+def test_tile_scales_matches_the_tiled_layout():
+    rng = np.random.default_rng(5)
+    for rows, K in ((128, 128), (384, 640), (256, 8192)):
+        src = rng.integers(0, 256, size=(rows, K // 32), dtype=np.uint8)
+        s_dev = torch.from_numpy(src).cuda()
+        d_dev = torch.empty_like(s_dev)
+        M.moe_tile_scales(s_dev, rows, K, d_dev)
+        torch.cuda.synchronize()
+        tiles = [(0, 128 * t, 128, 0) for t in range(rows // 128)]
+        np.testing.assert_array_equal(_untile(d_dev.cpu().numpy().ravel(), tiles, rows, K), src)
