@@ -18,6 +18,11 @@
 // weight and token scales as contiguous 512-byte blocks of the tiled scale
 // layout (sf_tiled_offset), which tcgen05.cp moves into tensor memory.
 //
+// Each stage carries two 128-row weight tiles that share the token tile (gate
+// and up rows for gate/up, two consecutive row tiles of Wd for down): two
+// independent accumulation chains keep the tensor pipe busy, where one chain
+// would wait on the latency of each MMA.
+//
 // Roles (192 threads, one CTA per SM):
 //   warp 0     TMA producer
 //   warp 1     allocates tensor memory; lane 0 issues scale copies and MMAs
@@ -46,8 +51,8 @@ constexpr int kThreads = 192;
 
 template <bool kGateUp>
 struct Shape {
-  static constexpr int kA = kGateUp ? 2 : 1;             // weight operands per stage
-  static constexpr int kStages = kGateUp ? 4 : 6;
+  static constexpr int kA = 2;                           // weight tiles per stage
+  static constexpr int kStages = 4;
   static constexpr int kOffB = kA * kATileBytes;
   static constexpr int kOffSfa = kOffB + kBTileBytes;
   static constexpr int kOffSfb = kOffSfa + kA * kSfBytes;
@@ -57,8 +62,8 @@ struct Shape {
   static constexpr int kBarOff = kStagesBytes + kStagingBytes;
   static constexpr int kSmem = 1024 + kBarOff + 256;     // + alignment slack of the base
   // tensor-memory columns: two accumulator buffers, then the scale factors
-  static constexpr uint32_t kAccCols = kGateUp ? 2 * kTileRows : kTileRows;
-  static constexpr uint32_t kColUp = kTileRows;          // gate/up: up accumulator in a buffer
+  static constexpr uint32_t kAccCols = 2 * kTileRows;
+  static constexpr uint32_t kColUp = kTileRows;          // second accumulator of a buffer
   static constexpr uint32_t kColSfa = 2 * kAccCols;      // kA x 8 columns
   static constexpr uint32_t kColSfb = kColSfa + 8 * kA;  // 8 columns
 };
@@ -216,7 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
   const uint32_t tbase = *tmem_slot;
 
   const int NT = __ldg(a.n_tiles);
-  const int MT = a.M / 128;
+  // gate/up: an m-tile is 128 rows of Wg and the same rows of Wu; down: 256
+  // rows of Wd as two 128-row tiles (the second absent past the last row)
+  const int MT = kGateUp ? a.M / 128 : (a.M + 255) / 256;
   const int KT = (a.K + 255) / 256;
   const int k128 = a.K / 128;                     // 512-byte scale blocks per tile row of K
   const int kb_last = (a.K - (KT - 1) * 256) / 64;     // MMAs in the last stage: 2 or 4
@@ -234,20 +241,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
       bool ok = true;
       for (long q = blockIdx.x; q < items && ok; q += gridDim.x) {
         const Item it = item_of(q, NT, a.tiles);
-        const int ya = it.tile.x * a.M + it.mt * 128;
+        const int ya = it.tile.x * a.M + it.mt * (kGateUp ? 128 : 256);
+        const bool two = kGateUp || it.mt * 256 + 128 < a.M;
         const uint8_t* sfa0 = a.sa0 + ((size_t)(ya / 128) * k128) * 512;
-        const uint8_t* sfa1 = a.sa1 + ((size_t)(ya / 128) * k128) * 512;
+        const uint8_t* sfa1 = kGateUp ? a.sa1 + ((size_t)(ya / 128) * k128) * 512
+                                      : sfa0 + (size_t)k128 * 512;
         const uint8_t* sfb = a.bs + ((size_t)it.t * k128) * 512;
         for (int kt = 0; kt < KT; ++kt) {
           if (!tc::wait_or_abort(&empty[s], ph ^ 1u, abort)) { ok = false; break; }
           uint8_t* st = smem + s * S::kStageBytes;
           const uint32_t sf_bytes = (kt == KT - 1 && kb_last == 2) ? 512u : 1024u;
-          mbar_expect_tx(&full[s], S::kA * kATileBytes + kBTileBytes + (S::kA + 1) * sf_bytes);
+          const int na = two ? 2 : 1;
+          mbar_expect_tx(&full[s], na * kATileBytes + kBTileBytes + (na + 1) * sf_bytes);
           tc::tma_load_2d(st, &a.map_a0, kt * 128, ya, &full[s]);
           if (kGateUp) tc::tma_load_2d(st + kATileBytes, &a.map_a1, kt * 128, ya, &full[s]);
+          else if (two) tc::tma_load_2d(st + kATileBytes, &a.map_a0, kt * 128, ya + 128, &full[s]);
           tc::tma_load_2d(st + S::kOffB, &a.map_b, kt * 128, it.tile.y, &full[s]);
           bulk_g2s(st + S::kOffSfa, sfa0 + kt * 1024, sf_bytes, &full[s]);
-          if (kGateUp) bulk_g2s(st + S::kOffSfa + kSfBytes, sfa1 + kt * 1024, sf_bytes, &full[s]);
+          if (two) bulk_g2s(st + S::kOffSfa + kSfBytes, sfa1 + kt * 1024, sf_bytes, &full[s]);
           bulk_g2s(st + S::kOffSfb, sfb + kt * 1024, sf_bytes, &full[s]);
           last_ph[s] = ph;
           filled[s] = true;
@@ -270,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
       const Item it = item_of(q, NT, a.tiles);
       const int npad = (it.tile.z + 15) & ~15;
       const uint32_t idesc = tc::idesc_mxf4(npad);
+      const bool two = kGateUp || it.mt * 256 + 128 < a.M;
       const int buf = n_it & 1;
       const uint32_t acc_ph = (uint32_t)((n_it >> 1) & 1);
       if (!tc::wait_or_abort(&acc_empty[buf], acc_ph ^ 1u, abort)) break;
@@ -285,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
           const int nkb = (kt == KT - 1) ? kb_last : 4;
           for (int b = 0; b < nkb / 2; ++b) {
             tc::cp_sf_block(sfa0 + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfa + b * 512)));
-            if (kGateUp)
+            if (two)
               tc::cp_sf_block(sfa1 + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfa + kSfBytes + b * 512)));
             tc::cp_sf_block(sfb + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfb + b * 512)));
           }
@@ -298,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
             const uint64_t bdesc = tc::desc_sw128(bb + 32 * kb);
             tc::mma_mxf4(d0, tc::desc_sw128(a0 + 32 * kb), bdesc, idk, (sfa0 + col) | (id << 30),
                          (sfb + col) | (id << 30), acc);
-            if (kGateUp)
+            if (two)
               tc::mma_mxf4(d1, tc::desc_sw128(a1 + 32 * kb), bdesc, idk, (sfa1 + col) | (id << 30),
                            (sfb + col) | (id << 30), acc);
           }
@@ -327,16 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
       if (!tc::wait_or_abort(&acc_full[buf], acc_ph, abort)) break;
       tc::fence_after_sync();
       const uint32_t dcol = tbase + lane_off + S::kAccCols * buf;
-      const int m0 = it.mt * 128 + 32 * wq;          // first weight row of this warp
+      const bool two = kGateUp || it.mt * 256 + 128 < a.M;
+      // first weight row of this warp (down: of its lanes in the first 128-row tile)
+      const int m0 = it.mt * (kGateUp ? 128 : 256) + 32 * wq;
       for (int c0 = 0; c0 < nrows; c0 += 32) {
         const bool last = c0 + 32 >= nrows;
         uint32_t g[32], u[32];
         if (c0 + 32 <= kTileRows) {
           tc::ld_32cols(dcol + c0, g);
-          if (kGateUp) tc::ld_32cols(dcol + S::kColUp + c0, u);
+          if (two) tc::ld_32cols(dcol + S::kColUp + c0, u);
         } else {                                     // the last 16 columns of a tile
           tc::ld_16cols(dcol + c0, g);
-          if (kGateUp) tc::ld_16cols(dcol + S::kColUp + c0, u);
+          if (two) tc::ld_16cols(dcol + S::kColUp + c0, u);
         }
         tc::wait_ld();
         if (last) {                                  // accumulators read: the MMA may reuse them
@@ -367,6 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (c < nc) yrow[(size_t)c * a.M] = __uint_as_float(g[c]);
+          if (two) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c < nc) yrow[(size_t)c * a.M + 128] = __uint_as_float(u[c]);
+          }
         }
       }
     }

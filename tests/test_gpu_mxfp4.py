@@ -13,7 +13,8 @@ tensor cores) against the fp64 oracle, stage by stage:
 
 Full-size prefill (T=4096, H=8192, I=2048, E=512, top-10) is checked on sampled
 tokens; the smaller shapes span several M, N and K tiles, ragged N tails, a K
-that is not a multiple of 256 and experts with more than 128 tokens.
+that is not a multiple of 256, a W that is not a multiple of 256 and experts
+with more than one token tile.
 """
 import gc
 
@@ -36,11 +37,14 @@ WIN_POW2 = 2e-5     # relative window of a block maximum around a power of two
 MEDIUM = synth.MoeWorkload("mx_medium", T=300, H=512, I=384, E=6, k=3, I_shared=256, seed=81)
 SKEWED = synth.MoeWorkload("mx_skewed", T=1024, H=1024, I=256, E=16, k=4, I_shared=256,
                            skew="zipf", seed=82)
+# H = 384: the down projection's last 256-row pair of Wd has a single 128-row tile
+ODD_H = synth.MoeWorkload("mx_odd_h", T=200, H=384, I=128, E=5, k=2, I_shared=128, seed=83)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
     (MEDIUM, None),
     (SKEWED, None),
+    (ODD_H, None),
     (synth.WORKLOADS["prefill4096"], [0, 1, 2047, 4095]),
 ]
 
