@@ -47,9 +47,24 @@ int dense_splits(int N, int T, int K) {
   return S;
 }
 
+// Token count from which the router and the shared expert run on the tcgen05
+// bf16 GEMM (below it the split-K GEMV streams the weights once).
+constexpr int kDenseTcTokens = 128;
+
+// K splits of the tcgen05 router GEMM: enough items for two waves of SMs,
+// each split a whole number of 64-element stages, at most 8 splits.
+int tc_splits(int N, int T, int K) {
+  const long units = (long)((N + 255) / 256) * ((T + 127) / 128);
+  int S = 1;
+  while (S < 8 && units * S < 2L * kNumSMs && (K / 64) % (2 * S) == 0) S *= 2;
+  return S;
+}
+
 struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   int S_router, S_sgu, S_sd, S_ld, S_lu;
+  bool dense_tc;             // router and shared expert on the tcgen05 bf16 GEMM
+  size_t off_hsb;            // tcgen05 shared expert: h as bf16 hi/lo [2][T, I_shared]
   size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_hs, off_gl, off_sd, off_ld,
       off_ylat, off_lu, off_hsf, total;
   int max_tiles;
@@ -84,9 +99,16 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.W = d->L ? d->L : d->H;
   p.R = d->T * d->k;
   p.mode = d->act_mode;
-  p.S_router = dense_splits(p.E, p.T, p.H);
-  p.S_sgu = dense_splits(2 * p.Is + 1, p.T, p.H);
-  p.S_sd = dense_splits(p.H, p.T, p.Is);
+  p.dense_tc = p.T >= kDenseTcTokens;
+  if (p.dense_tc) {
+    p.S_router = tc_splits(p.E, p.T, p.H);
+    p.S_sgu = 1;               // only the sigmoid-gate row stays on the GEMV
+    p.S_sd = 1;
+  } else {
+    p.S_router = dense_splits(p.E, p.T, p.H);
+    p.S_sgu = dense_splits(2 * p.Is + 1, p.T, p.H);
+    p.S_sd = dense_splits(p.H, p.T, p.Is);
+  }
   p.S_ld = p.L ? dense_splits(p.L, p.T, p.H) : 0;
   p.S_lu = p.L ? dense_splits(p.H, p.T, p.L) : 0;
   size_t o = 0;
@@ -96,8 +118,9 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_h16 = take((size_t)p.R * p.I * 2);
   p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
   p.off_h32 = take((size_t)p.R * p.I * 4);
-  p.off_sgu = take((size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
-  p.off_hs = take((size_t)p.T * p.Is * 4);
+  p.off_sgu = take(p.dense_tc ? 0 : (size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
+  p.off_hs = take(p.dense_tc ? 0 : (size_t)p.T * p.Is * 4);
+  p.off_hsb = take(p.dense_tc ? (size_t)2 * p.T * p.Is * 2 : 0);
   p.off_gl = take((size_t)p.T * 4);
   p.off_sd = take((size_t)p.S_sd * p.T * p.H * 4);
   p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
@@ -172,6 +195,9 @@ moe_status device_state(DeviceState** out) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::k_mxf4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)moe::mxf4_gemm_smem_bytes(false));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_bf16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)moe::bf16_gemm_smem_bytes());
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.gemv_ctas_per_sm, moe::k_gateup_mxfp4, 32,
@@ -204,16 +230,6 @@ moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, 
   const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (T + 31) / 32);
   moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, st>>>(a);
   return launched(what);
-}
-
-moe_status do_route(const Plan& p, const uint16_t* x, const uint16_t* wr, int32_t* idx, float* w,
-                    float* logits, void* ws, cudaStream_t st) {
-  float* part = at<float>(ws, p.off_router);
-  moe_status s = launch_dense(wr, p.E, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H,
-                              p.S_router, st, "router gemv");
-  if (s != MOE_OK) return s;
-  moe::k_topk<<<p.T, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
-  return launched("top-k");
 }
 
 moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, int32_t* counts,
@@ -304,22 +320,95 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D map over a [rows, row_bytes] uint8 matrix read in boxes of box_rows
-// rows x 128 bytes with the 128-byte swizzle (row_bytes a multiple of 64).
-moe_status code_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
-                    uint32_t box_rows, const char* what) {
+// 2-D map over a row-major [rows, cols] matrix read in boxes of box_rows rows
+// x 128 bytes with the 128-byte swizzle (a row a multiple of 16 bytes).
+moe_status tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, uint32_t elem_bytes,
+                    uint64_t rows, uint64_t cols, uint32_t box_rows, const char* what) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem_bytes};
+  const cuuint32_t box[2] = {128 / elem_bytes, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
-                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
   return MOE_OK;
+}
+
+// MXFP4 codes: [rows, row_bytes] bytes
+moe_status code_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_rows, const char* what) {
+  return tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, row_bytes, box_rows, what);
+}
+
+// bf16 matrices: [rows, cols] elements
+moe_status bf16_map(CUtensorMap* m, const uint16_t* base, uint64_t rows, uint64_t cols,
+                    const char* what) {
+  return tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 128, what);
+}
+
+moe_status launch_bf16_gemm(const DeviceState& ds, moe::Bf16GemmArgs& g, cudaStream_t st,
+                            const char* what) {
+  const long units = (long)(g.mode == moe::kBf16SwiGLU ? g.M / 128 : (g.M + 255) / 256) *
+                     ((g.T + 127) / 128) * g.S;
+  const int grid = (int)std::min<long>(units, ds.num_sms);
+  moe::k_bf16_gemm<<<grid, moe::bf16_gemm_threads(), moe::bf16_gemm_smem_bytes(), st>>>(g);
+  return launched(what);
+}
+
+moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
+                    int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st) {
+  float* part = at<float>(ws, p.off_router);
+  moe_status s;
+  if (p.dense_tc) {
+    moe::Bf16GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    if ((s = bf16_map(&g.map_a0, wr, p.E, p.H, "router weights")) != MOE_OK ||
+        (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens")) != MOE_OK)
+      return s;
+    g.out = part; g.status = at<int32_t>(ws, p.off_status);
+    g.mode = moe::kBf16Plain; g.M = p.E; g.K = p.H; g.T = p.T; g.S = p.S_router; g.passes = 1;
+    s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)");
+  } else {
+    s = launch_dense(wr, p.E, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_router, st,
+                     "router gemv");
+  }
+  if (s != MOE_OK) return s;
+  moe::k_topk<<<p.T, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
+  return launched("top-k");
+}
+
+// many tokens: SwiGLU GEMM (h as a bf16 hi/lo pair), the sigmoid-gate row on
+// the GEMV, the down GEMM over both halves of h
+moe_status do_shared_tc(const Plan& p, const DeviceState& ds, const uint16_t* x,
+                        const uint16_t* w_sgate, const uint16_t* ws_gate, const uint16_t* ws_up,
+                        const uint16_t* ws_down, void* ws, cudaStream_t st) {
+  uint16_t* h_hi = at<uint16_t>(ws, p.off_hsb);
+  uint16_t* h_lo = h_hi + (size_t)p.T * p.Is;
+  moe_status s;
+  moe::Bf16GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  if ((s = bf16_map(&g.map_a0, ws_gate, p.Is, p.H, "shared gate weights")) != MOE_OK ||
+      (s = bf16_map(&g.map_a1, ws_up, p.Is, p.H, "shared up weights")) != MOE_OK ||
+      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens")) != MOE_OK)
+    return s;
+  g.h_hi = h_hi; g.h_lo = h_lo; g.status = at<int32_t>(ws, p.off_status);
+  g.mode = moe::kBf16SwiGLU; g.M = p.Is; g.K = p.H; g.T = p.T; g.S = 1; g.passes = 1;
+  if ((s = launch_bf16_gemm(ds, g, st, "shared gate/up gemm (tcgen05)")) != MOE_OK) return s;
+  if ((s = launch_dense(w_sgate, 1, nullptr, 0, nullptr, 0, x, false, at<float>(ws, p.off_gl), p.T,
+                        p.H, 1, st, "shared gate gemv")) != MOE_OK)
+    return s;
+  moe::Bf16GemmArgs d;
+  memset(&d, 0, sizeof(d));
+  if ((s = bf16_map(&d.map_a0, ws_down, p.H, p.Is, "shared down weights")) != MOE_OK ||
+      (s = bf16_map(&d.map_b0, h_hi, p.T, p.Is, "shared h (hi)")) != MOE_OK ||
+      (s = bf16_map(&d.map_b1, h_lo, p.T, p.Is, "shared h (lo)")) != MOE_OK)
+    return s;
+  d.out = at<float>(ws, p.off_sd); d.status = g.status;
+  d.mode = moe::kBf16Plain; d.M = p.H; d.K = p.Is; d.T = p.T; d.S = 1; d.passes = 2;
+  return launch_bf16_gemm(ds, d, st, "shared down gemm (tcgen05)");
 }
 
 // MXFP4 activations: gate/up (+ SwiGLU, h quantised to MXFP4) and down on the
@@ -412,9 +501,10 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   return launched("expert down");
 }
 
-moe_status do_shared(const Plan& p, const uint16_t* x, const uint16_t* w_sgate,
+moe_status do_shared(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* w_sgate,
                      const uint16_t* ws_gate, const uint16_t* ws_up, const uint16_t* ws_down,
                      void* ws, cudaStream_t st) {
+  if (p.dense_tc) return do_shared_tc(p, ds, x, w_sgate, ws_gate, ws_up, ws_down, ws, st);
   float* sgu = at<float>(ws, p.off_sgu);
   moe_status s = launch_dense(ws_gate, p.Is, ws_up, p.Is, w_sgate, 1, x, false, sgu, p.T, p.H,
                               p.S_sgu, st, "shared gate/up gemv");
@@ -563,7 +653,9 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
   CHECK_PTR(x); CHECK_PTR(w_router); CHECK_PTR(topk_idx); CHECK_PTR(topk_w);
   if (logits && !aligned16(logits)) return fail(MOE_ERR_ALIGNMENT, "logits not 16-byte aligned");
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
-  return do_route(p, x, w_router, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  return do_route(p, *ds, x, w_router, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
 }
 
 moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
@@ -614,7 +706,9 @@ moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t*
   else if (w_lat_up) return fail(MOE_ERR_INVALID_ARG, "w_lat_up given but L == 0");
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
   const cudaStream_t st = (cudaStream_t)stream;
-  if ((s = do_shared(p, x, w_sgate, ws_gate, ws_up, ws_down, ws, st)) != MOE_OK) return s;
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  if ((s = do_shared(p, *ds, x, w_sgate, ws_gate, ws_up, ws_down, ws, st)) != MOE_OK) return s;
   return do_final(p, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
 }
 
@@ -658,12 +752,12 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
     if ((e = cudaEventRecord(ds->ev_lat, ds->side)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   }
-  if ((s = do_shared(p, a->x, a->w_sgate, a->ws_gate, a->ws_up, a->ws_down, ws, ds->side)) != MOE_OK)
+  if ((s = do_shared(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, a->ws_down, ws, ds->side)) != MOE_OK)
     return s;
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   // main stream: routing, experts, combine
-  if ((s = do_route(p, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st)) != MOE_OK) return s;
+  if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st)) != MOE_OK) return s;
   if (p.L && (e = cudaStreamWaitEvent(st, ds->ev_lat, 0)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
   if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets,

@@ -94,6 +94,26 @@ template <bool kGateUp> __global__ void k_mxf4_gemm(const __grid_constant__ Mxf4
 size_t mxf4_gemm_smem_bytes(bool gate_up);
 int mxf4_gemm_threads();
 
+// --- dense bf16 GEMM on tcgen05 (many tokens) ------------------------------
+// Weights [rows, K] and tokens [T, K] bf16 through 2-D tensor maps (boxes of
+// 128 rows x 64 elements, 128-byte swizzle). K / S a multiple of 64.
+constexpr int kBf16Plain = 0;     // out[s, t, m] fp32 partial sums over K split s
+constexpr int kBf16SwiGLU = 1;    // h = silu(Wg x) * (Wu x) as a bf16 hi/lo pair [T, M]
+struct Bf16GemmArgs {
+  CUtensorMap map_a0;        // plain: W; SwiGLU: Wg
+  CUtensorMap map_a1;        // SwiGLU: Wu
+  CUtensorMap map_b0;        // tokens (pass 0)
+  CUtensorMap map_b1;        // tokens of pass 1 (plain, passes == 2: the lo half)
+  float* out;                // plain: [S, T, M]
+  uint16_t* h_hi;            // SwiGLU: [T, M]
+  uint16_t* h_lo;
+  int32_t* status;
+  int mode, M, K, T, S, passes;
+};
+__global__ void k_bf16_gemm(const __grid_constant__ Bf16GemmArgs a);
+size_t bf16_gemm_smem_bytes();
+int bf16_gemm_threads();
+
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
 struct DenseArgs {
   const uint16_t* w[3];      // row segments of the weight matrix, each [rows, K]

@@ -28,11 +28,15 @@ from parity_harness import (TOL, GpuRun, check_permutation, check_routing, check
 MEDIUM = synth.MoeWorkload("medium_ragged", T=70, H=640, I=384, E=6, k=3, I_shared=256, seed=77)
 LATENT_SMALL = synth.MoeWorkload("latent_small", T=5, H=384, I=128, E=12, k=3, I_shared=128, L=256,
                                  seed=78)
+# T >= 128: router and shared expert on the tcgen05 bf16 GEMM (E = 6 < 128 rows,
+# I_shared = 384 = three 128-row tiles, H = 640 = two 256-row pairs + one tile)
+WIDE = synth.MoeWorkload("wide_tc", T=260, H=640, I=256, E=6, k=2, I_shared=384, seed=79)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
     (MEDIUM, None),
     (LATENT_SMALL, None),
+    (WIDE, None),
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
