@@ -256,13 +256,9 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
 }
 
 // CUDA-core GEMV launch shape for reduction length K (up to 8192): lanes own
-// BPL = ceil(K/1024) blocks; shared memory for MOE_FMA_CTAS CTAs per SM;
-// down-projection stages of about MOE_FMA_STAGE_KB KB of codes.
-#ifndef MOE_FMA_CTAS
-#define MOE_FMA_CTAS 3
-#endif
-#ifndef MOE_FMA_STAGE_KB
-#define MOE_FMA_STAGE_KB 4
+// BPL = ceil(K/1024) blocks; one CTA per SM with a ring of MOE_FMA_SMEM_KB KB.
+#ifndef MOE_FMA_SMEM_KB
+#define MOE_FMA_SMEM_KB 200
 #endif
 struct FmaPlan {
   int bpl = 0;
@@ -273,7 +269,7 @@ FmaPlan fma_plan(int K, bool gate_up) {
   const int kb = K / 32;
   f.bpl = kb <= 32 ? 1 : kb <= 64 ? 2 : kb <= 128 ? 4 : kb <= 256 ? 8 : 0;
   if (!f.bpl) return f;
-  f.g = moe::fma_geometry(K, gate_up, (216 * 1024) / MOE_FMA_CTAS, MOE_FMA_STAGE_KB * 1024);
+  f.g = moe::fma_geometry(K, gate_up, (size_t)MOE_FMA_SMEM_KB * 1024);
   return f;
 }
 // the CUDA-core path serves single-token experts when both projections fit it
@@ -285,22 +281,18 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   const FmaPlan f = fma_plan(K, kGateUp);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
   void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
-  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp>;
-  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp>;
-  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp>;
-  if (f.bpl == 8) kern = moe::k_fma_gemv<8, kGateUp>;
+  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp, kGateUp ? 1 : 8>;
+  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp, kGateUp ? 1 : 4>;
+  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp, kGateUp ? 1 : 2>;
+  if (f.bpl == 8) kern = moe::k_fma_gemv<8, kGateUp, 1>;
   if (!kern || !f.g.ok) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
-  const int threads = 32 * moe::kFmaWarps;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)f.g.smem_bytes);
-  int per_sm = 0;
-  if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, f.g.smem_bytes);
+  const int threads = 32 * (moe::kFmaConsumers + 1);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)f.g.smem_bytes);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
-  // every warp takes an equal share of the rows of the single-token experts
-  const long rows = (long)std::min(a.E, a.R) * (kGateUp ? a.I : a.W);
-  const long ctas = std::max<long>(1, std::min<long>((rows + moe::kFmaWarps - 1) / moe::kFmaWarps,
-                                                     (long)ds.num_sms * std::max(1, per_sm)));
+  // one CTA per SM, each with an equal share of the units of the single-token experts
+  const long units = (long)std::min(a.E, a.R) * (kGateUp ? a.I : a.W);
+  const long ctas = std::max<long>(1, std::min<long>((units + f.g.units - 1) / f.g.units, ds.num_sms));
   kern<<<(int)ctas, threads, f.g.smem_bytes, st>>>(a, f.g);
   return launched(what);
 }

@@ -3,30 +3,35 @@
 //
 // With one token a tensor-core MMA would use 1 of its 8 columns, and the
 // legacy mma.sync rate of sm_100 then caps the kernel near half the HBM
-// bandwidth. Here every warp works alone on a contiguous range of weight rows:
+// bandwidth. Here one CTA per SM streams a contiguous share of the weight rows
+// of all single-token experts through a ring of shared-memory stages:
 //
 // * the rows of all single-token experts form one list (gate/up: I row pairs
-//   per expert; down: W rows per expert); warp w of the grid takes the w-th
-//   equal share of it, so the load is balanced to one row and a warp reloads
-//   its activation row only when its range crosses into another expert;
-// * lane l owns the 32-element K blocks l, l+32, l+64, ... of the activation
-//   row (BPL of them), kept in registers as f16;
-// * the warp streams its rows through a private ring of shared-memory stages
-//   filled by bulk TMA copies (cp.async.bulk of the packed codes and of the
-//   covering 16-byte-aligned span of E8M0 codes) that lane 0 issues NST stages
-//   ahead, completing on one mbarrier per stage;
-// * per 32 weights a lane spends 16 cvt.rn.f16x2.e2m1x2 (exact decode) and
-//   32 fma.rn.f32.f16 (exact f16 x f16 products, fp32 sums) and one fp32 FMA
-//   for the block scale; a row's sum is a 5-step warp shuffle reduction;
-// * no barrier couples the warps after the CTA has listed the experts.
+//   per expert; down: W rows per expert); CTA c takes the c-th equal share;
+// * a producer warp fills each stage with a few large bulk TMA copies
+//   (cp.async.bulk): gate/up -> kFmaConsumers gate rows and the same up rows,
+//   down -> kFmaConsumers * RPS rows, each with the covering 16-byte-aligned
+//   span of E8M0 codes; a stage never crosses an expert, so every stage has
+//   one activation row;
+// * kFmaConsumers consumer warps share each stage: warp w takes row pair w
+//   (gate/up) or rows RPS*w .. RPS*w+RPS-1 (down); lane l owns the 32-element
+//   K blocks l, l+32, ... (BPL of them) of the activation row, kept in
+//   registers as f16;
+// * per 32 weights a lane spends 16 cvt.rn.f16x2.e2m1x2 (exact decode), 32
+//   fma.rn.f32.f16 (exact f16 x f16 products, fp32 sums) and one fp32 FMA for
+//   the block scale (E8M0 decoded without a branch, codes 0 and 255 included);
+//   the rows of a warp are computed interleaved for independent FMA chains;
+//   a row's sum is a 5-step warp shuffle reduction.
 //
 // gate/up writes h = silu(g) * u in fp32 to h32; down reads h32 of the
 // expert's token and converts it to f16 with one power-of-two scale per row
 // (the largest |h| maps into [2^14, 2^15): relative rounding <= 2^-11).
-// Every wait is bounded: on timeout the status word gets kStatusWaitTimeout
-// and the warp stops waiting (its results are then undefined).
+// Every wait is bounded: on a timeout the CTA raises an abort flag, the
+// status word gets kStatusWaitTimeout and every role stops (the results are
+// then undefined); copies in flight land before the CTA exits.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc05.cuh"
 
 namespace moe {
 
@@ -50,21 +55,11 @@ MOE_DEV float dot_block(uint4 w, const uint32_t (&x)[16]) {
   return a0 + a1;
 }
 
-// E8M0 code -> fp32 scale for codes 1..254 (one shift); codes 0 and 255 go
-// through e8m0_to_f32 (a stage holding either takes the exact path).
-MOE_DEV float e8m0_fast(uint32_t c) { return __uint_as_float(c << 23); }
-
-// true when any of the n bytes at p (16-byte aligned span) is 0x00 or 0xFF;
-// every lane checks 16-byte pieces, the warp votes
-MOE_DEV bool span_has_special(const uint8_t* p, int n, int lane) {
-  bool any = false;
-  for (int i = lane * 16; i < n; i += 32 * 16) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) any |= (__vcmpeq4(w[k], 0u) | __vcmpeq4(w[k], 0xFFFFFFFFu)) != 0u;
-  }
-  return __any_sync(0xFFFFFFFFu, any);
+// E8M0 code -> fp32 without a branch: 2^(c-127) for c = 1..254, the
+// subnormal 2^-127 for c = 0, NaN for c = 255 (0x7F800000 | 0x400000).
+MOE_DEV float e8m0_exact(uint32_t c) {
+  const uint32_t special = (c - 1u) > 253u ? 0x00400000u : 0u;
+  return __uint_as_float((c << 23) | special);
 }
 
 MOE_DEV float warp_sum(float v) {
@@ -81,25 +76,29 @@ MOE_DEV float warp_max(float v) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// block = kFmaWarps warps; grid sized so that every warp has work; dynamic
-// shared memory = kFmaWarps * g.nst * (g.stage_bytes + 8)
+// block = 32 * (kFmaConsumers + 1) threads (warp 0: producer); one CTA per SM;
+// dynamic shared memory = g.nst * g.stage_bytes
 // ---------------------------------------------------------------------------
-template <int BPL, bool kGateUp>
-__global__ void __launch_bounds__(32 * kFmaWarps, 3) k_fma_gemv(FmaArgs a, FmaGeometry g) {
+template <int BPL, bool kGateUp, int RPS>
+__global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArgs a, FmaGeometry g) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
-  __shared__ int s_wsum[kFmaWarps];
+  __shared__ int s_wsum[kFmaConsumers + 1];
+  __shared__ uint64_t s_bars[2 * kFmaMaxStages];
+  __shared__ int s_abort;
+  constexpr int kWarps = kFmaConsumers + 1;
+  constexpr int P = kGateUp ? kFmaConsumers : kFmaConsumers * RPS;   // units per stage
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int K = kGateUp ? a.W : a.I;
   const int KB = K >> 5;
-  const size_t qrow = (size_t)K / 2, srow = (size_t)K / 32;
+  const uint32_t qrow = (uint32_t)K / 2, srow = (uint32_t)K / 32;
   const int N = kGateUp ? a.I : a.W;                      // rows of one matrix
   const size_t s_total = (size_t)a.E * N * srow;          // bytes of a stacked E8M0 array
 
   // 1) the single-token experts, in the order of the expert list
   const int n_act = __ldg(a.expert_list);
   int n_single = 0;
-  for (int base = 0; base < n_act; base += 32 * kFmaWarps) {
+  for (int base = 0; base < n_act; base += 32 * kWarps) {
     const int i = base + threadIdx.x;
     int e = -1;
     if (i < n_act) {
@@ -112,201 +111,233 @@ __global__ void __launch_bounds__(32 * kFmaWarps, 3) k_fma_gemv(FmaArgs a, FmaGe
     int before = n_single;
     for (int w = 0; w < warp; ++w) before += s_wsum[w];
     if (e >= 0) s_list[before + __popc(m & ((1u << lane) - 1u))] = (int16_t)e;
-    for (int w = 0; w < kFmaWarps; ++w) n_single += s_wsum[w];
+    for (int w = 0; w < kWarps; ++w) n_single += s_wsum[w];
     __syncthreads();
   }
 
-  // 2) this warp's share of the units (gate/up: row pairs; down: rows)
-  const int total = n_single * N;                        // < 2^27
-  const int nwarps = gridDim.x * kFmaWarps;
-  const int gw = blockIdx.x * kFmaWarps + warp;
-  const int lo = (int)((long)total * gw / nwarps), hi = (int)((long)total * (gw + 1) / nwarps);
-  if (lo >= hi) return;
-  const int hi_si = hi / N, hi_r = hi - hi_si * N;       // end of the range as (expert, row)
-
-  uint8_t* ring = smem + (size_t)warp * g.nst * g.stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kFmaWarps * g.nst * g.stage_bytes) +
-                   warp * g.nst;
-  if (lane == 0) {
-    for (int i = 0; i < g.nst; ++i) mbar_init(&bars[i], 1);
+  // 2) this CTA's share of the units (gate/up: row pairs; down: rows)
+  const long total = (long)n_single * N;
+  const long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+  if (lo >= hi) return;                                   // uniform across the CTA
+  uint64_t* full = s_bars;
+  uint64_t* empty = s_bars + kFmaMaxStages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < g.nst; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kFmaConsumers);
+    }
+    s_abort = 0;
     fence_mbar_init();
   }
-  __syncwarp();
-
-  // A cursor walks the stage sequence: gate/up -> for each row pair the gate
-  // row, then the up row; down -> up to g.rps rows of one expert per stage.
-  struct Cursor { int si, r, half; };
-  auto rows_in_stage = [&](const Cursor& c) -> int {
-    if (kGateUp) return 1;
-    const int left = (c.si == hi_si) ? hi_r - c.r : N - c.r;
-    return min(g.rps, left);
+  __syncthreads();
+  volatile int* abort = &s_abort;
+  // a stage takes at most P units, never crossing an expert or the range end
+  auto stage_units = [&](long u) -> int {
+    const long end_e = (u / N + 1) * N;
+    return (int)min((long)P, min(end_e, hi) - u);
   };
-  auto advance = [&](Cursor& c, int n) {
-    if (kGateUp) {
-      c.half ^= 1;
-      if (c.half) return;
-      n = 1;
-    }
-    c.r += n;
-    if (c.r == N) { c.r = 0; ++c.si; }
-  };
-  auto done = [&](const Cursor& c) { return c.si > hi_si || (c.si == hi_si && c.r >= hi_r); };
 
-  // producer (lane 0): stage copies, g.nst ahead of the consumer
-  Cursor pc{lo / N, lo - (lo / N) * N, 0};
-  int p_v = 0;
-  auto issue_next = [&]() {
-    if (done(pc)) return;
-    const int n = rows_in_stage(pc);
-    const int e = s_list[pc.si];
-    const size_t row = (size_t)e * N + pc.r;
-    const uint8_t* q = kGateUp ? (pc.half ? a.wu_q : a.wg_q) : a.wd_q;
-    const uint8_t* sp = kGateUp ? (pc.half ? a.wu_s : a.wg_s) : a.wd_s;
-    const size_t s0 = row * srow, s1 = (row + n) * srow;
-    const size_t a0 = s0 & ~(size_t)15, a1 = min((s1 + 15) & ~(size_t)15, s_total);
-    const int slot = p_v % g.nst;
-    uint8_t* dst = ring + (size_t)slot * g.stage_bytes;
-    const uint32_t cb = (uint32_t)(n * qrow);
-    fence_proxy_async_smem();            // earlier generic reads of the slot come first
-    mbar_expect_tx(&bars[slot], cb + (uint32_t)(a1 - a0));
-    bulk_g2s(dst, q + row * qrow, cb, &bars[slot]);
-    bulk_g2s(dst + g.sbuf_off, sp + a0, (uint32_t)(a1 - a0), &bars[slot]);
-    ++p_v;
-    advance(pc, n);
-  };
-  if (lane == 0)
-    for (int i = 0; i < g.nst; ++i) issue_next();
-
-  bool dead = false;
-  int v = 0, slot = 0, phase = 0;
-  int cur_si = -1, r0 = 0;
-  uint32_t xr[BPL][16];
-  float xs = 1.0f, gsum = 0.0f;
-  Cursor c{lo / N, lo - (lo / N) * N, 0};
-  while (!done(c)) {
-    if (c.si != cur_si) {                 // new expert: load its activation row
-      cur_si = c.si;
-      const int e = s_list[c.si];
-      r0 = __ldg(a.offsets + e);
-      if (kGateUp) {
-        const int tok = __ldg(a.row_token + r0);
-        const __half* xrow = a.x16 + (size_t)tok * a.W;
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      uint32_t last_ph[kFmaMaxStages];
+      bool filled[kFmaMaxStages];
 #pragma unroll
-        for (int j = 0; j < BPL; ++j) {
-          const int b = lane + 32 * j;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 t = make_uint4(0u, 0u, 0u, 0u);
-            if (b < KB) t = ldg16(xrow + b * 32 + 8 * q);
-            xr[j][4 * q] = t.x; xr[j][4 * q + 1] = t.y; xr[j][4 * q + 2] = t.z; xr[j][4 * q + 3] = t.w;
-          }
+      for (int s = 0; s < kFmaMaxStages; ++s) { last_ph[s] = 0; filled[s] = false; }
+      int k = 0;
+      for (long u = lo; u < hi; ++k) {
+        const int n = stage_units(u);
+        const int slot = k % g.nst;
+        const uint32_t ph = (uint32_t)((k / g.nst) & 1);
+        if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) break;
+        const int si = (int)(u / N), r = (int)(u - (long)si * N);
+        const size_t row = (size_t)s_list[si] * N + r;
+        const uint32_t cb = n * qrow;
+        const size_t s0 = row * srow, s1 = (row + n) * srow;
+        const size_t a0 = s0 & ~(size_t)15, a1 = min((s1 + 15) & ~(size_t)15, s_total);
+        const uint32_t sb = (uint32_t)(a1 - a0);
+        uint8_t* st = smem + (size_t)slot * g.stage_bytes;
+        fence_proxy_async_smem();            // the consumers' reads of the slot come first
+        if (kGateUp) {
+          mbar_expect_tx(&full[slot], 2 * cb + 2 * sb);
+          bulk_g2s(st, a.wg_q + row * qrow, cb, &full[slot]);
+          bulk_g2s(st + g.code_bytes, a.wu_q + row * qrow, cb, &full[slot]);
+          bulk_g2s(st + g.sbuf_off, a.wg_s + a0, sb, &full[slot]);
+          bulk_g2s(st + g.sbuf2_off, a.wu_s + a0, sb, &full[slot]);
+        } else {
+          mbar_expect_tx(&full[slot], cb + sb);
+          bulk_g2s(st, a.wd_q + row * qrow, cb, &full[slot]);
+          bulk_g2s(st + g.sbuf_off, a.wd_s + a0, sb, &full[slot]);
         }
-        xs = __ldg(a.xscale + tok);
-      } else {
-        // h32 row -> f16 with one power-of-two scale for the row
-        const float* hrow = a.h32 + (size_t)r0 * a.I;
-        float m = 0.0f;
+        last_ph[slot] = ph;
+        filled[slot] = true;
+        u += n;
+      }
+      if (*abort) {     // let every issued copy land before the CTA can exit
+        for (int s = 0; s < g.nst; ++s)
+          if (filled[s]) mbar_wait(&full[s], last_ph[s]);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const int w = warp - 1;
+    uint32_t xr[BPL][16];
+    float xs = 1.0f;
+    int cur_e = -1, r0 = 0;
+    int k = 0;
+    for (long u = lo; u < hi; ++k) {
+      const int n = stage_units(u);
+      const int slot = k % g.nst;
+      const uint32_t ph = (uint32_t)((k / g.nst) & 1);
+      const int si = (int)(u / N), r = (int)(u - (long)si * N);
+      const int e = s_list[si];
+      if (e != cur_e) {                     // new expert: load its activation row
+        cur_e = e;
+        r0 = __ldg(a.offsets + e);
+        if (kGateUp) {
+          const int tok = __ldg(a.row_token + r0);
+          const __half* xrow = a.x16 + (size_t)tok * a.W;
 #pragma unroll
-        for (int j = 0; j < BPL; ++j) {
-          const int b = lane + 32 * j;
-          if (b < KB)
-            for (int q = 0; q < 8; ++q) {
-              const float4 t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
-              m = fmaxf(m, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+          for (int j = 0; j < BPL; ++j) {
+            const int b = lane + 32 * j;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 t = make_uint4(0u, 0u, 0u, 0u);
+              if (b < KB) t = ldg16(xrow + b * 32 + 8 * q);
+              xr[j][4 * q] = t.x; xr[j][4 * q + 1] = t.y; xr[j][4 * q + 2] = t.z; xr[j][4 * q + 3] = t.w;
             }
-        }
-        m = warp_max(m);
-        float inv = 1.0f;
-        xs = 1.0f;
-        if (m > 0.0f && isfinite(m)) {
-          int ex;
-          frexpf(m, &ex);
-          ex = max(-100, min(127, ex));
-          xs = ldexpf(1.0f, ex - 15);
-          inv = ldexpf(1.0f, 15 - ex);
-        }
+          }
+          xs = __ldg(a.xscale + tok);
+        } else {
+          // h32 row -> f16 with one power-of-two scale for the row
+          const float* hrow = a.h32 + (size_t)r0 * a.I;
+          float m = 0.0f;
 #pragma unroll
-        for (int j = 0; j < BPL; ++j) {
-          const int b = lane + 32 * j;
+          for (int j = 0; j < BPL; ++j) {
+            const int b = lane + 32 * j;
+            if (b < KB)
+              for (int q = 0; q < 8; ++q) {
+                const float4 t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+              }
+          }
+          m = warp_max(m);
+          float inv = 1.0f;
+          xs = 1.0f;
+          if (m > 0.0f && isfinite(m)) {
+            int ex;
+            frexpf(m, &ex);
+            ex = max(-100, min(127, ex));
+            xs = ldexpf(1.0f, ex - 15);
+            inv = ldexpf(1.0f, 15 - ex);
+          }
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (b < KB) t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
-            const __half2 l2 = __floats2half2_rn(t.x * inv, t.y * inv);
-            const __half2 h2 = __floats2half2_rn(t.z * inv, t.w * inv);
-            xr[j][2 * q] = *reinterpret_cast<const uint32_t*>(&l2);
-            xr[j][2 * q + 1] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int j = 0; j < BPL; ++j) {
+            const int b = lane + 32 * j;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (b < KB) t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
+              const __half2 l2 = __floats2half2_rn(t.x * inv, t.y * inv);
+              const __half2 h2 = __floats2half2_rn(t.z * inv, t.w * inv);
+              xr[j][2 * q] = *reinterpret_cast<const uint32_t*>(&l2);
+              xr[j][2 * q + 1] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
           }
         }
       }
-    }
-    const int n = rows_in_stage(c);
-    if (!dead && !mbar_wait(&bars[slot], (uint32_t)phase)) {
-      dead = true;
-      if (lane == 0) atomicOr(a.status, kStatusWaitTimeout);
-    }
-    const uint8_t* stg = ring + (size_t)slot * g.stage_bytes;
-    const int e = s_list[c.si];
-    const uint32_t soff = (uint32_t)((((size_t)e * N + c.r) * srow) & 15);
-    const uint8_t* ssc = stg + g.sbuf_off + soff;
-    // the span copied with the stage is scanned once: codes 0 / 255 are rare
-    const bool special = span_has_special(stg + g.sbuf_off, (int)((soff + n * srow + 15) & ~15u), lane);
-    for (int rr = 0; rr < n; ++rr) {
-      float acc = 0.0f;
+      if (!tc::wait_or_abort(&full[slot], ph, abort)) break;
+      const uint32_t st = smem_u32(smem + (size_t)slot * g.stage_bytes);
+      const uint32_t soff = (uint32_t)((((size_t)e * N + r) * srow) & 15u);
+      // units of this warp: gate/up -> pair w (row 0 gate, row 1 up);
+      // down -> rows RPS*w ... (codes qrow apart, scales srow apart)
+      constexpr int NR = kGateUp ? 2 : RPS;
+      const int u0 = kGateUp ? w : RPS * w;
+      float acc[NR];
 #pragma unroll
-      for (int j = 0; j < BPL; ++j) {
-        const int b = lane + 32 * j;
-        if (b < KB) {
-          const uint4 w = *reinterpret_cast<const uint4*>(stg + rr * qrow + b * 16);
-          const uint32_t code = ssc[rr * srow + b];
-          acc = fmaf(dot_block(w, xr[j]), special ? e8m0_to_f32(code) : e8m0_fast(code), acc);
+      for (int rr = 0; rr < NR; ++rr) acc[rr] = 0.0f;
+      if (u0 < n) {
+        uint32_t cb[NR], sbs[NR];
+#pragma unroll
+        for (int rr = 0; rr < NR; ++rr) {
+          if (kGateUp) {
+            cb[rr] = st + rr * g.code_bytes + u0 * qrow + 16u * lane;
+            sbs[rr] = st + (rr ? g.sbuf2_off : g.sbuf_off) + soff + u0 * srow + lane;
+          } else {
+            cb[rr] = st + (u0 + rr) * qrow + 16u * lane;
+            sbs[rr] = st + g.sbuf_off + soff + (u0 + rr) * srow + lane;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < BPL; ++j) {
+          if (lane + 32 * j < KB) {
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) {
+              if (kGateUp || u0 + rr < n) {
+                const uint4 wv = lds16(cb[rr] + 512u * j);
+                const uint32_t code = lds8(sbs[rr] + 32u * j);
+                acc[rr] = fmaf(dot_block(wv, xr[j]), e8m0_exact(code), acc[rr]);
+              }
+            }
+          }
+        }
+        if (kGateUp) {
+          const float gs = warp_sum(acc[0]), us = warp_sum(acc[1]);
+          if (lane == 0) a.h32[(size_t)r0 * a.I + r + u0] = silu_f32(gs * xs) * (us * xs);
+        } else {
+#pragma unroll
+          for (int rr = 0; rr < NR; ++rr) {
+            if (u0 + rr < n) {
+              const float sum = warp_sum(acc[rr]);
+              if (lane == 0) a.y_perm[(size_t)r0 * a.W + r + u0 + rr] = sum * xs;
+            }
+          }
         }
       }
-      const float sum = warp_sum(acc);
-      if (kGateUp) {
-        if (!c.half) gsum = sum;
-        else if (lane == 0) a.h32[(size_t)r0 * a.I + c.r] = silu_f32(gsum * xs) * (sum * xs);
-      } else if (lane == 0) {
-        a.y_perm[(size_t)r0 * a.W + c.r + rr] = sum * xs;
-      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[slot]);   // this warp is done with the slot
+      u += n;
     }
-    __syncwarp();
-    ++v;
-    if (++slot == g.nst) { slot = 0; phase ^= 1; }
-    if (lane == 0 && !dead) issue_next();  // refill the slot just consumed
-    advance(c, n);
   }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) atomicOr(a.status, kStatusWaitTimeout);
 }
 
-// Geometry for reduction length K (host side): rows per down stage rps (a
-// power of two with about stage_target bytes of codes), stage buffer size
-// (codes, then the E8M0 span with 32 bytes of alignment slack), ring depth
-// nst from the shared-memory budget per CTA.
-FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, size_t stage_target) {
+// Geometry for reduction length K (host side): rows per consumer warp in a
+// down stage rps = 8 / BPL; a stage holds kFmaConsumers units (gate/up: the
+// gate rows, then the up rows, then the two E8M0 spans; down: the codes of
+// kFmaConsumers * rps rows, then their span; every span with 32 bytes of
+// alignment slack); ring depth nst from the shared-memory budget.
+FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   FmaGeometry g{};
   const size_t qrow = K / 2, srow = K / 32;
-  int rps = 1;
-  if (!gate_up)
-    while (rps < 32 && (size_t)(2 * rps) * qrow <= stage_target) rps *= 2;
+  const int bpl = (K + 1023) / 1024;
+  if (bpl > 8) return g;
+  const int rps = gate_up ? 1 : 8 / (bpl > 4 ? 8 : bpl > 2 ? 4 : bpl > 1 ? 2 : 1);
+  const int units = gate_up ? kFmaConsumers : kFmaConsumers * rps;
   g.rps = rps;
-  g.sbuf_off = (uint32_t)((rps * qrow + 15) / 16 * 16);
-  g.stage_bytes = (uint32_t)((g.sbuf_off + rps * srow + 32 + 127) / 128 * 128);
-  const size_t per_warp = smem_budget / kFmaWarps;
-  int nst = (int)(per_warp / (g.stage_bytes + 8));
+  g.units = units;
+  g.code_bytes = (uint32_t)((units * qrow + 127) / 128 * 128);
+  const uint32_t code_all = gate_up ? 2 * g.code_bytes : g.code_bytes;
+  const uint32_t span = (uint32_t)((units * srow + 32 + 127) / 128 * 128);
+  g.sbuf_off = code_all;
+  g.sbuf2_off = code_all + span;
+  g.stage_bytes = code_all + (gate_up ? 2 : 1) * span;
+  int nst = (int)(smem_budget / g.stage_bytes);
   if (nst < 2) return g;
-  g.nst = nst > 8 ? 8 : nst;
-  g.smem_bytes = (uint32_t)(kFmaWarps * g.nst * (g.stage_bytes + 8));
+  g.nst = nst > kFmaMaxStages ? kFmaMaxStages : nst;
+  g.smem_bytes = (uint32_t)(g.nst * g.stage_bytes);
   g.ok = 1;
   return g;
 }
 
-#define MOE_FMA_INST(BPL)                                                   \
-  template __global__ void k_fma_gemv<BPL, true>(FmaArgs, FmaGeometry);    \
-  template __global__ void k_fma_gemv<BPL, false>(FmaArgs, FmaGeometry);
-MOE_FMA_INST(1)
-MOE_FMA_INST(2)
-MOE_FMA_INST(4)
-MOE_FMA_INST(8)
+#define MOE_FMA_INST(BPL, RPS)                                                 \
+  template __global__ void k_fma_gemv<BPL, true, 1>(FmaArgs, FmaGeometry);    \
+  template __global__ void k_fma_gemv<BPL, false, RPS>(FmaArgs, FmaGeometry);
+MOE_FMA_INST(1, 8)
+MOE_FMA_INST(2, 4)
+MOE_FMA_INST(4, 2)
+MOE_FMA_INST(8, 1)
 #undef MOE_FMA_INST
 
 }  // namespace moe

@@ -41,7 +41,8 @@ __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
 // CUDA-core path: experts with exactly 1 token (gemv_fma.cu)
-constexpr int kFmaWarps = 4;     // independent warps per CTA
+constexpr int kFmaConsumers = 8;   // consumer warps per CTA (plus one producer warp)
+constexpr int kFmaMaxStages = 8;
 struct FmaArgs {
   const __half* x16;         // gate/up: [T, W] f16 rows, xscale [T]
   const float* xscale;
@@ -54,15 +55,16 @@ struct FmaArgs {
   int32_t* status;           // device status word
   int W, I, E, R;
 };
-// Launch geometry: rps rows per down-projection ring stage (gate/up stages
-// hold one row), sbuf_off = offset of the E8M0 span inside a stage, nst ring
-// stages per warp.
+// Launch geometry: rps rows per consumer warp of a down stage, units per stage
+// (gate/up: row pairs; down: rows), code_bytes = one matrix's codes of a
+// stage, sbuf_off / sbuf2_off = offsets of the E8M0 spans (the second:
+// gate/up only), nst ring stages.
 struct FmaGeometry {
-  int ok, rps, nst;
-  uint32_t sbuf_off, stage_bytes, smem_bytes;
+  int ok, rps, nst, units;
+  uint32_t code_bytes, sbuf_off, sbuf2_off, stage_bytes, smem_bytes;
 };
-FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, size_t stage_target);
-template <int BPL, bool kGateUp> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
+FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget);
+template <int BPL, bool kGateUp, int RPS> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
 
 // --- grouped MXFP4 GEMM on tcgen05 (many tokens per expert) ----------------
 // Token rows are grouped in tiles of at most kTileRows consecutive permuted
