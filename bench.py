@@ -237,9 +237,10 @@ def run_ours(args, w):
     n_active = int((layer.counts > 0).sum())
 
     # kernels enqueued by one moe_layer call: router 2, permute 2, shared expert 3,
-    # combine 1, routed experts 4 (bf16: two GEMV pairs) or 3 (mxfp4: tile list +
-    # two tcgen05 GEMMs), latent projections 4
-    launches_per_step = 8 + (3 if act == "mxfp4" else 4) + (4 if w.L else 0)
+    # combine 1, routed experts 4 (bf16: two GEMV pairs; 2 for one token, whose
+    # experts all have a single token) or 3 (mxfp4: tile list + two tcgen05
+    # GEMMs), latent projections 4
+    launches_per_step = 8 + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (4 if w.L else 0)
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -169,6 +169,25 @@ moe_status launched(const char* what) {
   return MOE_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream is still running (every kernel of this
+// library waits in pdl_wait() before it reads memory), hiding the launch gap.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // per-device one-time setup: kernel attributes, the side stream and events of moe_layer
 struct DeviceState {
   bool ready = false;
@@ -219,7 +238,7 @@ moe_status device_state(DeviceState** out) {
 // ---------------------------------------------------------------------------
 moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, const uint16_t* w2,
                         int r2, const void* x, bool x_f32, float* part, int T, int K, int S,
-                        cudaStream_t st, const char* what) {
+                        cudaStream_t st, const char* what, bool pdl = true) {
   moe::DenseArgs a;
   a.w[0] = w0; a.w[1] = w1 ? w1 : w0; a.w[2] = w2 ? w2 : w0;
   a.rows[0] = r0; a.rows[1] = r1; a.rows[2] = r2;
@@ -228,21 +247,21 @@ moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, 
   a.part = part;
   a.T = T; a.K = K; a.S = S; a.kper = K / S;
   const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (T + 31) / 32);
-  moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, st>>>(a);
+  if (pdl) launch_pdl(moe::k_dense_gemv, grid, dim3(32 * moe::kDenseWarps), 0, st, a);
+  else moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, st>>>(a);
   return launched(what);
 }
 
 moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, int32_t* counts,
                       int32_t* offsets, int32_t* expert_list, int32_t* row_token, int32_t* row_slot,
                       int32_t* slot_row, void* x_op, void* ws, cudaStream_t st) {
-  moe::k_permute<<<1, 1024, moe::permute_smem_bytes(p.E), st>>>(
-      idx, p.T, p.k, p.E, counts, offsets, expert_list, row_token, row_slot, slot_row,
-      at<int32_t>(ws, p.off_status));
+  launch_pdl(moe::k_permute, dim3(1), dim3(1024), moe::permute_smem_bytes(p.E), st, idx, p.T, p.k, p.E,
+             counts, offsets, expert_list, row_token, row_slot, slot_row, at<int32_t>(ws, p.off_status));
   moe_status s = launched("permute");
   if (s != MOE_OK) return s;
   if (p.mode == MOE_ACT_BF16) {
-    moe::k_act_to_f16<<<p.T, 256, 0, st>>>(xin, p.W, static_cast<__half*>(x_op),
-                                            at<float>(x_op, p.xop_scale_off));
+    launch_pdl(moe::k_act_to_f16, dim3(p.T), dim3(256), 0, st, xin, p.W, static_cast<__half*>(x_op),
+               at<float>(x_op, p.xop_scale_off));
   } else {
     moe::k_tile_list<<<1, 1024, 0, st>>>(offsets, expert_list, at<int4>(x_op, p.xop_tiles_off),
                                          at<int32_t>(x_op, p.xop_tbase_off),
@@ -293,7 +312,7 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   // one CTA per SM, each with an equal share of the units of the single-token experts
   const long units = (long)std::min(a.E, a.R) * (kGateUp ? a.I : a.W);
   const long ctas = std::max<long>(1, std::min<long>((units + f.g.units - 1) / f.g.units, ds.num_sms));
-  kern<<<(int)ctas, threads, f.g.smem_bytes, st>>>(a, f.g);
+  launch_pdl(kern, dim3((unsigned)ctas), dim3(threads), f.g.smem_bytes, st, a, f.g);
   return launched(what);
 }
 
@@ -368,7 +387,8 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
                      "router gemv");
   }
   if (s != MOE_OK) return s;
-  moe::k_topk<<<p.T, 256, 0, st>>>(part, p.S_router, p.T, p.E, p.k, idx, w, logits);
+  launch_pdl(moe::k_topk, dim3(p.T), dim3(256), 0, st, (const float*)part, p.S_router, p.T, p.E, p.k, idx, w,
+             logits);
   return launched("top-k");
 }
 
@@ -476,20 +496,25 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   f.status = at<int32_t>(ws, p.off_status);
   f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
   g.min_tokens = fma ? 2 : 1;
+  // one token: its k experts are distinct, so every active expert has exactly
+  // one token and the tensor-core kernels would find no work
+  const bool mma = !(fma && p.T == 1);
   moe_status s = MOE_OK;
   if (fma && (s = launch_fma<true>(ds, f, st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
-  moe::k_gateup_mxfp4<<<grid_g, 32, smem, st>>>(g);
-  s = launched("expert gate/up");
-  if (s != MOE_OK) return s;
+  if (mma) {
+    launch_pdl(moe::k_gateup_mxfp4, dim3(grid_g), dim3(32), smem, st, g);
+    if ((s = launched("expert gate/up")) != MOE_OK) return s;
+  }
   moe::DownArgs d;
   d.h16 = g.h16; d.hscale = g.hscale; d.offsets = offsets; d.expert_list = expert_list;
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
   d.min_tokens = g.min_tokens;
   if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
+  if (!mma) return MOE_OK;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
-  moe::k_down_mxfp4<<<grid_d, 32, smem, st>>>(d);
+  launch_pdl(moe::k_down_mxfp4, dim3(grid_d), dim3(32), smem, st, d);
   return launched("expert down");
 }
 
@@ -499,10 +524,10 @@ moe_status do_shared(const Plan& p, const DeviceState& ds, const uint16_t* x, co
   if (p.dense_tc) return do_shared_tc(p, ds, x, w_sgate, ws_gate, ws_up, ws_down, ws, st);
   float* sgu = at<float>(ws, p.off_sgu);
   moe_status s = launch_dense(ws_gate, p.Is, ws_up, p.Is, w_sgate, 1, x, false, sgu, p.T, p.H,
-                              p.S_sgu, st, "shared gate/up gemv");
+                              p.S_sgu, st, "shared gate/up gemv", false);
   if (s != MOE_OK) return s;
-  moe::k_shared_swiglu<<<dim3((p.Is + 255) / 256, p.T), 256, 0, st>>>(
-      sgu, p.S_sgu, p.T, p.Is, at<float>(ws, p.off_hs), at<float>(ws, p.off_gl));
+  launch_pdl(moe::k_shared_swiglu, dim3((p.Is + 255) / 256, p.T), dim3(256), 0, st, (const float*)sgu,
+             p.S_sgu, p.T, p.Is, at<float>(ws, p.off_hs), at<float>(ws, p.off_gl));
   s = launched("shared swiglu");
   if (s != MOE_OK) return s;
   return launch_dense(ws_down, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_hs), true,
@@ -542,7 +567,8 @@ moe_status do_latent_down(const Plan& p, const uint16_t* x, const uint16_t* w_ld
   moe_status s = launch_dense(w_ld, p.L, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_ld, st,
                               "latent down gemv");
   if (s != MOE_OK) return s;
-  moe::k_round_bf16<<<dim3((p.L + 255) / 256, p.T), 256, 0, st>>>(part, p.S_ld, p.T, p.L, x_lat);
+  launch_pdl(moe::k_round_bf16, dim3((p.L + 255) / 256, p.T), dim3(256), 0, st, (const float*)part, p.S_ld,
+             p.T, p.L, x_lat);
   return launched("latent round");
 }
 

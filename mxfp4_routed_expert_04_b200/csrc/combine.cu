@@ -11,6 +11,8 @@ namespace moe {
 
 // grid (ceil(width/4/256), T), block 256; width a multiple of 4
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y;
   const int c = (blockIdx.x * 256 + threadIdx.x) * 4;
   if (c >= a.width) return;
@@ -54,6 +56,8 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 __global__ void __launch_bounds__(256) k_shared_swiglu(const float* __restrict__ part, int S, int T,
                                                      int Is, float* __restrict__ hs,
                                                      float* __restrict__ gate_logit) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y;
   const int i = blockIdx.x * 256 + threadIdx.x;
   const int N = 2 * Is + 1;
@@ -76,6 +80,8 @@ __global__ void __launch_bounds__(256) k_shared_swiglu(const float* __restrict__
 // grid (ceil(N/256), T), block 256
 __global__ void __launch_bounds__(256) k_round_bf16(const float* __restrict__ part, int S, int T,
                                                   int N, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y;
   const int n = blockIdx.x * 256 + threadIdx.x;
   if (n >= N) return;

@@ -145,6 +145,13 @@ MOE_DEV uint32_t lds8(uint32_t addr) {
 // misc
 // ---------------------------------------------------------------------------
 MOE_DEV float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+
+// Programmatic dependent launch: wait until the previous kernel of the stream
+// has completed and its writes are visible (no-op for a kernel launched
+// without the attribute), then let the next kernel of the stream launch
+// while this one runs (it waits in its own pdl_wait before reading anything).
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 MOE_DEV float sigmoid_f32(float z) { return 1.0f / (1.0f + expf(-z)); }
 
 // Expert of the a-th non-empty segment of `offsets` (E+1 entries), or -1.

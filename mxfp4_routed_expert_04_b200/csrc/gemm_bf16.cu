@@ -58,6 +58,8 @@ struct Work {
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant__ Bf16GemmArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));

@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(1024) k_tile_list(const int32_t* __restrict__ 
                                                     int4* __restrict__ tiles,
                                                     int32_t* __restrict__ tile_base,
                                                     int32_t* __restrict__ n_tiles) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t warp_sum[32];
   const int n_act = __ldg(expert_list);
   const int a = threadIdx.x;
@@ -166,6 +168,8 @@ __global__ void __launch_bounds__(1024) k_tile_list(const int32_t* __restrict__ 
 // (row m in tile m/128 at position m%128). rows % 128 == 0, K % 128 == 0.
 __global__ void k_tile_scales(const uint8_t* __restrict__ src, long rows, int K,
                               uint8_t* __restrict__ dst) {
+  pdl_wait();
+  pdl_trigger();
   const int groups = K / 128;                    // 512-byte blocks per tile along K
   const long n = rows * (K / 128);
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
@@ -178,6 +182,8 @@ __global__ void k_tile_scales(const uint8_t* __restrict__ src, long rows, int K,
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant__ Mxf4GemmArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using S = Shape<kGateUp>;
   constexpr int kStages = S::kStages;
   extern __shared__ uint8_t smem_raw[];

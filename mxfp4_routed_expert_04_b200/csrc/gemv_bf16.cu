@@ -45,6 +45,8 @@ MOE_DEV void split8(const float (&v)[8], uint32_t (&hw)[4], uint32_t (&lw)[4]) {
 
 // grid (ceil(N / (16*kDenseWarps)), S, ceil(T/32)), block 32*kDenseWarps
 __global__ void __launch_bounds__(32 * kDenseWarps) k_dense_gemv(DenseArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int n0 = (blockIdx.x * kDenseWarps + warp) * 16;

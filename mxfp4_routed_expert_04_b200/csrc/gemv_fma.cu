@@ -81,6 +81,8 @@ MOE_DEV float warp_max(float v) {
 // ---------------------------------------------------------------------------
 template <int BPL, bool kGateUp, int RPS>
 __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArgs a, FmaGeometry g) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
   __shared__ int s_wsum[kFmaConsumers + 1];

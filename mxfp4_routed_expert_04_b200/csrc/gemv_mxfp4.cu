@@ -105,6 +105,8 @@ MOE_DEV void f16_block_scale(float m, float& scale, float& inv) {
 // (active expert, 16-row tile), item = ai * (I/16) + tile
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
@@ -257,6 +259,8 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
 // (active expert, 32-row tile of W), item = ai * (W/32) + tile
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;

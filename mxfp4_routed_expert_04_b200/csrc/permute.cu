@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
                                                         int32_t* __restrict__ row_slot,
                                                         int32_t* __restrict__ slot_row,
                                                         int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;                   // [E]  running cursor per expert
   int32_t* whist = sm + E;             // [32][E] per-warp counts -> exclusive bases
@@ -165,6 +167,8 @@ MOE_DEV float block_max_256(float v) {
 __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__ x, int W,
                                                   __half* __restrict__ x16,
                                                   float* __restrict__ xscale) {
+  pdl_wait();
+  pdl_trigger();
   const int tok = blockIdx.x;
   const uint16_t* row = x + (size_t)tok * W;
   float m = 0.0f;
@@ -209,6 +213,8 @@ __global__ void __launch_bounds__(256) k_act_to_mxfp4_perm(
     const int32_t* __restrict__ slot_row, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ expert_list, const int32_t* __restrict__ tile_base,
     uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t s_row[32], s_tile[32], s_n[32];
   if (__ldg(expert_list) == 0) return;
   const int tok = blockIdx.x;

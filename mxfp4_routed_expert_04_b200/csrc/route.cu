@@ -21,6 +21,8 @@ constexpr int kMaxPerLane = 32;   // E <= 1024
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, int S, int T, int E,
                                               int k, int32_t* __restrict__ idx,
                                               float* __restrict__ w, float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float lg[1024];
   const int tok = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += 256) {
