@@ -5,7 +5,7 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--w
 One step = one pass of the whole layer (route, permute, routed experts, gated
 shared expert, combine) over one batch of synthetic input, weights resident in
 HBM. Each timed step is a CUDA-graph replay of moe_layer, bracketed by CUDA
-events on the launching stream; L2 is flushed (512 MiB write) before every
+events on the launching stream; L2 is flushed before every
 step, outside the events. With N > 1 (torchrun) every rank runs an independent
 replica of the layer (the layer does not shard: no collective on the data
 path); timing is the max over ranks and ``value`` counts the tokens of all
@@ -219,7 +219,16 @@ def run_ours(args, w):
     layer = M.MoeLayer(dims, {k: v for k, v in dev.items() if k != "x"})
     x = dev["x"]
     stream = torch.cuda.Stream()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    # L2 flush outside the timed region: write 512 MiB, then read another
+    # 512 MiB so the written lines are evicted (written back) before the events
+    # start and no write-back of the flush itself lands inside a timed step
+    flush_w = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=flush_sink)
 
     def barrier():
         if world > 1:
@@ -247,7 +256,7 @@ def run_ours(args, w):
                for _ in range(steps)]
         with torch.cuda.stream(stream):
             for a, b in evs:
-                flush.zero_()
+                flush()
                 a.record(stream)
                 fn()
                 b.record(stream)
@@ -256,7 +265,7 @@ def run_ours(args, w):
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             graph.replay()
     torch.cuda.synchronize()
     barrier()
@@ -267,7 +276,7 @@ def run_ours(args, w):
         while time.perf_counter() < t_end:
             with torch.cuda.stream(stream):
                 for _ in range(50):
-                    flush.zero_()
+                    flush()
                     graph.replay()
             torch.cuda.synchronize()
 
@@ -356,7 +365,8 @@ def run_ours(args, w):
                   if act == "mxfp4" else "mxfp4 weights x f16 activations, fp32 accumulate"),
         "data": "synthetic (seeded; BASELINE distributions)",
         "config": {"workload": workload_label(w), "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every step (512 MiB write, outside the events)",
+                   "l2": "flushed before every step (512 MiB write, then 512 MiB read of another "
+                         "buffer, outside the events)",
                    "act_mode": act, "active_experts": n_active},
         "layer": {"algorithmic_bytes": lb, "hbm_gbs": lb / (step_ms * 1e-3) / 1e9,
                   "hbm_frac": lb / (step_ms * 1e-3) / 1e9 / peak,

@@ -300,9 +300,9 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   const FmaPlan f = fma_plan(K, kGateUp);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
   void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
-  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp, kGateUp ? 1 : 8>;
-  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp, kGateUp ? 1 : 4>;
-  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp, kGateUp ? 1 : 2>;
+  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp, kGateUp ? 1 : 4>;
+  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp, kGateUp ? 1 : 2>;
+  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp, 1>;
   if (f.bpl == 8) kern = moe::k_fma_gemv<8, kGateUp, 1>;
   if (!kern || !f.g.ok) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
   const int threads = 32 * (moe::kFmaConsumers + 1);

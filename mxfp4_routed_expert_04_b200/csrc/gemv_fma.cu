@@ -9,14 +9,15 @@
 // * the rows of all single-token experts form one list (gate/up: I row pairs
 //   per expert; down: W rows per expert); CTA c takes the c-th equal share;
 // * a producer warp fills each stage with a few large bulk TMA copies
-//   (cp.async.bulk): gate/up -> kFmaConsumers gate rows and the same up rows,
+//   (cp.async.bulk): gate/up -> kFmaConsumers/2 gate rows and the same up rows,
 //   down -> kFmaConsumers * RPS rows, each with the covering 16-byte-aligned
 //   span of E8M0 codes; a stage never crosses an expert, so every stage has
 //   one activation row;
-// * kFmaConsumers consumer warps share each stage: warp w takes row pair w
-//   (gate/up) or rows RPS*w .. RPS*w+RPS-1 (down); lane l owns the 32-element
-//   K blocks l, l+32, ... (BPL of them) of the activation row, kept in
-//   registers as f16;
+// * kFmaConsumers consumer warps share each stage: gate/up -> warps 2p and
+//   2p+1 take row pair p, each over one half of K, and add their partial
+//   sums in shared memory; down -> warp w takes rows RPS*w .. RPS*w+RPS-1;
+//   lane l owns the 32-element K blocks l, l+32, ... of its warp's K range of
+//   the activation row, kept in registers as f16;
 // * per 32 weights a lane spends 16 cvt.rn.f16x2.e2m1x2 (exact decode), 32
 //   fma.rn.f32.f16 (exact f16 x f16 products, fp32 sums) and one fp32 FMA for
 //   the block scale (E8M0 decoded without a branch, codes 0 and 255 included);
@@ -88,8 +89,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   __shared__ int s_wsum[kFmaConsumers + 1];
   __shared__ uint64_t s_bars[2 * kFmaMaxStages];
   __shared__ int s_abort;
+  __shared__ float2 s_part[2][kFmaConsumers / 2][2];   // gate/up partial sums [stage&1][pair][half]
   constexpr int kWarps = kFmaConsumers + 1;
-  constexpr int P = kGateUp ? kFmaConsumers : kFmaConsumers * RPS;   // units per stage
+  constexpr int P = kGateUp ? kFmaConsumers / 2 : kFmaConsumers * RPS;   // units per stage
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int K = kGateUp ? a.W : a.I;
   const int KB = K >> 5;
@@ -182,8 +184,15 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
     }
   } else {
     // ---------------- consumers ----------------
+    // gate/up: warps 2p and 2p+1 share row pair p of a stage, each over one
+    // half of K (half the activation registers), and combine their partial
+    // sums through shared memory; down: warp w takes rows RPS*w ... of a stage
     const int w = warp - 1;
-    uint32_t xr[BPL][16];
+    constexpr int BW = kGateUp ? (BPL + 1) / 2 : BPL;    // blocks per lane of this warp
+    const int half = kGateUp ? (w & 1) : 0;
+    const int KBw = kGateUp ? KB / 2 : KB;                // blocks of this warp's K range
+    const int kb0 = half * KBw;                           // its first block
+    uint32_t xr[BW][16];
     float xs = 1.0f;
     int cur_e = -1, r0 = 0;
     int k = 0;
@@ -200,12 +209,12 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
           const int tok = __ldg(a.row_token + r0);
           const __half* xrow = a.x16 + (size_t)tok * a.W;
 #pragma unroll
-          for (int j = 0; j < BPL; ++j) {
+          for (int j = 0; j < BW; ++j) {
             const int b = lane + 32 * j;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint4 t = make_uint4(0u, 0u, 0u, 0u);
-              if (b < KB) t = ldg16(xrow + b * 32 + 8 * q);
+              if (b < KBw) t = ldg16(xrow + (kb0 + b) * 32 + 8 * q);
               xr[j][4 * q] = t.x; xr[j][4 * q + 1] = t.y; xr[j][4 * q + 2] = t.z; xr[j][4 * q + 3] = t.w;
             }
           }
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
           const float* hrow = a.h32 + (size_t)r0 * a.I;
           float m = 0.0f;
 #pragma unroll
-          for (int j = 0; j < BPL; ++j) {
+          for (int j = 0; j < BW; ++j) {
             const int b = lane + 32 * j;
             if (b < KB)
               for (int q = 0; q < 8; ++q) {
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
             inv = ldexpf(1.0f, 15 - ex);
           }
 #pragma unroll
-          for (int j = 0; j < BPL; ++j) {
+          for (int j = 0; j < BW; ++j) {
             const int b = lane + 32 * j;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -251,10 +260,10 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       if (!tc::wait_or_abort(&full[slot], ph, abort)) break;
       const uint32_t st = smem_u32(smem + (size_t)slot * g.stage_bytes);
       const uint32_t soff = (uint32_t)((((size_t)e * N + r) * srow) & 15u);
-      // units of this warp: gate/up -> pair w (row 0 gate, row 1 up);
+      // rows of this warp: gate/up -> row 0 = gate, row 1 = up of pair w/2;
       // down -> rows RPS*w ... (codes qrow apart, scales srow apart)
       constexpr int NR = kGateUp ? 2 : RPS;
-      const int u0 = kGateUp ? w : RPS * w;
+      const int u0 = kGateUp ? (w >> 1) : RPS * w;
       float acc[NR];
 #pragma unroll
       for (int rr = 0; rr < NR; ++rr) acc[rr] = 0.0f;
@@ -263,16 +272,16 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 #pragma unroll
         for (int rr = 0; rr < NR; ++rr) {
           if (kGateUp) {
-            cb[rr] = st + rr * g.code_bytes + u0 * qrow + 16u * lane;
-            sbs[rr] = st + (rr ? g.sbuf2_off : g.sbuf_off) + soff + u0 * srow + lane;
+            cb[rr] = st + rr * g.code_bytes + u0 * qrow + 16u * (kb0 + lane);
+            sbs[rr] = st + (rr ? g.sbuf2_off : g.sbuf_off) + soff + u0 * srow + kb0 + lane;
           } else {
             cb[rr] = st + (u0 + rr) * qrow + 16u * lane;
             sbs[rr] = st + g.sbuf_off + soff + (u0 + rr) * srow + lane;
           }
         }
 #pragma unroll
-        for (int j = 0; j < BPL; ++j) {
-          if (lane + 32 * j < KB) {
+        for (int j = 0; j < BW; ++j) {
+          if (lane + 32 * j < KBw) {
 #pragma unroll
             for (int rr = 0; rr < NR; ++rr) {
               if (kGateUp || u0 + rr < n) {
@@ -285,7 +294,13 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
         }
         if (kGateUp) {
           const float gs = warp_sum(acc[0]), us = warp_sum(acc[1]);
-          if (lane == 0) a.h32[(size_t)r0 * a.I + r + u0] = silu_f32(gs * xs) * (us * xs);
+          float2* part = s_part[k & 1][u0];
+          if (lane == 0) part[half] = make_float2(gs, us);
+          asm volatile("bar.sync %0, 64;\n" ::"r"(1 + u0) : "memory");   // the two warps of the pair
+          if (half == 0 && lane == 0) {
+            const float2 o = part[1];
+            a.h32[(size_t)r0 * a.I + r + u0] = silu_f32((gs + o.x) * xs) * ((us + o.y) * xs);
+          }
         } else {
 #pragma unroll
           for (int rr = 0; rr < NR; ++rr) {
@@ -306,17 +321,17 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 }
 
 // Geometry for reduction length K (host side): rows per consumer warp in a
-// down stage rps = 8 / BPL; a stage holds kFmaConsumers units (gate/up: the
-// gate rows, then the up rows, then the two E8M0 spans; down: the codes of
-// kFmaConsumers * rps rows, then their span; every span with 32 bytes of
-// alignment slack); ring depth nst from the shared-memory budget.
+// down stage rps = max(1, 4 / BPL); a stage holds kFmaConsumers / 2 row pairs
+// (gate/up: the gate rows, then the up rows, then the two E8M0 spans) or
+// kFmaConsumers * rps rows (down: codes, then their span); every span with 32
+// bytes of alignment slack; ring depth nst from the shared-memory budget.
 FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   FmaGeometry g{};
   const size_t qrow = K / 2, srow = K / 32;
   const int bpl = (K + 1023) / 1024;
   if (bpl > 8) return g;
-  const int rps = gate_up ? 1 : 8 / (bpl > 4 ? 8 : bpl > 2 ? 4 : bpl > 1 ? 2 : 1);
-  const int units = gate_up ? kFmaConsumers : kFmaConsumers * rps;
+  const int rps = gate_up ? 1 : (bpl > 2 ? 1 : bpl > 1 ? 2 : 4);
+  const int units = gate_up ? kFmaConsumers / 2 : kFmaConsumers * rps;
   g.rps = rps;
   g.units = units;
   g.code_bytes = (uint32_t)((units * qrow + 127) / 128 * 128);
@@ -336,9 +351,9 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
 #define MOE_FMA_INST(BPL, RPS)                                                 \
   template __global__ void k_fma_gemv<BPL, true, 1>(FmaArgs, FmaGeometry);    \
   template __global__ void k_fma_gemv<BPL, false, RPS>(FmaArgs, FmaGeometry);
-MOE_FMA_INST(1, 8)
-MOE_FMA_INST(2, 4)
-MOE_FMA_INST(4, 2)
+MOE_FMA_INST(1, 4)
+MOE_FMA_INST(2, 2)
+MOE_FMA_INST(4, 1)
 MOE_FMA_INST(8, 1)
 #undef MOE_FMA_INST
 

@@ -41,7 +41,7 @@ __global__ void k_gateup_mxfp4(GateUpArgs a);
 __global__ void k_down_mxfp4(DownArgs a);
 size_t gemv_mxfp4_smem_bytes();
 // CUDA-core path: experts with exactly 1 token (gemv_fma.cu)
-constexpr int kFmaConsumers = 8;   // consumer warps per CTA (plus one producer warp)
+constexpr int kFmaConsumers = 16;  // consumer warps per CTA (plus one producer warp)
 constexpr int kFmaMaxStages = 8;
 struct FmaArgs {
   const __half* x16;         // gate/up: [T, W] f16 rows, xscale [T]
