@@ -47,25 +47,44 @@ int dense_splits(int N, int T, int K) {
   return S;
 }
 
-// Token count from which the router and the shared expert run on the tcgen05
-// bf16 GEMM (below it the split-K GEMV streams the weights once).
-constexpr int kDenseTcTokens = 128;
+// Token count from which the shared expert's gate/up GEMM applies SwiGLU in its
+// epilogue (below it the gate, up and sigmoid-gate rows write split-K
+// partial sums and a finaliser applies SwiGLU).
+constexpr int kDenseSwiGLUTokens = 128;
 
-// K splits of the tcgen05 router GEMM: enough items for two waves of SMs,
-// each split a whole number of 64-element stages, at most 8 splits.
-int tc_splits(int N, int T, int K) {
-  const long units = (long)((N + 255) / 256) * ((T + 127) / 128);
+// One token: the router and the shared expert stream whole weight rows on the
+// CUDA cores (k_rows_bf16) when both reduction lengths (H, I_shared) are
+// powers of two in 1024..8192; otherwise they take the tcgen05 GEMM with a
+// 16-token tile.
+bool rows_k_ok(int K) { return K == 1024 || K == 2048 || K == 4096 || K == 8192; }
+bool rows_path_for(int T, int H, int Is) { return T == 1 && rows_k_ok(H) && rows_k_ok(Is); }
+constexpr size_t kRowsSmemBudget = 200 * 1024;
+constexpr int kRowsFreeSMs = 8;     // SMs a side-stream row GEMV leaves to the routing chain
+
+// Token tile of the tcgen05 bf16 GEMM: the MMA's N, a multiple of 16 up to 128.
+int tc_tile_tokens(int T) { return T >= 128 ? 128 : (T + 15) / 16 * 16; }
+
+// K splits of a tcgen05 bf16 GEMM over `units` (weight units x token tiles):
+// double while the SMs are covered less than four times over, each split keeps
+// at least two 64-element stages and the partial sums (`split_bytes` per
+// split) stay within 40 MB.
+int tc_splits(long units, int K, size_t split_bytes) {
+  const int ks = K / 64;
   int S = 1;
-  while (S < 8 && units * S < 2L * kNumSMs && (K / 64) % (2 * S) == 0) S *= 2;
+  while (S < 64 && units * S < 4L * kNumSMs && ks % (2 * S) == 0 && ks / (2 * S) >= 2 &&
+         (size_t)(2 * S) * split_bytes <= (40u << 20))
+    S *= 2;
   return S;
 }
 
 struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   int S_router, S_sgu, S_sd, S_ld, S_lu;
-  bool dense_tc;             // router and shared expert on the tcgen05 bf16 GEMM
-  size_t off_hsb;            // tcgen05 shared expert: h as bf16 hi/lo [2][T, I_shared]
-  size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_hs, off_gl, off_sd, off_ld,
+  int Nt;                    // token tile of the tcgen05 bf16 GEMMs
+  bool swiglu_tc;            // shared gate/up GEMM applies SwiGLU in its epilogue
+  bool rows;                 // one token: router and shared expert on k_rows_bf16
+  size_t off_hsb;            // shared expert h as a bf16 hi/lo pair [2][T, I_shared]
+  size_t off_status, off_router, off_h16, off_hscale, off_h32, off_sgu, off_gl, off_sd, off_ld,
       off_ylat, off_lu, off_hsf, total;
   int max_tiles;
   size_t xop_bytes, xop_scale_off, xop_tiles_off, xop_tbase_off, xop_ntiles_off;
@@ -99,15 +118,21 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.W = d->L ? d->L : d->H;
   p.R = d->T * d->k;
   p.mode = d->act_mode;
-  p.dense_tc = p.T >= kDenseTcTokens;
-  if (p.dense_tc) {
-    p.S_router = tc_splits(p.E, p.T, p.H);
-    p.S_sgu = 1;               // only the sigmoid-gate row stays on the GEMV
+  p.Nt = tc_tile_tokens(p.T);
+  p.swiglu_tc = p.T >= kDenseSwiGLUTokens;
+  p.rows = rows_path_for(p.T, p.H, p.Is);
+  if (p.rows) {
+    p.S_router = 1;
+    p.S_sgu = 1;
     p.S_sd = 1;
   } else {
-    p.S_router = dense_splits(p.E, p.T, p.H);
-    p.S_sgu = dense_splits(2 * p.Is + 1, p.T, p.H);
-    p.S_sd = dense_splits(p.H, p.T, p.Is);
+    const long ntt = (p.T + p.Nt - 1) / p.Nt;
+    p.S_router = tc_splits((long)((p.E + 255) / 256) * ntt, p.H, (size_t)p.T * p.E * 4);
+    // SwiGLU epilogue: one split, the sigmoid-gate row on the GEMV
+    p.S_sgu = p.swiglu_tc ? 1
+                          : tc_splits((long)(2 * ((p.Is + 255) / 256) + 1) * ntt, p.H,
+                                      (size_t)p.T * (2 * p.Is + 1) * 4);
+    p.S_sd = tc_splits((long)((p.H + 255) / 256) * ntt, p.Is, (size_t)p.T * p.H * 4);
   }
   p.S_ld = p.L ? dense_splits(p.L, p.T, p.H) : 0;
   p.S_lu = p.L ? dense_splits(p.H, p.T, p.L) : 0;
@@ -118,9 +143,10 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_h16 = take((size_t)p.R * p.I * 2);
   p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
   p.off_h32 = take((size_t)p.R * p.I * 4);
-  p.off_sgu = take(p.dense_tc ? 0 : (size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
-  p.off_hs = take(p.dense_tc ? 0 : (size_t)p.T * p.Is * 4);
-  p.off_hsb = take(p.dense_tc ? (size_t)2 * p.T * p.Is * 2 : 0);
+  p.off_sgu = take(p.swiglu_tc || p.rows ? 0 : (size_t)p.S_sgu * p.T * (2 * p.Is + 1) * 4);
+  // shared expert h: a bf16 hi/lo pair [2][T, I_shared]; one token on the row
+  // GEMV: fp32 [I_shared] in the same bytes
+  p.off_hsb = take((size_t)2 * p.T * p.Is * 2);
   p.off_gl = take((size_t)p.T * 4);
   p.off_sd = take((size_t)p.S_sd * p.T * p.H * 4);
   p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
@@ -207,7 +233,7 @@ moe_status device_state(DeviceState** out) {
   DeviceState& s = g_dev[dev];
   if (!s.ready) {
     cudaError_t e = cudaFuncSetAttribute(moe::k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)moe::permute_smem_bytes(1024));
+                                         (int)moe::permute_smem_bytes(1024, 1 << 24));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::k_mxf4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)moe::mxf4_gemm_smem_bytes(true));
@@ -216,7 +242,16 @@ moe_status device_state(DeviceState** out) {
                                (int)moe::mxf4_gemm_smem_bytes(false));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::k_bf16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)moe::bf16_gemm_smem_bytes());
+                               moe::kBf16SmemBudget + 1024 + 256);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_rows_bf16<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kRowsSmemBudget);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_rows_bf16<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kRowsSmemBudget);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_rows_bf16<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kRowsSmemBudget);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.gemv_ctas_per_sm, moe::k_gateup_mxfp4, 32,
@@ -252,10 +287,29 @@ moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, 
   return launched(what);
 }
 
+// single-token row GEMV: one CTA per SM (at most max_ctas), ring depth from
+// the shared-memory budget
+moe_status launch_rows(const DeviceState& ds, moe::RowsArgs& r, bool swiglu, bool x_f32, int max_ctas,
+                       cudaStream_t st, const char* what, bool pdl = true) {
+  r.nst = moe::rows_stages(r.K, kRowsSmemBudget);
+  if (!r.nst) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: K=%d too long for the row GEMV", what, r.K);
+  const long units = swiglu ? r.rows[0] : (long)r.rows[0] + r.rows[1] + r.rows[2];
+  const long slots = moe::kRowsConsumers / moe::rows_warps_per_row(r.K);
+  const long per = swiglu ? slots / 2 : slots;
+  const int grid = (int)std::max<long>(1, std::min<long>((units + per - 1) / per, max_ctas));
+  const size_t smem = (size_t)r.nst * moe::rows_stage_bytes(r.K);
+  void (*kern)(moe::RowsArgs) = swiglu ? moe::k_rows_bf16<true, false>
+                                       : (x_f32 ? moe::k_rows_bf16<false, true> : moe::k_rows_bf16<false, false>);
+  const dim3 block(32 * (moe::kRowsConsumers + 1));
+  if (pdl) launch_pdl(kern, dim3(grid), block, smem, st, r);
+  else kern<<<grid, block, smem, st>>>(r);
+  return launched(what);
+}
+
 moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, int32_t* counts,
                       int32_t* offsets, int32_t* expert_list, int32_t* row_token, int32_t* row_slot,
                       int32_t* slot_row, void* x_op, void* ws, cudaStream_t st) {
-  launch_pdl(moe::k_permute, dim3(1), dim3(1024), moe::permute_smem_bytes(p.E), st, idx, p.T, p.k, p.E,
+  launch_pdl(moe::k_permute, dim3(1), dim3(1024), moe::permute_smem_bytes(p.E, p.R), st, idx, p.T, p.k, p.E,
              counts, offsets, expert_list, row_token, row_slot, slot_row, at<int32_t>(ws, p.off_status));
   moe_status s = launched("permute");
   if (s != MOE_OK) return s;
@@ -277,7 +331,7 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
 // CUDA-core GEMV launch shape for reduction length K (up to 8192): lanes own
 // BPL = ceil(K/1024) blocks; one CTA per SM with a ring of MOE_FMA_SMEM_KB KB.
 #ifndef MOE_FMA_SMEM_KB
-#define MOE_FMA_SMEM_KB 200
+#define MOE_FMA_SMEM_KB 210
 #endif
 struct FmaPlan {
   int bpl = 0;
@@ -300,9 +354,9 @@ moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t
   const FmaPlan f = fma_plan(K, kGateUp);
   const char* what = kGateUp ? "expert gate/up (cuda cores)" : "expert down (cuda cores)";
   void (*kern)(moe::FmaArgs, moe::FmaGeometry) = nullptr;
-  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp, kGateUp ? 1 : 4>;
-  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp, kGateUp ? 1 : 2>;
-  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp, 1>;
+  if (f.bpl == 1) kern = moe::k_fma_gemv<1, kGateUp, kGateUp ? 1 : 8>;
+  if (f.bpl == 2) kern = moe::k_fma_gemv<2, kGateUp, kGateUp ? 1 : 4>;
+  if (f.bpl == 4) kern = moe::k_fma_gemv<4, kGateUp, kGateUp ? 1 : 2>;
   if (f.bpl == 8) kern = moe::k_fma_gemv<8, kGateUp, 1>;
   if (!kern || !f.g.ok) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no kernel for K=%d", what, K);
   const int threads = 32 * (moe::kFmaConsumers + 1);
@@ -356,70 +410,137 @@ moe_status code_map(CUtensorMap* m, const uint8_t* base, uint64_t rows, uint64_t
 
 // bf16 matrices: [rows, cols] elements
 moe_status bf16_map(CUtensorMap* m, const uint16_t* base, uint64_t rows, uint64_t cols,
-                    const char* what) {
-  return tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 128, what);
+                    const char* what, uint32_t box_rows = 128) {
+  return tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box_rows, what);
 }
 
+// grid: one CTA per SM at most (the stage ring takes most of shared memory)
 moe_status launch_bf16_gemm(const DeviceState& ds, moe::Bf16GemmArgs& g, cudaStream_t st,
-                            const char* what) {
-  const long units = (long)(g.mode == moe::kBf16SwiGLU ? g.M / 128 : (g.M + 255) / 256) *
-                     ((g.T + 127) / 128) * g.S;
-  const int grid = (int)std::min<long>(units, ds.num_sms);
-  moe::k_bf16_gemm<<<grid, moe::bf16_gemm_threads(), moe::bf16_gemm_smem_bytes(), st>>>(g);
+                            const char* what, bool pdl = true) {
+  long units = 0;
+  for (int i = 0; i < 3; ++i)
+    units += g.mode == moe::kBf16SwiGLU ? (i == 0 ? g.seg_rows[0] / 128 : 0) : (g.seg_rows[i] + 255) / 256;
+  const long items = units * ((g.T + g.N - 1) / g.N) * g.S;
+  const int grid = (int)std::min<long>(items, ds.num_sms);
+  const size_t smem = moe::bf16_gemm_smem_bytes(g.N, g.passes);
+  if (pdl) launch_pdl(moe::k_bf16_gemm, dim3(grid), dim3(moe::bf16_gemm_threads()), smem, st, g);
+  else moe::k_bf16_gemm<<<grid, moe::bf16_gemm_threads(), smem, st>>>(g);
   return launched(what);
 }
 
+// The router logits (and, when w_sgate is given, the shared expert's sigmoid
+// gate logit from the same pass over x), then top-k.
 moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
-                    int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st) {
+                    int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st,
+                    const uint16_t* w_sgate = nullptr) {
   float* part = at<float>(ws, p.off_router);
   moe_status s;
-  if (p.dense_tc) {
-    moe::Bf16GemmArgs g;
-    memset(&g, 0, sizeof(g));
-    if ((s = bf16_map(&g.map_a0, wr, p.E, p.H, "router weights")) != MOE_OK ||
-        (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens")) != MOE_OK)
-      return s;
-    g.out = part; g.status = at<int32_t>(ws, p.off_status);
-    g.mode = moe::kBf16Plain; g.M = p.E; g.K = p.H; g.T = p.T; g.S = p.S_router; g.passes = 1;
-    s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)");
-  } else {
-    s = launch_dense(wr, p.E, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_router, st,
-                     "router gemv");
+  if (p.rows) {
+    moe::RowsArgs r;
+    memset(&r, 0, sizeof(r));
+    r.w[0] = wr; r.rows[0] = p.E; r.out[0] = part;
+    if (w_sgate) { r.w[1] = w_sgate; r.rows[1] = 1; r.out[1] = at<float>(ws, p.off_gl); }
+    r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
+    if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
+    launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
+               p.k, idx, w, logits);
+    return launched("top-k");
   }
-  if (s != MOE_OK) return s;
-  launch_pdl(moe::k_topk, dim3(p.T), dim3(256), 0, st, (const float*)part, p.S_router, p.T, p.E, p.k, idx, w,
+  if (w_sgate) return fail(MOE_ERR_INVALID_ARG, "internal: sigmoid gate only with the row GEMV");
+  moe::Bf16GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  if ((s = bf16_map(&g.map_a[0], wr, p.E, p.H, "router weights")) != MOE_OK ||
+      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK)
+    return s;
+  g.out = part; g.status = at<int32_t>(ws, p.off_status);
+  g.mode = moe::kBf16Plain; g.K = p.H; g.T = p.T; g.S = p.S_router; g.passes = 1; g.N = p.Nt;
+  g.seg_rows[0] = p.E; g.ld = p.E;
+  if ((s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)")) != MOE_OK) return s;
+  launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E, p.k, idx, w,
              logits);
   return launched("top-k");
 }
 
-// many tokens: SwiGLU GEMM (h as a bf16 hi/lo pair), the sigmoid-gate row on
-// the GEMV, the down GEMM over both halves of h
-moe_status do_shared_tc(const Plan& p, const DeviceState& ds, const uint16_t* x,
-                        const uint16_t* w_sgate, const uint16_t* ws_gate, const uint16_t* ws_up,
-                        const uint16_t* ws_down, void* ws, cudaStream_t st) {
+// Shared expert on the tcgen05 GEMM, first half: h = silu(Wg x) * (Wu x) as
+// a bf16 hi/lo pair and the sigmoid-gate logit. Many tokens: SwiGLU in the
+// gate/up epilogue, the sigmoid-gate row on the GEMV. Few tokens: the gate,
+// up and sigmoid-gate rows as three segments of one split-K GEMM, SwiGLU in
+// the finaliser.
+moe_status do_shared_up(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* w_sgate,
+                        const uint16_t* ws_gate, const uint16_t* ws_up, void* ws, cudaStream_t st,
+                        bool sgate_done = false, int max_ctas = 0) {
+  if (p.rows) {
+    moe::RowsArgs r;
+    memset(&r, 0, sizeof(r));
+    r.w[0] = ws_gate; r.w[1] = ws_up; r.rows[0] = p.Is; r.out[0] = at<float>(ws, p.off_hsb);
+    r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
+    moe_status s = launch_rows(ds, r, true, false, max_ctas ? max_ctas : ds.num_sms, st,
+                               "shared gate/up gemv", false);
+    if (s != MOE_OK || sgate_done) return s;
+    moe::RowsArgs g;
+    memset(&g, 0, sizeof(g));
+    g.w[0] = w_sgate; g.rows[0] = 1; g.out[0] = at<float>(ws, p.off_gl);
+    g.x = x; g.K = p.H; g.status = r.status;
+    return launch_rows(ds, g, false, false, 1, st, "shared gate gemv");
+  }
   uint16_t* h_hi = at<uint16_t>(ws, p.off_hsb);
   uint16_t* h_lo = h_hi + (size_t)p.T * p.Is;
+  int32_t* status = at<int32_t>(ws, p.off_status);
   moe_status s;
   moe::Bf16GemmArgs g;
   memset(&g, 0, sizeof(g));
-  if ((s = bf16_map(&g.map_a0, ws_gate, p.Is, p.H, "shared gate weights")) != MOE_OK ||
-      (s = bf16_map(&g.map_a1, ws_up, p.Is, p.H, "shared up weights")) != MOE_OK ||
-      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens")) != MOE_OK)
+  if ((s = bf16_map(&g.map_a[0], ws_gate, p.Is, p.H, "shared gate weights")) != MOE_OK ||
+      (s = bf16_map(&g.map_a[1], ws_up, p.Is, p.H, "shared up weights")) != MOE_OK ||
+      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK)
     return s;
-  g.h_hi = h_hi; g.h_lo = h_lo; g.status = at<int32_t>(ws, p.off_status);
-  g.mode = moe::kBf16SwiGLU; g.M = p.Is; g.K = p.H; g.T = p.T; g.S = 1; g.passes = 1;
-  if ((s = launch_bf16_gemm(ds, g, st, "shared gate/up gemm (tcgen05)")) != MOE_OK) return s;
-  if ((s = launch_dense(w_sgate, 1, nullptr, 0, nullptr, 0, x, false, at<float>(ws, p.off_gl), p.T,
-                        p.H, 1, st, "shared gate gemv")) != MOE_OK)
-    return s;
+  g.status = status;
+  g.K = p.H; g.T = p.T; g.passes = 1; g.N = p.Nt;
+  if (p.swiglu_tc) {
+    g.mode = moe::kBf16SwiGLU; g.S = 1;
+    g.seg_rows[0] = p.Is;
+    g.h_hi = h_hi; g.h_lo = h_lo;
+    if ((s = launch_bf16_gemm(ds, g, st, "shared gate/up gemm (tcgen05)", false)) != MOE_OK) return s;
+    if ((s = launch_dense(w_sgate, 1, nullptr, 0, nullptr, 0, x, false, at<float>(ws, p.off_gl), p.T,
+                          p.H, 1, st, "shared gate gemv")) != MOE_OK)
+      return s;
+  } else {
+    if ((s = bf16_map(&g.map_a[2], w_sgate, 1, p.H, "shared sigmoid-gate weights")) != MOE_OK) return s;
+    float* sgu = at<float>(ws, p.off_sgu);
+    g.mode = moe::kBf16Plain; g.S = p.S_sgu;
+    g.seg_rows[0] = p.Is; g.seg_rows[1] = p.Is; g.seg_rows[2] = 1; g.ld = 2 * p.Is + 1;
+    g.out = sgu;
+    if ((s = launch_bf16_gemm(ds, g, st, "shared gate/up gemm (tcgen05)", false)) != MOE_OK) return s;
+    launch_pdl(moe::k_shared_swiglu, dim3((p.Is + moe::kFinThreads - 1) / moe::kFinThreads, p.T),
+               dim3(moe::kFinThreads), 0, st, (const float*)sgu,
+               p.S_sgu, p.T, p.Is, h_hi, h_lo, at<float>(ws, p.off_gl));
+    if ((s = launched("shared swiglu")) != MOE_OK) return s;
+  }
+  return MOE_OK;
+}
+
+// Shared expert, second half: the down GEMM over both halves of h (split-K
+// partial sums for the combine).
+moe_status do_shared_down(const Plan& p, const DeviceState& ds, const uint16_t* ws_down, void* ws,
+                          cudaStream_t st, int max_ctas = 0) {
+  if (p.rows) {
+    moe::RowsArgs r;
+    memset(&r, 0, sizeof(r));
+    r.w[0] = ws_down; r.rows[0] = p.H; r.out[0] = at<float>(ws, p.off_sd);
+    r.x = at<float>(ws, p.off_hsb); r.K = p.Is; r.status = at<int32_t>(ws, p.off_status);
+    return launch_rows(ds, r, false, true, max_ctas ? max_ctas : ds.num_sms, st, "shared down gemv");
+  }
+  uint16_t* h_hi = at<uint16_t>(ws, p.off_hsb);
+  uint16_t* h_lo = h_hi + (size_t)p.T * p.Is;
+  moe_status s;
   moe::Bf16GemmArgs d;
   memset(&d, 0, sizeof(d));
-  if ((s = bf16_map(&d.map_a0, ws_down, p.H, p.Is, "shared down weights")) != MOE_OK ||
-      (s = bf16_map(&d.map_b0, h_hi, p.T, p.Is, "shared h (hi)")) != MOE_OK ||
-      (s = bf16_map(&d.map_b1, h_lo, p.T, p.Is, "shared h (lo)")) != MOE_OK)
+  if ((s = bf16_map(&d.map_a[0], ws_down, p.H, p.Is, "shared down weights")) != MOE_OK ||
+      (s = bf16_map(&d.map_b0, h_hi, p.T, p.Is, "shared h (hi)", p.Nt)) != MOE_OK ||
+      (s = bf16_map(&d.map_b1, h_lo, p.T, p.Is, "shared h (lo)", p.Nt)) != MOE_OK)
     return s;
-  d.out = at<float>(ws, p.off_sd); d.status = g.status;
-  d.mode = moe::kBf16Plain; d.M = p.H; d.K = p.Is; d.T = p.T; d.S = 1; d.passes = 2;
+  d.out = at<float>(ws, p.off_sd); d.status = at<int32_t>(ws, p.off_status);
+  d.mode = moe::kBf16Plain; d.K = p.Is; d.T = p.T; d.S = p.S_sd; d.passes = 2; d.N = p.Nt;
+  d.seg_rows[0] = p.H; d.ld = p.H;
   return launch_bf16_gemm(ds, d, st, "shared down gemm (tcgen05)");
 }
 
@@ -518,22 +639,6 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   return launched("expert down");
 }
 
-moe_status do_shared(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* w_sgate,
-                     const uint16_t* ws_gate, const uint16_t* ws_up, const uint16_t* ws_down,
-                     void* ws, cudaStream_t st) {
-  if (p.dense_tc) return do_shared_tc(p, ds, x, w_sgate, ws_gate, ws_up, ws_down, ws, st);
-  float* sgu = at<float>(ws, p.off_sgu);
-  moe_status s = launch_dense(ws_gate, p.Is, ws_up, p.Is, w_sgate, 1, x, false, sgu, p.T, p.H,
-                              p.S_sgu, st, "shared gate/up gemv", false);
-  if (s != MOE_OK) return s;
-  launch_pdl(moe::k_shared_swiglu, dim3((p.Is + 255) / 256, p.T), dim3(256), 0, st, (const float*)sgu,
-             p.S_sgu, p.T, p.Is, at<float>(ws, p.off_hs), at<float>(ws, p.off_gl));
-  s = launched("shared swiglu");
-  if (s != MOE_OK) return s;
-  return launch_dense(ws_down, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_hs), true,
-                      at<float>(ws, p.off_sd), p.T, p.Is, p.S_sd, st, "shared down gemv");
-}
-
 moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row, const float* topk_w,
                     const uint16_t* w_lat_up, float* y, void* ws, cudaStream_t st) {
   moe::CombineArgs c;
@@ -544,7 +649,8 @@ moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row,
     // routed weighted sum at width L, then the up-projection, then + shared
     c.y_perm = y_perm; c.add1 = nullptr; c.S1 = 0; c.add2 = nullptr; c.S2 = 0;
     c.out = at<float>(ws, p.off_ylat); c.width = p.L;
-    moe::k_combine<<<dim3((p.L / 4 + 255) / 256, p.T), 256, 0, st>>>(c);
+    moe::k_combine<<<dim3((p.L / 4 + moe::kCombineThreads - 1) / moe::kCombineThreads, p.T),
+                     moe::kCombineThreads, 0, st>>>(c);
     moe_status s = launched("latent combine");
     if (s != MOE_OK) return s;
     s = launch_dense(w_lat_up, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_ylat), true,
@@ -557,7 +663,8 @@ moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row,
   }
   c.add2 = at<float>(ws, p.off_sd); c.S2 = p.S_sd;
   c.out = y; c.width = p.H;
-  moe::k_combine<<<dim3((p.H / 4 + 255) / 256, p.T), 256, 0, st>>>(c);
+  moe::k_combine<<<dim3((p.H / 4 + moe::kCombineThreads - 1) / moe::kCombineThreads, p.T),
+                   moe::kCombineThreads, 0, st>>>(c);
   return launched("combine");
 }
 
@@ -567,7 +674,8 @@ moe_status do_latent_down(const Plan& p, const uint16_t* x, const uint16_t* w_ld
   moe_status s = launch_dense(w_ld, p.L, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_ld, st,
                               "latent down gemv");
   if (s != MOE_OK) return s;
-  launch_pdl(moe::k_round_bf16, dim3((p.L + 255) / 256, p.T), dim3(256), 0, st, (const float*)part, p.S_ld,
+  launch_pdl(moe::k_round_bf16, dim3((p.L + moe::kFinThreads - 1) / moe::kFinThreads, p.T),
+             dim3(moe::kFinThreads), 0, st, (const float*)part, p.S_ld,
              p.T, p.L, x_lat);
   return launched("latent round");
 }
@@ -726,7 +834,8 @@ moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t*
   const cudaStream_t st = (cudaStream_t)stream;
   DeviceState* ds;
   if ((s = device_state(&ds)) != MOE_OK) return s;
-  if ((s = do_shared(p, *ds, x, w_sgate, ws_gate, ws_up, ws_down, ws, st)) != MOE_OK) return s;
+  if ((s = do_shared_up(p, *ds, x, w_sgate, ws_gate, ws_up, ws, st)) != MOE_OK) return s;
+  if ((s = do_shared_down(p, *ds, ws_down, ws, st)) != MOE_OK) return s;
   return do_final(p, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
 }
 
@@ -762,31 +871,42 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   std::lock_guard<std::mutex> lk(g_mu);
   const cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaEventRecord(ds->ev_fork, st);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(ds->side, ds->ev_fork, 0);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
-  // side stream: latent projection, then the shared expert
+  // main stream first: the router's CTAs are queued before the shared expert's
+  // (one token: the sigmoid-gate row rides along with the router rows)
+  if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st,
+                    p.rows ? a->w_sgate : nullptr)) != MOE_OK)
+    return s;
+  // side stream: latent projection, then the first half of the shared expert
+  // (it streams its weights while the routing chain runs)
+  if ((e = cudaStreamWaitEvent(ds->side, ds->ev_fork, 0)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
   if (p.L) {
     if ((s = do_latent_down(p, a->x, a->w_lat_down, a->x_lat, ws, ds->side)) != MOE_OK) return s;
     if ((e = cudaEventRecord(ds->ev_lat, ds->side)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   }
-  if ((s = do_shared(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, a->ws_down, ws, ds->side)) != MOE_OK)
+  // (the row GEMV leaves a few SMs to the routing chain's small kernels)
+  if ((s = do_shared_up(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, ws, ds->side, p.rows,
+                        ds->num_sms - kRowsFreeSMs)) != MOE_OK)
     return s;
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
-  // main stream: routing, experts, combine
-  if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st)) != MOE_OK) return s;
+  // main stream: dispatch, experts, combine
   if (p.L && (e = cudaStreamWaitEvent(st, ds->ev_lat, 0)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
   if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets,
                       a->expert_list, a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) !=
       MOE_OK)
     return s;
+  // the routed experts start once the shared expert's first half is done, so
+  // that they have every SM from their first stage on
+  if ((e = cudaStreamWaitEvent(st, ds->ev_shared, 0)) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
   if ((s = do_expert_ffn(p, *ds, a->x_op, a->offsets, a->expert_list, a->row_token, a->wg_q,
                          a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
     return s;
-  if ((e = cudaStreamWaitEvent(st, ds->ev_shared, 0)) != cudaSuccess)
-    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
+  if ((s = do_shared_down(p, *ds, a->ws_down, ws, st)) != MOE_OK) return s;
   return do_final(p, a->y_perm, a->slot_row, a->topk_w, a->w_lat_up, a->y, ws, st);
 }
 

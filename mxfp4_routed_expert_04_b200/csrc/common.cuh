@@ -144,6 +144,29 @@ MOE_DEV uint32_t lds8(uint32_t addr) {
 // ---------------------------------------------------------------------------
 // misc
 // ---------------------------------------------------------------------------
+// Sum of S split-K partials p[0], p[stride], ... in the order s = 0, 1, ...;
+// the loads are issued sixteen at a time ahead of their additions.
+MOE_DEV float sum_splits(const float* __restrict__ p, int S, size_t stride) {
+  float acc = 0.0f;
+  int s = 0;
+  for (; s + 16 <= S; s += 16) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(p + (size_t)(s + i) * stride);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc += v[i];
+  }
+  for (; s + 4 <= S; s += 4) {
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __ldg(p + (size_t)(s + i) * stride);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc += v[i];
+  }
+  for (; s < S; ++s) acc += __ldg(p + (size_t)s * stride);
+  return acc;
+}
+
 MOE_DEV float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
 // Programmatic dependent launch: wait until the previous kernel of the stream

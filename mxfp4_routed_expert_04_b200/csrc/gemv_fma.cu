@@ -135,11 +135,11 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   }
   __syncthreads();
   volatile int* abort = &s_abort;
-  // a stage takes at most P units, never crossing an expert or the range end
-  auto stage_units = [&](long u) -> int {
-    const long end_e = (u / N + 1) * N;
-    return (int)min((long)P, min(end_e, hi) - u);
-  };
+  // a stage takes at most P units, never crossing an expert or the range end;
+  // both roles walk the stages with the same incremental cursor (expert slot
+  // si, row r within it, ring slot and phase): no division per stage
+  const int si0 = (int)(lo / N), r_lo = (int)(lo - (long)si0 * N);
+  auto stage_units = [&](long u, int r) -> int { return (int)min((long)min(P, N - r), hi - u); };
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -148,13 +148,11 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       bool filled[kFmaMaxStages];
 #pragma unroll
       for (int s = 0; s < kFmaMaxStages; ++s) { last_ph[s] = 0; filled[s] = false; }
-      int k = 0;
-      for (long u = lo; u < hi; ++k) {
-        const int n = stage_units(u);
-        const int slot = k % g.nst;
-        const uint32_t ph = (uint32_t)((k / g.nst) & 1);
+      int si = si0, r = r_lo, slot = 0;
+      uint32_t ph = 0;
+      for (long u = lo; u < hi;) {
+        const int n = stage_units(u, r);
         if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) break;
-        const int si = (int)(u / N), r = (int)(u - (long)si * N);
         const size_t row = (size_t)s_list[si] * N + r;
         const uint32_t cb = n * qrow;
         const size_t s0 = row * srow, s1 = (row + n) * srow;
@@ -176,6 +174,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
         last_ph[slot] = ph;
         filled[slot] = true;
         u += n;
+        r += n;
+        if (r == N) { r = 0; ++si; }
+        if (++slot == g.nst) { slot = 0; ph ^= 1u; }
       }
       if (*abort) {     // let every issued copy land before the CTA can exit
         for (int s = 0; s < g.nst; ++s)
@@ -195,12 +196,10 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
     uint32_t xr[BW][16];
     float xs = 1.0f;
     int cur_e = -1, r0 = 0;
-    int k = 0;
+    int si = si0, r = r_lo, slot = 0, k = 0;
+    uint32_t ph = 0;
     for (long u = lo; u < hi; ++k) {
-      const int n = stage_units(u);
-      const int slot = k % g.nst;
-      const uint32_t ph = (uint32_t)((k / g.nst) & 1);
-      const int si = (int)(u / N), r = (int)(u - (long)si * N);
+      const int n = stage_units(u, r);
       const int e = s_list[si];
       if (e != cur_e) {                     // new expert: load its activation row
         cur_e = e;
@@ -314,6 +313,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[slot]);   // this warp is done with the slot
       u += n;
+      r += n;
+      if (r == N) { r = 0; ++si; }
+      if (++slot == g.nst) { slot = 0; ph ^= 1u; }
     }
   }
   __syncthreads();
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 }
 
 // Geometry for reduction length K (host side): rows per consumer warp in a
-// down stage rps = max(1, 4 / BPL); a stage holds kFmaConsumers / 2 row pairs
+// down stage rps = max(1, 8 / BPL); a stage holds kFmaConsumers / 2 row pairs
 // (gate/up: the gate rows, then the up rows, then the two E8M0 spans) or
 // kFmaConsumers * rps rows (down: codes, then their span); every span with 32
 // bytes of alignment slack; ring depth nst from the shared-memory budget.
@@ -330,7 +332,7 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   const size_t qrow = K / 2, srow = K / 32;
   const int bpl = (K + 1023) / 1024;
   if (bpl > 8) return g;
-  const int rps = gate_up ? 1 : (bpl > 2 ? 1 : bpl > 1 ? 2 : 4);
+  const int rps = gate_up ? 1 : (bpl > 4 ? 1 : bpl > 2 ? 2 : bpl > 1 ? 4 : 8);
   const int units = gate_up ? kFmaConsumers / 2 : kFmaConsumers * rps;
   g.rps = rps;
   g.units = units;
@@ -351,9 +353,9 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
 #define MOE_FMA_INST(BPL, RPS)                                                 \
   template __global__ void k_fma_gemv<BPL, true, 1>(FmaArgs, FmaGeometry);    \
   template __global__ void k_fma_gemv<BPL, false, RPS>(FmaArgs, FmaGeometry);
-MOE_FMA_INST(1, 4)
-MOE_FMA_INST(2, 2)
-MOE_FMA_INST(4, 1)
+MOE_FMA_INST(1, 8)
+MOE_FMA_INST(2, 4)
+MOE_FMA_INST(4, 2)
 MOE_FMA_INST(8, 1)
 #undef MOE_FMA_INST
 

@@ -96,24 +96,60 @@ template <bool kGateUp> __global__ void k_mxf4_gemm(const __grid_constant__ Mxf4
 size_t mxf4_gemm_smem_bytes(bool gate_up);
 int mxf4_gemm_threads();
 
-// --- dense bf16 GEMM on tcgen05 (many tokens) ------------------------------
-// Weights [rows, K] and tokens [T, K] bf16 through 2-D tensor maps (boxes of
-// 128 rows x 64 elements, 128-byte swizzle). K / S a multiple of 64.
-constexpr int kBf16Plain = 0;     // out[s, t, m] fp32 partial sums over K split s
+// --- single-token bf16 GEMV on the CUDA cores (whole rows per CTA) ---------
+constexpr int kRowsConsumers = 16;   // consumer warps (plus one producer warp)
+constexpr int kRowsMaxStages = 8;
+constexpr int kRowsMaxChunks = 8;    // 8-element chunks per lane (2048 elements per warp)
+struct RowsArgs {
+  const uint16_t* w[3];      // bf16 [rows[i], K]; SwiGLU: w[0] gate, w[1] up
+  int rows[3];               // plain: segment rows (0: unused); SwiGLU: rows[0] = row pairs
+  float* out[3];             // plain: out[i][row] per segment; SwiGLU: out[0][i] = h_i
+  const void* x;             // [K] bf16, or fp32 (k_rows_bf16<*, true>)
+  int32_t* status;
+  int K, nst;
+};
+template <bool kSwiGLU, bool kXF32> __global__ void k_rows_bf16(RowsArgs a);
+// K a power of two in 1024..8192: warps per row K/2048 (at least 1), a stage
+// of 16 / that many rows
+__host__ __device__ constexpr int rows_warps_per_row(int K) { return K > 2048 ? K / 2048 : 1; }
+__host__ __device__ constexpr size_t rows_stage_bytes(int K) {
+  return (size_t)(kRowsConsumers / rows_warps_per_row(K)) * K * 2;
+}
+int rows_stages(int K, size_t smem_budget);
+
+// --- dense bf16 GEMM on tcgen05 -----------------------------------------------
+// Weights [rows, K] and tokens [T, K] bf16 through 2-D tensor maps (weights:
+// boxes of 128 rows x 64 elements; tokens: N rows x 64 elements; 128-byte
+// swizzle). K / S a multiple of 64; N (tokens per tile, the MMA's N) a
+// multiple of 16 in 16..128.
+constexpr int kBf16Plain = 0;     // out[(s*T + t)*ld + col] fp32 partial sums over K split s
 constexpr int kBf16SwiGLU = 1;    // h = silu(Wg x) * (Wu x) as a bf16 hi/lo pair [T, M]
 struct Bf16GemmArgs {
-  CUtensorMap map_a0;        // plain: W; SwiGLU: Wg
-  CUtensorMap map_a1;        // SwiGLU: Wu
+  CUtensorMap map_a[3];      // plain: up to three row segments of W; SwiGLU: [0] Wg, [1] Wu
   CUtensorMap map_b0;        // tokens (pass 0)
   CUtensorMap map_b1;        // tokens of pass 1 (plain, passes == 2: the lo half)
-  float* out;                // plain: [S, T, M]
+  float* out;                // plain
   uint16_t* h_hi;            // SwiGLU: [T, M]
   uint16_t* h_lo;
   int32_t* status;
-  int mode, M, K, T, S, passes;
+  int mode, K, T, S, passes, N;
+  int seg_rows[3];           // plain: rows of each segment (0: unused); SwiGLU: seg_rows[0] = M
+  int ld;                    // plain: row stride of out; segment i starts at column rows(0..i-1)
 };
 __global__ void k_bf16_gemm(const __grid_constant__ Bf16GemmArgs a);
-size_t bf16_gemm_smem_bytes();
+// Stage = two 128-row weight tiles + one N-row token tile per pass; as many
+// stages (at most 8) as fit in the budget: all of a CTA's shared memory for
+// large token tiles, 144 KB for N <= 64 so that the small kernels of the
+// routing chain still fit on an SM beside a CTA of a weight-streaming GEMM.
+constexpr int kBf16SmemBudget = 232448 - 1024 - 256;
+constexpr int kBf16SmallBudget = 144 * 1024;
+__host__ __device__ constexpr int bf16_stage_bytes(int N, int passes) { return 32768 + passes * N * 128; }
+__host__ __device__ constexpr int bf16_stages(int N, int passes) {
+  return ((N <= 64 ? kBf16SmallBudget : kBf16SmemBudget) / bf16_stage_bytes(N, passes)) < 8
+             ? (N <= 64 ? kBf16SmallBudget : kBf16SmemBudget) / bf16_stage_bytes(N, passes)
+             : 8;
+}
+size_t bf16_gemm_smem_bytes(int N, int passes);
 int bf16_gemm_threads();
 
 // --- dense bf16 GEMV with split-K partial sums -----------------------------
@@ -130,6 +166,7 @@ __global__ void k_dense_gemv(DenseArgs a);
 constexpr int kDenseWarps = 4;   // warps (16-row tiles) per CTA
 
 // --- router tail ------------------------------------------------------------
+constexpr int kTopkThreads = 1024;
 __global__ void k_topk(const float* part, int S, int T, int E, int k, int32_t* idx, float* w,
                        float* logits);
 
@@ -137,7 +174,7 @@ __global__ void k_topk(const float* part, int S, int T, int E, int k, int32_t* i
 __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
                           int32_t* offsets, int32_t* expert_list, int32_t* row_token,
                           int32_t* row_slot, int32_t* slot_row, int32_t* status);
-size_t permute_smem_bytes(int E);
+size_t permute_smem_bytes(int E, int R);
 __global__ void k_act_to_f16(const uint16_t* x, int W, __half* x16, float* xscale);
 __global__ void k_act_to_mxfp4_perm(const uint16_t* x, int W, int k, const int32_t* idx,
                                     const int32_t* slot_row, const int32_t* offsets,
@@ -145,8 +182,9 @@ __global__ void k_act_to_mxfp4_perm(const uint16_t* x, int W, int k, const int32
                                     uint8_t* q, uint8_t* sf);
 
 // --- finalisers of split-K partials ----------------------------------------
-__global__ void k_shared_swiglu(const float* part, int S, int T, int Is, float* hs,
-                                float* gate_logit);
+constexpr int kFinThreads = 64;
+__global__ void k_shared_swiglu(const float* part, int S, int T, int Is, uint16_t* h_hi,
+                                uint16_t* h_lo, float* gate_logit);
 __global__ void k_round_bf16(const float* part, int S, int T, int N, uint16_t* out);
 
 struct CombineArgs {
@@ -162,6 +200,7 @@ struct CombineArgs {
   float* out;                // [T, width]
   int T, width;
 };
+constexpr int kCombineThreads = 64;
 __global__ void k_combine(CombineArgs a);
 
 // one-line reason for moe_last_error() (defined with the C ABI in api.cu)

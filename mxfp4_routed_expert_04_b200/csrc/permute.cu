@@ -25,11 +25,13 @@ namespace moe {
 constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
 
-size_t permute_smem_bytes(int E) {
-  return (size_t)(kPermWarps + 2) * E * sizeof(int32_t) + 16;
+// cursors [E], a flag word, and (more than one warp of pairs) the per-warp
+// counts [32][E]
+size_t permute_smem_bytes(int E, int R) {
+  return ((size_t)E + 4 + (R > 32 ? (size_t)kPermWarps * E : 0)) * sizeof(int32_t);
 }
 
-// grid 1, block 1024, dynamic smem permute_smem_bytes(E)
+// grid 1, block 1024, dynamic smem permute_smem_bytes(E, T * k)
 __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restrict__ idx, int T, int k,
                                                         int E, int32_t* __restrict__ counts,
                                                         int32_t* __restrict__ offsets,
@@ -42,8 +44,8 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
   pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;                   // [E]  running cursor per expert
-  int32_t* whist = sm + E;             // [32][E] per-warp counts -> exclusive bases
-  int32_t* flag = sm + (kPermWarps + 1) * E;
+  int32_t* flag = sm + E;
+  int32_t* whist = sm + E + 4;         // [32][E] per-warp counts -> exclusive bases
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = T * k;
 
@@ -115,7 +117,22 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
   }
   __syncthreads();
 
-  // stable placement, chunk by chunk
+  // stable placement; at most 32 pairs: one warp, ranks from its match masks
+  if (R <= 32) {
+    if (warp == 0) {
+      const int e = (lane < R) ? idx[lane] : -1;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      if (e >= 0) {
+        const int pos = cnt[e] + __popc(peers & ((1u << lane) - 1u));
+        const int t = lane / k;
+        row_token[pos] = t;
+        row_slot[pos] = lane - t * k;
+        slot_row[lane] = pos;
+      }
+    }
+    return;
+  }
+  // chunk by chunk
   for (int base = 0; base < R; base += kPermThreads) {
     for (int i = tid; i < kPermWarps * E; i += kPermThreads) whist[i] = 0;
     __syncthreads();

@@ -1,8 +1,9 @@
 // Router tail: softmax top-k with renormalised weights (rabbit README, model
 // table row "MoE routing": softmax top-10 of 512).
 //
-// One CTA per token. The router logits arrive as split-K partial sums
-// [S, T, E] from k_dense_gemv and are summed in a fixed order (s = 0..S-1),
+// One CTA per token, one thread per expert. The router logits arrive as
+// split-K partial sums [S, T, E] from the router GEMM and are summed in a
+// fixed order (s = 0..S-1),
 // so the logits, and with them the selection, are reproducible run to run.
 // Selection ranks by fp32 logit (the softmax is monotone); equal logits go to
 // the lower expert index. Weights: w_j = exp(l_j - l_max) / sum_sel exp(l - l_max),
@@ -14,62 +15,82 @@
 
 namespace moe {
 
-constexpr int kMaxPerLane = 32;   // E <= 1024
-
-// grid T, block 256: the CTA sums the S partial logits of its token (all
-// threads, independent loads), then warp 0 selects the top k.
-__global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, int S, int T, int E,
-                                              int k, int32_t* __restrict__ idx,
-                                              float* __restrict__ w, float* __restrict__ logits) {
+// grid T, block kTopkThreads (one thread per expert, E <= 1024):
+// 1) thread e sums the S partial logits of expert e in a fixed order;
+// 2) the k-th largest logit is found by a bitwise search over order-preserving
+//    32-bit keys (one CTA-wide count per bit);
+// 3) the experts above it are taken, then experts equal to it by ascending
+//    index until k are taken;
+// 4) warp 0 orders the k by descending logit, equal logits by ascending index,
+//    and computes the renormalised weights.
+__global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ part, int S, int T,
+                                                     int E, int k, int32_t* __restrict__ idx,
+                                                     float* __restrict__ w,
+                                                     float* __restrict__ logits) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float lg[1024];
+  __shared__ int s_cnt[kTopkThreads / 32];
+  __shared__ uint32_t s_key[32];
+  __shared__ int s_exp[32];
+  __shared__ float s_val[32];
   const int tok = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += 256) {
-    const float* p = part + (size_t)tok * E + e;
-    const size_t stride = (size_t)T * E;
-    float acc = 0.0f;
-    int s = 0;
-    for (; s + 4 <= S; s += 4) {                // fixed summation order s = 0, 1, 2, ...
-      const float v0 = __ldg(p + (s + 0) * stride), v1 = __ldg(p + (s + 1) * stride);
-      const float v2 = __ldg(p + (s + 2) * stride), v3 = __ldg(p + (s + 3) * stride);
-      acc += v0; acc += v1; acc += v2; acc += v3;
-    }
-    for (; s < S; ++s) acc += __ldg(p + s * stride);
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const bool live = e < E;
+  float acc = 0.0f;
+  if (live) {
+    acc = sum_splits(part + (size_t)tok * E + e, S, (size_t)T * E);
     if (logits) logits[(size_t)tok * E + e] = acc;
-    lg[e] = isnan(acc) ? -INFINITY : acc;      // a NaN logit never wins
+  }
+  // a NaN logit never wins; -0 ranks equal to +0
+  const float v = (live && !isnan(acc)) ? (acc == 0.0f ? 0.0f : acc) : -INFINITY;
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+
+  // largest thr with #{key >= thr} >= k: the k-th largest key
+  uint32_t thr = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t c = thr | (1u << b);
+    if (__syncthreads_count(live && key >= c) >= k) thr = c;
+  }
+  const bool gt = live && key > thr, eq = live && key == thr;
+  const int n_gt = __syncthreads_count(gt);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const unsigned eq_m = __ballot_sync(0xFFFFFFFFu, eq);
+  if (lane == 0) s_cnt[warp] = __popc(eq_m);
+  __syncthreads();
+  int before = __popc(eq_m & lt_mask);
+  for (int w2 = 0; w2 < warp; ++w2) before += s_cnt[w2];
+  const bool sel = gt || (eq && before < k - n_gt);
+  const unsigned sel_m = __ballot_sync(0xFFFFFFFFu, sel);
+  __syncthreads();
+  if (lane == 0) s_cnt[warp] = __popc(sel_m);
+  __syncthreads();
+  if (sel) {
+    int pos = __popc(sel_m & lt_mask);
+    for (int w2 = 0; w2 < warp; ++w2) pos += s_cnt[w2];
+    s_key[pos] = key;
+    s_exp[pos] = e;
+    s_val[pos] = v;
   }
   __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  float v[kMaxPerLane];
-#pragma unroll
-  for (int j = 0; j < kMaxPerLane; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (e < E) ? lg[e] : -INFINITY;
+  if (warp != 0) return;
+  // lane i < k: its rank among the k taken (descending key, then ascending index)
+  uint32_t ki = 0;
+  int ei = 0;
+  float vi = 0.0f;
+  if (lane < k) { ki = s_key[lane]; ei = s_exp[lane]; vi = s_val[lane]; }
+  int rank = 0;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t kj = s_key[j];
+    const int ej = s_exp[j];
+    rank += (kj > ki || (kj == ki && ej < ei)) ? 1 : 0;
   }
-  uint32_t taken = 0;
-  float selv = 0.0f;     // lane r keeps the r-th selection
-  int sele = 0;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u)) {
-        if (v[j] > bv || be == 0x7FFFFFFF) { bv = v[j]; be = e; }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == r) { selv = bv; sele = be; }
-  }
+  __syncwarp();
+  if (lane < k) { s_exp[rank] = ei; s_val[rank] = vi; }
+  __syncwarp();
+  // lane r now holds the r-th selection
+  const float selv = (lane < k) ? s_val[lane] : 0.0f;
+  const int sele = (lane < k) ? s_exp[lane] : 0;
   const float m = __shfl_sync(0xFFFFFFFFu, selv, 0);
   const float ex = (lane < k) ? expf(selv - m) : 0.0f;
   float den = ex;

@@ -31,12 +31,17 @@ LATENT_SMALL = synth.MoeWorkload("latent_small", T=5, H=384, I=128, E=12, k=3, I
 # T >= 128: router and shared expert on the tcgen05 bf16 GEMM (E = 6 < 128 rows,
 # I_shared = 384 = three 128-row tiles, H = 640 = two 256-row pairs + one tile)
 WIDE = synth.MoeWorkload("wide_tc", T=260, H=640, I=256, E=6, k=2, I_shared=384, seed=79)
+# one token with K multiples of 1024: router, sigmoid gate and shared expert on
+# the whole-row CUDA-core GEMV (E = 10 router rows: the last stage holds two;
+# the sigmoid-gate row is a segment of its own)
+ROWS_T1 = synth.MoeWorkload("rows_t1", T=1, H=2048, I=256, E=10, k=3, I_shared=1024, seed=80)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
     (MEDIUM, None),
     (LATENT_SMALL, None),
     (WIDE, None),
+    (ROWS_T1, None),
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
