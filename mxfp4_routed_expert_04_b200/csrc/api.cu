@@ -331,7 +331,7 @@ moe_status do_permute(const Plan& p, const int32_t* idx, const uint16_t* xin, in
 // CUDA-core GEMV launch shape for reduction length K (up to 8192): lanes own
 // BPL = ceil(K/1024) blocks; one CTA per SM with a ring of MOE_FMA_SMEM_KB KB.
 #ifndef MOE_FMA_SMEM_KB
-#define MOE_FMA_SMEM_KB 210
+#define MOE_FMA_SMEM_KB 224
 #endif
 struct FmaPlan {
   int bpl = 0;

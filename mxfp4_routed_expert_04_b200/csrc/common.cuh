@@ -140,10 +140,34 @@ MOE_DEV uint32_t lds8(uint32_t addr) {
   asm volatile("ld.shared.u8 %0, [%1];\n" : "=r"(v) : "r"(addr));
   return v;
 }
+MOE_DEV uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+MOE_DEV void sts16(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+MOE_DEV void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // misc
 // ---------------------------------------------------------------------------
+// Exponent of m = f * 2^e with f in [0.5, 1) for finite m > 0, read from the
+// IEEE-754 fields (subnormals by their leading one).
+MOE_DEV int frexp_exponent(float m) {
+  const uint32_t b = __float_as_uint(m);
+  const int e = (int)((b >> 23) & 0xFFu);
+  return e != 0 ? e - 126 : (31 - __clz((int)(b & 0x7FFFFFu))) - 148;
+}
+// 2^n as fp32 for n in [-149, 127], built from its bit pattern
+MOE_DEV float pow2_f32(int n) {
+  return n >= -126 ? __uint_as_float((uint32_t)(n + 127) << 23) : __uint_as_float(1u << (n + 149));
+}
+
 // Sum of S split-K partials p[0], p[stride], ... in the order s = 0, 1, ...;
 // the loads are issued sixteen at a time ahead of their additions.
 MOE_DEV float sum_splits(const float* __restrict__ p, int S, size_t stride) {

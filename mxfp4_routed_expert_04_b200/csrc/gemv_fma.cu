@@ -78,16 +78,20 @@ MOE_DEV float warp_max(float v) {
 
 // ---------------------------------------------------------------------------
 // block = 32 * (kFmaConsumers + 1) threads (warp 0: producer); one CTA per SM;
-// dynamic shared memory = g.nst * g.stage_bytes
+// dynamic shared memory = g.smem_bytes (the ring, then the activation buffer
+// at g.act_off).
+// The producer waits for the previous kernel (griddepcontrol.wait) only before
+// it copies an activation row (x from the dispatch, h from the gate/up
+// kernel), which goes out ahead of the weights of its first stage.
 // ---------------------------------------------------------------------------
 template <int BPL, bool kGateUp, int RPS>
 __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArgs a, FmaGeometry g) {
-  pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
   __shared__ int s_wsum[kFmaConsumers + 1];
   __shared__ uint64_t s_bars[2 * kFmaMaxStages];
+  __shared__ uint64_t s_act[3];         // activation buffer: [0] full, [1] empty, [2] down: h converted
   __shared__ int s_abort;
   __shared__ float2 s_part[2][kFmaConsumers / 2][2];   // gate/up partial sums [stage&1][pair][half]
   constexpr int kWarps = kFmaConsumers + 1;
@@ -98,16 +102,18 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   const uint32_t qrow = (uint32_t)K / 2, srow = (uint32_t)K / 32;
   const int N = kGateUp ? a.I : a.W;                      // rows of one matrix
   const size_t s_total = (size_t)a.E * N * srow;          // bytes of a stacked E8M0 array
+  uint8_t* act = smem + g.act_off;
 
-  // 1) the single-token experts, in the order of the expert list
-  const int n_act = __ldg(a.expert_list);
+  // 1) the single-token experts, in the order of the expert list (the
+  //    dispatch's output: complete before this grid can start, read through L2)
+  const int n_act = __ldcg(a.expert_list);
   int n_single = 0;
   for (int base = 0; base < n_act; base += 32 * kWarps) {
     const int i = base + threadIdx.x;
     int e = -1;
     if (i < n_act) {
-      e = __ldg(a.expert_list + 1 + i);
-      if (__ldg(a.offsets + e + 1) - __ldg(a.offsets + e) != 1) e = -1;
+      e = __ldcg(a.expert_list + 1 + i);
+      if (__ldcg(a.offsets + e + 1) - __ldcg(a.offsets + e) != 1) e = -1;
     }
     const unsigned m = __ballot_sync(0xFFFFFFFFu, e >= 0);
     if (lane == 0) s_wsum[warp] = __popc(m);
@@ -130,6 +136,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kFmaConsumers);
     }
+    mbar_init(&s_act[0], 1);
+    mbar_init(&s_act[1], kFmaConsumers);
+    mbar_init(&s_act[2], 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -140,6 +149,11 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   // si, row r within it, ring slot and phase): no division per stage
   const int si0 = (int)(lo / N), r_lo = (int)(lo - (long)si0 * N);
   auto stage_units = [&](long u, int r) -> int { return (int)min((long)min(P, N - r), hi - u); };
+  // the activation row of expert slot si: gate/up -> its token's f16 row
+  // (key = token), down -> the expert's h row (key = slot)
+  auto act_key = [&](int si) -> int {
+    return kGateUp ? __ldcg(a.row_token + __ldcg(a.offsets + s_list[si])) : si;
+  };
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -148,11 +162,47 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       bool filled[kFmaMaxStages];
 #pragma unroll
       for (int s = 0; s < kFmaMaxStages; ++s) { last_ph[s] = 0; filled[s] = false; }
-      int si = si0, r = r_lo, slot = 0;
+      int si = si0, r = r_lo, slot = 0, k = 0;
       uint32_t ph = 0;
-      for (long u = lo; u < hi;) {
+      // activation rows: the slots whose row is still to be copied, in order
+      int pend[4], n_pend = 0, n_loaded = 0, cur_key = -1, cur_si = -1;
+      bool waited = false, ok = true;
+      auto load_acts = [&]() -> bool {        // after the wait: copy the pending rows
+        if (!waited) {
+          pdl_wait();
+          asm volatile("fence.proxy.async;\n" ::: "memory");   // the previous grid's writes, then bulk reads
+          waited = true;
+        }
+        for (int i = 0; i < n_pend; ++i) {
+          if (n_loaded > 0 && !tc::wait_or_abort(&s_act[1], (uint32_t)((n_loaded - 1) & 1), abort))
+            return false;
+          const int sp = pend[i];
+          const int r0 = __ldcg(a.offsets + s_list[sp]);
+          const uint32_t bytes = kGateUp ? (uint32_t)a.W * 2 : (uint32_t)a.I * 4;
+          const void* src = kGateUp ? static_cast<const void*>(a.x16 + (size_t)__ldcg(a.row_token + r0) * a.W)
+                                    : static_cast<const void*>(a.h32 + (size_t)r0 * a.I);
+          fence_proxy_async_smem();
+          mbar_expect_tx(&s_act[0], bytes);
+          bulk_g2s(act, src, bytes, &s_act[0]);
+          ++n_loaded;
+        }
+        n_pend = 0;
+        return true;
+      };
+      for (long u = lo; u < hi && ok; ++k) {
         const int n = stage_units(u, r);
-        if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) break;
+        if (si != cur_si) {                   // a new expert: a new activation row?
+          cur_si = si;
+          const int key = act_key(si);
+          if (key != cur_key) {
+            cur_key = key;
+            pend[n_pend++] = si;
+          }
+        }
+        // a new activation row goes out ahead of the stage's weights (it is
+        // small, and the consumers need it before the stage)
+        if (n_pend > 0 && !load_acts()) { ok = false; break; }
+        if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) { ok = false; break; }
         const size_t row = (size_t)s_list[si] * N + r;
         const uint32_t cb = n * qrow;
         const size_t s0 = row * srow, s1 = (row + n) * srow;
@@ -178,9 +228,12 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
         if (r == N) { r = 0; ++si; }
         if (++slot == g.nst) { slot = 0; ph ^= 1u; }
       }
+      if (ok && n_pend > 0 && !load_acts()) ok = false;
+      if (!waited) pdl_wait();
       if (*abort) {     // let every issued copy land before the CTA can exit
         for (int s = 0; s < g.nst; ++s)
           if (filled[s]) mbar_wait(&full[s], last_ph[s]);
+        if (n_loaded > 0) mbar_wait(&s_act[0], (uint32_t)((n_loaded - 1) & 1));
       }
     }
   } else {
@@ -188,73 +241,101 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
     // gate/up: warps 2p and 2p+1 share row pair p of a stage, each over one
     // half of K (half the activation registers), and combine their partial
     // sums through shared memory; down: warp w takes rows RPS*w ... of a stage
+    pdl_wait();                             // the previous grid's outputs (xscale)
     const int w = warp - 1;
     constexpr int BW = kGateUp ? (BPL + 1) / 2 : BPL;    // blocks per lane of this warp
     const int half = kGateUp ? (w & 1) : 0;
     const int KBw = kGateUp ? KB / 2 : KB;                // blocks of this warp's K range
     const int kb0 = half * KBw;                           // its first block
     uint32_t xr[BW][16];
+    float bsc[BW];                                        // down: per-block scale of h
+#pragma unroll
+    for (int j = 0; j < BW; ++j) bsc[j] = 1.0f;
     float xs = 1.0f;
-    int cur_e = -1, r0 = 0;
+    int cur_key = -1, cur_si = -1, r0 = 0;
     int si = si0, r = r_lo, slot = 0, k = 0;
-    uint32_t ph = 0;
+    uint32_t ph = 0, act_seen = 0;
     for (long u = lo; u < hi; ++k) {
       const int n = stage_units(u, r);
       const int e = s_list[si];
-      if (e != cur_e) {                     // new expert: load its activation row
-        cur_e = e;
-        r0 = __ldg(a.offsets + e);
-        if (kGateUp) {
-          const int tok = __ldg(a.row_token + r0);
-          const __half* xrow = a.x16 + (size_t)tok * a.W;
+      bool new_act = false;
+      if (si != cur_si) {                     // a new expert: its row, and maybe a new activation row
+        cur_si = si;
+        r0 = __ldcg(a.offsets + e);
+        const int key = act_key(si);
+        new_act = key != cur_key;
+        cur_key = key;
+      }
+      if (new_act) {                          // the new activation row: into registers
+        if (kGateUp) xs = __ldg(a.xscale + __ldcg(a.row_token + r0));   // while the row is in flight
+        if (!tc::wait_or_abort(&s_act[0], act_seen & 1u, abort)) break;
+        const uint32_t ab = smem_u32(act);
+        // a lane's block is 64 contiguous bytes of f16 (gate/up: the token
+        // row; down: the converted h row); the lanes visit its 16-byte chunks
+        // in a rotated order so that each access spreads over all banks
+        uint32_t xb = ab;
+        if (!kGateUp) {
+          // warp 0 converts the fp32 h row once: block b -> f16 with the
+          // block's own power-of-two scale (its largest |h| into [2^14, 2^15))
+          const uint32_t h16 = ab + (uint32_t)K * 4u, hsc = h16 + (uint32_t)K * 2u;
+          if (w == 0) {
+            for (int b = lane; b < KB; b += 32) {
+              const uint32_t hb = ab + (uint32_t)b * 128u;
+              float m = 0.0f;
 #pragma unroll
-          for (int j = 0; j < BW; ++j) {
-            const int b = lane + 32 * j;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 t = make_uint4(0u, 0u, 0u, 0u);
-              if (b < KBw) t = ldg16(xrow + (kb0 + b) * 32 + 8 * q);
-              xr[j][4 * q] = t.x; xr[j][4 * q + 1] = t.y; xr[j][4 * q + 2] = t.z; xr[j][4 * q + 3] = t.w;
-            }
-          }
-          xs = __ldg(a.xscale + tok);
-        } else {
-          // h32 row -> f16 with one power-of-two scale for the row
-          const float* hrow = a.h32 + (size_t)r0 * a.I;
-          float m = 0.0f;
-#pragma unroll
-          for (int j = 0; j < BW; ++j) {
-            const int b = lane + 32 * j;
-            if (b < KB)
               for (int q = 0; q < 8; ++q) {
-                const float4 t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
-                m = fmaxf(m, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+                const uint4 v = lds16(hb + 16u * ((q + lane) & 7));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                                   fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
               }
+              float inv = 1.0f, sc = 1.0f;
+              if (m > 0.0f && isfinite(m)) {
+                const int ex = max(-100, min(127, frexp_exponent(m)));
+                sc = pow2_f32(ex - 15);
+                inv = pow2_f32(15 - ex);
+              }
+              sts32(hsc + 4u * b, __float_as_uint(sc));
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {          // 16 bytes of f16 from 32 bytes of fp32
+                const int qq = (q + (lane >> 1)) & 3;
+                const uint4 v0 = lds16(hb + 32u * qq), v1 = lds16(hb + 32u * qq + 16u);
+                const __half2 p0 = __floats2half2_rn(__uint_as_float(v0.x) * inv, __uint_as_float(v0.y) * inv);
+                const __half2 p1 = __floats2half2_rn(__uint_as_float(v0.z) * inv, __uint_as_float(v0.w) * inv);
+                const __half2 p2 = __floats2half2_rn(__uint_as_float(v1.x) * inv, __uint_as_float(v1.y) * inv);
+                const __half2 p3 = __floats2half2_rn(__uint_as_float(v1.z) * inv, __uint_as_float(v1.w) * inv);
+                sts16(h16 + (uint32_t)b * 64u + 16u * qq,
+                      make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+                                 *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3)));
+              }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&s_act[2]);
           }
-          m = warp_max(m);
-          float inv = 1.0f;
-          xs = 1.0f;
-          if (m > 0.0f && isfinite(m)) {
-            int ex;
-            frexpf(m, &ex);
-            ex = max(-100, min(127, ex));
-            xs = ldexpf(1.0f, ex - 15);
-            inv = ldexpf(1.0f, 15 - ex);
-          }
+          if (!tc::wait_or_abort(&s_act[2], act_seen & 1u, abort)) break;
+          xb = h16;
 #pragma unroll
           for (int j = 0; j < BW; ++j) {
             const int b = lane + 32 * j;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (b < KB) t = __ldg(reinterpret_cast<const float4*>(hrow + b * 32) + q);
-              const __half2 l2 = __floats2half2_rn(t.x * inv, t.y * inv);
-              const __half2 h2 = __floats2half2_rn(t.z * inv, t.w * inv);
-              xr[j][2 * q] = *reinterpret_cast<const uint32_t*>(&l2);
-              xr[j][2 * q + 1] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
+            bsc[j] = b < KB ? __uint_as_float(lds32(hsc + 4u * b)) : 1.0f;
           }
         }
+        ++act_seen;
+        const int kbx = kGateUp ? kb0 : 0;
+#pragma unroll
+        for (int j = 0; j < BW; ++j) {
+          const int b = lane + 32 * j;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int qq = (q + (lane >> 1)) & 3;
+            uint4 t = make_uint4(0u, 0u, 0u, 0u);
+            if (b < KBw) t = lds16(xb + (uint32_t)(kbx + b) * 64u + 16u * qq);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+              if (qq == s) { xr[j][4 * s] = t.x; xr[j][4 * s + 1] = t.y; xr[j][4 * s + 2] = t.z; xr[j][4 * s + 3] = t.w; }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&s_act[1]);   // this warp is done with the buffer
       }
       if (!tc::wait_or_abort(&full[slot], ph, abort)) break;
       const uint32_t st = smem_u32(smem + (size_t)slot * g.stage_bytes);
@@ -286,7 +367,8 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
               if (kGateUp || u0 + rr < n) {
                 const uint4 wv = lds16(cb[rr] + 512u * j);
                 const uint32_t code = lds8(sbs[rr] + 32u * j);
-                acc[rr] = fmaf(dot_block(wv, xr[j]), e8m0_exact(code), acc[rr]);
+                const float sc = kGateUp ? e8m0_exact(code) : e8m0_exact(code) * bsc[j];
+                acc[rr] = fmaf(dot_block(wv, xr[j]), sc, acc[rr]);
               }
             }
           }
@@ -305,7 +387,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
           for (int rr = 0; rr < NR; ++rr) {
             if (u0 + rr < n) {
               const float sum = warp_sum(acc[rr]);
-              if (lane == 0) a.y_perm[(size_t)r0 * a.W + r + u0 + rr] = sum * xs;
+              if (lane == 0) a.y_perm[(size_t)r0 * a.W + r + u0 + rr] = sum;
             }
           }
         }
@@ -326,7 +408,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 // down stage rps = max(1, 8 / BPL); a stage holds kFmaConsumers / 2 row pairs
 // (gate/up: the gate rows, then the up rows, then the two E8M0 spans) or
 // kFmaConsumers * rps rows (down: codes, then their span); every span with 32
-// bytes of alignment slack; ring depth nst from the shared-memory budget.
+// bytes of alignment slack; after the ring the activation buffer (gate/up: an
+// f16 token row of K; down: an fp32 h row of K, its f16 copy and K/32 fp32
+// block scales); ring depth nst from the shared-memory budget.
 FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   FmaGeometry g{};
   const size_t qrow = K / 2, srow = K / 32;
@@ -342,10 +426,13 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   g.sbuf_off = code_all;
   g.sbuf2_off = code_all + span;
   g.stage_bytes = code_all + (gate_up ? 2 : 1) * span;
-  int nst = (int)(smem_budget / g.stage_bytes);
-  if (nst < 2) return g;
+  // gate/up: the f16 token row; down: the fp32 h row, its f16 copy, the block scales
+  const uint32_t act_bytes = (uint32_t)(((size_t)K * (gate_up ? 2 : 6) + (gate_up ? 0 : K / 8) + 127) / 128 * 128);
+  if (smem_budget < act_bytes + 2 * (size_t)g.stage_bytes) return g;
+  const int nst = (int)((smem_budget - act_bytes) / g.stage_bytes);
   g.nst = nst > kFmaMaxStages ? kFmaMaxStages : nst;
-  g.smem_bytes = (uint32_t)(g.nst * g.stage_bytes);
+  g.act_off = (uint32_t)g.nst * g.stage_bytes;
+  g.smem_bytes = g.act_off + act_bytes;
   g.ok = 1;
   return g;
 }

@@ -90,11 +90,9 @@ MOE_DEV void decode_block(uint32_t wg, uint32_t wg8, uint32_t (&a0)[4], uint32_t
 // power-of-two scale mapping a block maximum m into [2^14, 2^15) as f16
 MOE_DEV void f16_block_scale(float m, float& scale, float& inv) {
   if (!(m > 0.0f) || !isfinite(m)) { scale = 1.0f; inv = 1.0f; return; }
-  int ex;
-  frexpf(m, &ex);                      // m = f * 2^ex, f in [0.5, 1)
-  ex = max(-100, min(127, ex));
-  scale = ldexpf(1.0f, ex - 15);
-  inv = ldexpf(1.0f, 15 - ex);
+  const int ex = max(-100, min(127, frexp_exponent(m)));   // m = f * 2^ex, f in [0.5, 1)
+  scale = pow2_f32(ex - 15);
+  inv = pow2_f32(15 - ex);
 }
 
 }  // namespace

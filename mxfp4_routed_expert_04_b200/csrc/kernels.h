@@ -58,10 +58,10 @@ struct FmaArgs {
 // Launch geometry: rps rows per consumer warp of a down stage, units per stage
 // (gate/up: row pairs; down: rows), code_bytes = one matrix's codes of a
 // stage, sbuf_off / sbuf2_off = offsets of the E8M0 spans (the second:
-// gate/up only), nst ring stages.
+// gate/up only), nst ring stages, act_off = the activation row buffer.
 struct FmaGeometry {
   int ok, rps, nst, units;
-  uint32_t code_bytes, sbuf_off, sbuf2_off, stage_bytes, smem_bytes;
+  uint32_t code_bytes, sbuf_off, sbuf2_off, stage_bytes, act_off, smem_bytes;
 };
 FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget);
 template <int BPL, bool kGateUp, int RPS> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);

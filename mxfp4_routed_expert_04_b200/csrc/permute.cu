@@ -198,11 +198,9 @@ __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__
   m = block_max_256(m);
   float scale = 1.0f, inv = 1.0f;
   if (m > 0.0f && isfinite(m)) {
-    int ex;
-    frexpf(m, &ex);
-    ex = max(-100, min(127, ex));
-    scale = ldexpf(1.0f, ex - 15);
-    inv = ldexpf(1.0f, 15 - ex);
+    const int ex = max(-100, min(127, frexp_exponent(m)));
+    scale = pow2_f32(ex - 15);
+    inv = pow2_f32(15 - ex);
   }
   for (int i = threadIdx.x * 8; i < W; i += 256 * 8) {
     const uint4 v = ldg16(row + i);
