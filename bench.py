@@ -90,11 +90,15 @@ def layer_flops(w):
     return f
 
 
-def _csrc_digest():
+# sources of the single-token expert kernels whose DRAM counters profiles/traffic.json holds
+TRAFFIC_SOURCES = ("gemv_fma.cu", "common.cuh", "tc05.cuh")
+
+
+def _csrc_digest(files=TRAFFIC_SOURCES):
     import hashlib
     d = os.path.join(ROOT, "mxfp4_routed_expert_04_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
+    for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -102,7 +106,7 @@ def _csrc_digest():
 
 def _traffic(workload):
     """DRAM bytes per moe_expert_ffn call from the committed ncu summary, if it
-    was taken on the current kernel sources (else None)."""
+    was taken on the current sources of those kernels (else None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
@@ -245,11 +249,16 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     n_active = int((layer.counts > 0).sum())
 
-    # kernels enqueued by one moe_layer call: router 2, permute 2, shared expert 3,
-    # combine 1, routed experts 4 (bf16: two GEMV pairs; 2 for one token, whose
-    # experts all have a single token) or 3 (mxfp4: tile list + two tcgen05
-    # GEMMs), latent projections 4
-    launches_per_step = 8 + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (4 if w.L else 0)
+    # kernels enqueued by one moe_layer call: router 2 (logits, top-k), permute 2
+    # (dispatch, activation operand), combine 1; shared expert 3 (gate/up,
+    # SwiGLU or sigmoid gate, down), or 2 for one token on the row GEMV (its
+    # sigmoid-gate row rides with the router); routed experts 4 (bf16: two GEMV
+    # pairs; 2 for one token, whose experts all have a single token) or 3
+    # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 4
+    rows_k = (1024, 2048, 4096, 8192)
+    rows_path = w.T == 1 and w.H in rows_k and w.I_shared in rows_k
+    launches_per_step = (5 + (2 if rows_path else 3) + (3 if act == "mxfp4" else (2 if w.T == 1 else 4))
+                         + (4 if w.L else 0))
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
