@@ -251,13 +251,15 @@ def run_ours(args, w):
 
     # kernels enqueued by one moe_layer call: router 2 (logits, top-k), permute 2
     # (dispatch, activation operand), combine 1; shared expert 3 (gate/up,
-    # SwiGLU or sigmoid gate, down), or 2 for one token on the row GEMV (its
-    # sigmoid-gate row rides with the router); routed experts 4 (bf16: two GEMV
+    # SwiGLU finaliser, down), or 2 for one token on the row GEMV and for 128+
+    # tokens (SwiGLU in the GEMM epilogue); routed experts 4 (bf16: two GEMV
     # pairs; 2 for one token, whose experts all have a single token) or 3
     # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 4
     rows_k = (1024, 2048, 4096, 8192)
     rows_path = w.T == 1 and w.H in rows_k and w.I_shared in rows_k
-    launches_per_step = (5 + (2 if rows_path else 3) + (3 if act == "mxfp4" else (2 if w.T == 1 else 4))
+    # (many tokens: the sigmoid-gate row rides with the router rows as well)
+    shared = 2 if (rows_path or w.T >= 128) else 3
+    launches_per_step = (5 + shared + (3 if act == "mxfp4" else (2 if w.T == 1 else 4))
                          + (4 if w.L else 0))
 
     def timed(fn, steps):

@@ -127,7 +127,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
     p.S_sd = 1;
   } else {
     const long ntt = (p.T + p.Nt - 1) / p.Nt;
-    p.S_router = tc_splits((long)((p.E + 255) / 256) * ntt, p.H, (size_t)p.T * p.E * 4);
+    p.S_router = tc_splits((long)((p.E + 255) / 256 + 1) * ntt, p.H, (size_t)p.T * (p.E + 1) * 4);
     // SwiGLU epilogue: one split, the sigmoid-gate row on the GEMV
     p.S_sgu = p.swiglu_tc ? 1
                           : tc_splits((long)(2 * ((p.Is + 255) / 256) + 1) * ntt, p.H,
@@ -139,7 +139,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 256); return r; };
   p.off_status = take(256);
-  p.off_router = take((size_t)p.S_router * p.T * p.E * 4);
+  p.off_router = take((size_t)p.S_router * p.T * (p.E + 1) * 4);   // + the sigmoid-gate column
   p.off_h16 = take((size_t)p.R * p.I * 2);
   p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
   p.off_h32 = take((size_t)p.R * p.I * 4);
@@ -443,21 +443,24 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
     r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
     if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
     launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
-               p.k, idx, w, logits);
+               p.E, p.k, idx, w, logits, (float*)nullptr);
     return launched("top-k");
   }
-  if (w_sgate) return fail(MOE_ERR_INVALID_ARG, "internal: sigmoid gate only with the row GEMV");
+  // many tokens: the router rows (and the sigmoid-gate row as a second
+  // segment, column E of the partial sums) on the tcgen05 GEMM
   moe::Bf16GemmArgs g;
   memset(&g, 0, sizeof(g));
   if ((s = bf16_map(&g.map_a[0], wr, p.E, p.H, "router weights")) != MOE_OK ||
-      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK)
+      (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK ||
+      (w_sgate && (s = bf16_map(&g.map_a[1], w_sgate, 1, p.H, "sigmoid-gate weights")) != MOE_OK))
     return s;
+  const int ld = w_sgate ? p.E + 1 : p.E;
   g.out = part; g.status = at<int32_t>(ws, p.off_status);
   g.mode = moe::kBf16Plain; g.K = p.H; g.T = p.T; g.S = p.S_router; g.passes = 1; g.N = p.Nt;
-  g.seg_rows[0] = p.E; g.ld = p.E;
+  g.seg_rows[0] = p.E; g.seg_rows[1] = w_sgate ? 1 : 0; g.ld = ld;
   if ((s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)")) != MOE_OK) return s;
-  launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E, p.k, idx, w,
-             logits);
+  launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E,
+             ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr);
   return launched("top-k");
 }
 
@@ -500,9 +503,24 @@ moe_status do_shared_up(const Plan& p, const DeviceState& ds, const uint16_t* x,
     g.seg_rows[0] = p.Is;
     g.h_hi = h_hi; g.h_lo = h_lo;
     if ((s = launch_bf16_gemm(ds, g, st, "shared gate/up gemm (tcgen05)", false)) != MOE_OK) return s;
-    if ((s = launch_dense(w_sgate, 1, nullptr, 0, nullptr, 0, x, false, at<float>(ws, p.off_gl), p.T,
-                          p.H, 1, st, "shared gate gemv")) != MOE_OK)
-      return s;
+    // the sigmoid-gate row: with the router rows in moe_layer; else alone on
+    // the same GEMM geometry (tile, splits, K order) and summed in the same
+    // order, so that both give the same bits (partials in the router region)
+    if (!sgate_done) {
+      moe::Bf16GemmArgs q;
+      memset(&q, 0, sizeof(q));
+      if ((s = bf16_map(&q.map_a[0], w_sgate, 1, p.H, "sigmoid-gate weights")) != MOE_OK ||
+          (s = bf16_map(&q.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK)
+        return s;
+      float* part = at<float>(ws, p.off_router);
+      q.out = part; q.status = status;
+      q.mode = moe::kBf16Plain; q.K = p.H; q.T = p.T; q.S = p.S_router; q.passes = 1; q.N = p.Nt;
+      q.seg_rows[0] = 1; q.ld = 1;
+      if ((s = launch_bf16_gemm(ds, q, st, "sigmoid-gate gemm (tcgen05)")) != MOE_OK) return s;
+      launch_pdl(moe::k_sum_column, dim3((p.T + moe::kFinThreads - 1) / moe::kFinThreads), dim3(moe::kFinThreads),
+                 0, st, (const float*)part, p.S_router, p.T, 1, 0, at<float>(ws, p.off_gl));
+      if ((s = launched("sigmoid-gate sum")) != MOE_OK) return s;
+    }
   } else {
     if ((s = bf16_map(&g.map_a[2], w_sgate, 1, p.H, "shared sigmoid-gate weights")) != MOE_OK) return s;
     float* sgu = at<float>(ws, p.off_sgu);
@@ -874,8 +892,9 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
   // main stream first: the router's CTAs are queued before the shared expert's
   // (one token: the sigmoid-gate row rides along with the router rows)
+  const bool sgate_with_router = p.rows || p.swiglu_tc;
   if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st,
-                    p.rows ? a->w_sgate : nullptr)) != MOE_OK)
+                    sgate_with_router ? a->w_sgate : nullptr)) != MOE_OK)
     return s;
   // side stream: latent projection, then the first half of the shared expert
   // (it streams its weights while the routing chain runs)
@@ -887,7 +906,7 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
       return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   }
   // (the row GEMV leaves a few SMs to the routing chain's small kernels)
-  if ((s = do_shared_up(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, ws, ds->side, p.rows,
+  if ((s = do_shared_up(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, ws, ds->side, sgate_with_router,
                         ds->num_sms - kRowsFreeSMs)) != MOE_OK)
     return s;
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)

@@ -94,6 +94,17 @@ __global__ void __launch_bounds__(kFinThreads) k_shared_swiglu(const float* __re
     gate_logit[t] = sum_splits(part + (size_t)t * N + 2 * Is, S, (size_t)T * N);
 }
 
+// out[t] = sum_s part[(s * T + t) * ld + col]   (the sigmoid-gate logit from
+// the split-K partials of its row, summed in the order the top-k kernel uses)
+// grid ceil(T/kFinThreads), block kFinThreads
+__global__ void __launch_bounds__(kFinThreads) k_sum_column(const float* __restrict__ part, int S, int T,
+                                                          int ld, int col, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int t = blockIdx.x * kFinThreads + threadIdx.x;
+  if (t < T) out[t] = sum_splits(part + (size_t)t * ld + col, S, (size_t)T * ld);
+}
+
 // out[t, n] = bf16_rne( sum_s part[s, t, n] )   (latent down-projection)
 // grid (ceil(N/kFinThreads), T), block kFinThreads
 __global__ void __launch_bounds__(kFinThreads) k_round_bf16(const float* __restrict__ part, int S,

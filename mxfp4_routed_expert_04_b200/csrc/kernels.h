@@ -167,8 +167,10 @@ constexpr int kDenseWarps = 4;   // warps (16-row tiles) per CTA
 
 // --- router tail ------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
-__global__ void k_topk(const float* part, int S, int T, int E, int k, int32_t* idx, float* w,
-                       float* logits);
+// part [S, T, ld] router partial sums (ld >= E); with gate_logit set, column E
+// holds the sigmoid-gate row's partials and gate_logit[t] gets their sum
+__global__ void k_topk(const float* part, int S, int T, int E, int ld, int k, int32_t* idx, float* w,
+                       float* logits, float* gate_logit);
 
 // --- permutation and activation operands ------------------------------------
 __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
@@ -186,6 +188,7 @@ constexpr int kFinThreads = 64;
 __global__ void k_shared_swiglu(const float* part, int S, int T, int Is, uint16_t* h_hi,
                                 uint16_t* h_lo, float* gate_logit);
 __global__ void k_round_bf16(const float* part, int S, int T, int N, uint16_t* out);
+__global__ void k_sum_column(const float* part, int S, int T, int ld, int col, float* out);
 
 struct CombineArgs {
   const float* y_perm;       // [R, width] or NULL

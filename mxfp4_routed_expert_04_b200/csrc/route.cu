@@ -16,7 +16,8 @@
 namespace moe {
 
 // grid T, block kTopkThreads (one thread per expert, E <= 1024):
-// 1) thread e sums the S partial logits of expert e in a fixed order;
+// 1) thread e sums the S partial logits of expert e in a fixed order (and
+//    thread E the sigmoid-gate row's, when it rides along);
 // 2) the k-th largest logit is found by a bitwise search over order-preserving
 //    32-bit keys (one CTA-wide count per bit);
 // 3) the experts above it are taken, then experts equal to it by ascending
@@ -24,9 +25,10 @@ namespace moe {
 // 4) warp 0 orders the k by descending logit, equal logits by ascending index,
 //    and computes the renormalised weights.
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ part, int S, int T,
-                                                     int E, int k, int32_t* __restrict__ idx,
+                                                     int E, int ld, int k, int32_t* __restrict__ idx,
                                                      float* __restrict__ w,
-                                                     float* __restrict__ logits) {
+                                                     float* __restrict__ logits,
+                                                     float* __restrict__ gate_logit) {
   pdl_wait();
   pdl_trigger();
   __shared__ int s_cnt[kTopkThreads / 32];
@@ -38,9 +40,10 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   const bool live = e < E;
   float acc = 0.0f;
   if (live) {
-    acc = sum_splits(part + (size_t)tok * E + e, S, (size_t)T * E);
+    acc = sum_splits(part + (size_t)tok * ld + e, S, (size_t)T * ld);
     if (logits) logits[(size_t)tok * E + e] = acc;
   }
+  if (gate_logit && e == E) gate_logit[tok] = sum_splits(part + (size_t)tok * ld + E, S, (size_t)T * ld);
   // a NaN logit never wins; -0 ranks equal to +0
   const float v = (live && !isnan(acc)) ? (acc == 0.0f ? 0.0f : acc) : -INFINITY;
   const uint32_t u = __float_as_uint(v);
