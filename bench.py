@@ -259,8 +259,11 @@ def run_ours(args, w):
     rows_path = w.T == 1 and w.H in rows_k and w.I_shared in rows_k
     # (many tokens: the sigmoid-gate row rides with the router rows as well)
     shared = 2 if (rows_path or w.T >= 128) else 3
-    launches_per_step = (5 + shared + (3 if act == "mxfp4" else (2 if w.T == 1 else 4))
-                         + (4 if w.L else 0))
+    # (one token, no latent projection, I_shared <= 2048: the combine runs in
+    # the shared down launch)
+    fused_combine = rows_path and not w.L and w.I_shared <= 2048
+    launches_per_step = (5 - (1 if fused_combine else 0) + shared
+                         + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (4 if w.L else 0))
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

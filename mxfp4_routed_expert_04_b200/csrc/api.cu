@@ -538,14 +538,28 @@ moe_status do_shared_up(const Plan& p, const DeviceState& ds, const uint16_t* x,
 
 // Shared expert, second half: the down GEMM over both halves of h (split-K
 // partial sums for the combine).
+// One token on the row GEMV with the shared down rows whole per warp
+// (I_shared <= 2048) and no latent projection: the shared down launch also
+// finishes the combine (same order of operations as k_combine).
+bool combine_in_shared_down(const Plan& p) { return p.rows && p.L == 0 && p.Is <= 2048; }
+
+// comb (combine_in_shared_down): y_perm, slot_row, topk_w of the routed
+// experts and the layer output y
 moe_status do_shared_down(const Plan& p, const DeviceState& ds, const uint16_t* ws_down, void* ws,
-                          cudaStream_t st, int max_ctas = 0) {
+                          cudaStream_t st, int max_ctas = 0, const float* y_perm = nullptr,
+                          const int32_t* slot_row = nullptr, const float* topk_w = nullptr,
+                          float* y = nullptr) {
   if (p.rows) {
     moe::RowsArgs r;
     memset(&r, 0, sizeof(r));
     r.w[0] = ws_down; r.rows[0] = p.H; r.out[0] = at<float>(ws, p.off_sd);
     r.x = at<float>(ws, p.off_hsb); r.K = p.Is; r.status = at<int32_t>(ws, p.off_status);
-    return launch_rows(ds, r, false, true, max_ctas ? max_ctas : ds.num_sms, st, "shared down gemv");
+    if (y && combine_in_shared_down(p)) {
+      r.y = y; r.y_perm = y_perm; r.slot_row = slot_row; r.topk_w = topk_w;
+      r.gate_logit = at<float>(ws, p.off_gl); r.k = p.k;
+    }
+    return launch_rows(ds, r, false, true, max_ctas ? max_ctas : ds.num_sms, st,
+                       r.y ? "shared down gemv + combine" : "shared down gemv");
   }
   uint16_t* h_hi = at<uint16_t>(ws, p.off_hsb);
   uint16_t* h_lo = h_hi + (size_t)p.T * p.Is;
@@ -853,6 +867,8 @@ moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t*
   DeviceState* ds;
   if ((s = device_state(&ds)) != MOE_OK) return s;
   if ((s = do_shared_up(p, *ds, x, w_sgate, ws_gate, ws_up, ws, st)) != MOE_OK) return s;
+  if (combine_in_shared_down(p))
+    return do_shared_down(p, *ds, ws_down, ws, st, 0, y_perm, slot_row, topk_w, y);
   if ((s = do_shared_down(p, *ds, ws_down, ws, st)) != MOE_OK) return s;
   return do_final(p, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
 }
@@ -925,6 +941,8 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if ((s = do_expert_ffn(p, *ds, a->x_op, a->offsets, a->expert_list, a->row_token, a->wg_q,
                          a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
     return s;
+  if (combine_in_shared_down(p))
+    return do_shared_down(p, *ds, a->ws_down, ws, st, 0, a->y_perm, a->slot_row, a->topk_w, a->y);
   if ((s = do_shared_down(p, *ds, a->ws_down, ws, st)) != MOE_OK) return s;
   return do_final(p, a->y_perm, a->slot_row, a->topk_w, a->w_lat_up, a->y, ws, st);
 }

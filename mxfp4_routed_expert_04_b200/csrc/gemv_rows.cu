@@ -18,7 +18,10 @@
 //   sums in fp32, a 5-step shuffle reduction per warp; the parts of a row are
 //   added in order through shared memory one stage later (after every warp
 //   has released the stage), so no warp waits inside a stage;
-// * plain writes out[s][row]; SwiGLU writes h[i] = silu(g_i) * u_i (fp32).
+// * plain writes out[s][row]; SwiGLU writes h[i] = silu(g_i) * u_i (fp32);
+//   for the shared down projection of one token the plain mode can instead
+//   finish the layer's combine for its rows (k <= 32 routed slots gathered
+//   by lanes, summed by every lane in slot order).
 // Every wait is bounded as in the other streaming kernels.
 #include "common.cuh"
 #include "kernels.h"
@@ -201,7 +204,21 @@ __global__ void __launch_bounds__(32 * (kRowsConsumers + 1), 1) k_rows_bf16(Rows
           }
         }
         const float sum = warp_sum_rows(a0 + a1);
-        if (lane == 0) {
+        if (direct && a.y) {
+          // the layer's combine for this output row, in the combine's own
+          // order: routed slots j = 0.. (fma), then the gated shared term
+          const int row = r + rs;
+          float v = 0.0f, wj = 0.0f;
+          if (lane < a.k) {
+            v = __ldg(a.y_perm + (size_t)__ldg(a.slot_row + lane) * a.rows[0] + row);
+            wj = __ldg(a.topk_w + lane);
+          }
+          float acc = 0.0f;
+          for (int j = 0; j < a.k; ++j)
+            acc = fmaf(__shfl_sync(0xFFFFFFFFu, wj, j), __shfl_sync(0xFFFFFFFFu, v, j), acc);
+          acc = fmaf(sigmoid_f32(__ldg(a.gate_logit)), sum, acc);
+          if (lane == 0) a.y[row] = acc;
+        } else if (lane == 0) {
           if (direct) a.out[seg][r + rs] = sum;
           else s_part[k % D][w] = sum;
         }

@@ -107,6 +107,15 @@ struct RowsArgs {
   const void* x;             // [K] bf16, or fp32 (k_rows_bf16<*, true>)
   int32_t* status;
   int K, nst;
+  // optional combine of one token (plain mode, K <= 2048): instead of
+  // out[0][row], y[row] = sum_j topk_w[j] * y_perm[slot_row[j], row]
+  //                      + sigmoid(gate_logit[0]) * (Wx)[row]
+  float* y;                  // [rows[0]] or NULL
+  const float* y_perm;       // [R, rows[0]]
+  const int32_t* slot_row;   // [k]
+  const float* topk_w;       // [k]
+  const float* gate_logit;   // [1]
+  int k;
 };
 template <bool kSwiGLU, bool kXF32> __global__ void k_rows_bf16(RowsArgs a);
 // K a power of two in 1024..8192: warps per row K/2048 (at least 1), a stage
