@@ -161,6 +161,11 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
       const uint8_t* ss = st + kStageWBytes;
       const int kb = slab * 256;
       const int nbp = min(8, (a.W - kb) >> 5) >> 1;
+      // the slab's activations of token group 0, all loads in flight at once
+      uint4 xpre[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        xpre[b] = (b < 2 * nbp) ? ldg16(xrow[0] + kb + 32 * b) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int bp = 0; bp < 4; ++bp) {
         if (bp < nbp) {
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(32) k_gateup_mxfp4(GateUpArgs a) {
 #pragma unroll
             for (int gi = 0; gi < 4; ++gi) {
               if (gi < ng) {
-                const uint4 xv = ldg16(xrow[gi] + kb + 32 * b);
+                const uint4 xv = gi == 0 ? xpre[b] : ldg16(xrow[gi] + kb + 32 * b);
                 float cg[4] = {0.f, 0.f, 0.f, 0.f}, cu[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_f16(cg, ag0, xv.x, xv.y);
                 mma_f16(cg, ag1, xv.z, xv.w);
@@ -314,6 +319,22 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
       const uint8_t* ss = st + kStageWBytes;
       const int kb = slab * 256;
       const int nbp = min(8, (a.I - kb) >> 5) >> 1;
+      // the slab's h of token group 0 and its group scales, all loads in flight at once
+      uint4 hpre[8];
+      float hspre[8][2][2];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const bool in = b < 2 * nbp;
+        hpre[b] = in ? ldg16(hrow[0] + kb + 32 * b) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = 2 * t + cc;
+          const bool ok = in && col < n;
+          const float* hsr = a.hscale + (size_t)(r0 + c0 + col) * (a.I >> 4) + 2 * ((kb >> 5) + b);
+          hspre[b][0][cc] = ok ? __ldg(hsr) : 0.0f;
+          hspre[b][1][cc] = ok ? __ldg(hsr + 1) : 0.0f;
+        }
+      }
 #pragma unroll
       for (int bp = 0; bp < 4; ++bp) {
         if (bp < nbp) {
@@ -335,15 +356,22 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
 #pragma unroll
             for (int gi = 0; gi < 4; ++gi) {
               if (gi < ng) {
-                const uint4 hv = ldg16(hrow[gi] + kb + 32 * b);
+                uint4 hv;
                 float hs0[2], hs1[2];
+                if (gi == 0) {
+                  hv = hpre[b];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                  const int col = gi * 8 + 2 * t + c;
-                  const bool ok = col < n;
-                  const float* hsr = a.hscale + (size_t)(r0 + c0 + col) * (a.I >> 4) + hb16;
-                  hs0[c] = ok ? __ldg(hsr) : 0.0f;
-                  hs1[c] = ok ? __ldg(hsr + 1) : 0.0f;
+                  for (int c = 0; c < 2; ++c) { hs0[c] = hspre[b][0][c]; hs1[c] = hspre[b][1][c]; }
+                } else {
+                  hv = ldg16(hrow[gi] + kb + 32 * b);
+#pragma unroll
+                  for (int c = 0; c < 2; ++c) {
+                    const int col = gi * 8 + 2 * t + c;
+                    const bool ok = col < n;
+                    const float* hsr = a.hscale + (size_t)(r0 + c0 + col) * (a.I >> 4) + hb16;
+                    hs0[c] = ok ? __ldg(hsr) : 0.0f;
+                    hs1[c] = ok ? __ldg(hsr + 1) : 0.0f;
+                  }
                 }
                 float c00[4] = {0.f, 0.f, 0.f, 0.f}, c01[4] = {0.f, 0.f, 0.f, 0.f};
                 float c10[4] = {0.f, 0.f, 0.f, 0.f}, c11[4] = {0.f, 0.f, 0.f, 0.f};
