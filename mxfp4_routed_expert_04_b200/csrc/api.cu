@@ -244,6 +244,9 @@ moe_status device_state(DeviceState** out) {
       e = cudaFuncSetAttribute(moe::k_bf16_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                moe::kBf16SmemBudget + 1024 + 256);
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_mma_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)moe::mma_gateup_smem_bytes());
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::k_rows_bf16<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kRowsSmemBudget);
     if (e == cudaSuccess)
@@ -397,6 +400,22 @@ moe_status tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype,
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
+  return MOE_OK;
+}
+
+// bytes [rows, row_bytes] read in unswizzled boxes of box_bytes x box_rows
+moe_status byte_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
+                    uint32_t box_rows, const char* what) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
   return MOE_OK;
@@ -655,7 +674,23 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   moe_status s = MOE_OK;
   if (fma && (s = launch_fma<true>(ds, f, st)) != MOE_OK) return s;
   const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
-  if (mma) {
+  if (mma && p.W % 512 == 0) {
+    // CTA-wide TMA ring (W a multiple of 512: whole 512-element slices, and
+    // scale rows a multiple of 16 bytes)
+    moe::MmaGateUpArgs m;
+    memset(&m, 0, sizeof(m));
+    const uint64_t rows = (uint64_t)p.E * p.I;
+    if ((s = code_map(&m.map_gq, wg_q, rows, p.W / 2, 64, "gate weights")) != MOE_OK ||
+        (s = code_map(&m.map_uq, wu_q, rows, p.W / 2, 64, "up weights")) != MOE_OK ||
+        (s = byte_map(&m.map_gs, wg_s, rows, p.W / 32, 16, 64, "gate scales")) != MOE_OK ||
+        (s = byte_map(&m.map_us, wu_s, rows, p.W / 32, 16, 64, "up scales")) != MOE_OK)
+      return s;
+    m.g = g;
+    m.status = at<int32_t>(ws, p.off_status);
+    launch_pdl(moe::k_mma_gateup, dim3(ds.num_sms), dim3(32 * (moe::kMmaConsumers + 1)),
+               moe::mma_gateup_smem_bytes(), st, m);
+    if ((s = launched("expert gate/up (tensor cores, multi-token)")) != MOE_OK) return s;
+  } else if (mma) {
     launch_pdl(moe::k_gateup_mxfp4, dim3(grid_g), dim3(32), smem, st, g);
     if ((s = launched("expert gate/up")) != MOE_OK) return s;
   }

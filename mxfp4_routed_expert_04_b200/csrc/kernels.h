@@ -25,6 +25,21 @@ struct GateUpArgs {
   int min_tokens;            // experts with fewer tokens are left to the CUDA-core path
 };
 
+// Gate/up of the experts with 2+ tokens through a CTA-wide TMA ring (W a
+// multiple of 512): codes by 2-D tensor maps over [E*I, W/2] bytes (boxes of
+// 128 bytes x 64 rows, 128-byte swizzle), scales over [E*I, W/32] bytes
+// (boxes of 16 bytes x 64 rows), token rows by bulk copies; output as in
+// k_gateup_mxfp4 (h16 + per-16-row-group scales).
+constexpr int kMmaConsumers = 8;     // consumer warps (4 row tiles x 2 K halves) plus one producer warp
+constexpr int kMmaStages = 3;
+struct MmaGateUpArgs {
+  CUtensorMap map_gq, map_uq, map_gs, map_us;
+  GateUpArgs g;
+  int32_t* status;
+};
+__global__ void k_mma_gateup(const __grid_constant__ MmaGateUpArgs a);
+size_t mma_gateup_smem_bytes();
+
 struct DownArgs {
   const __half* h16;
   const float* hscale;
