@@ -247,6 +247,9 @@ moe_status device_state(DeviceState** out) {
       e = cudaFuncSetAttribute(moe::k_mma_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)moe::mma_gateup_smem_bytes());
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::k_mma_down, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)moe::mma_down_smem_bytes());
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::k_rows_bf16<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kRowsSmemBudget);
     if (e == cudaSuccess)
@@ -701,6 +704,20 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.min_tokens = g.min_tokens;
   if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
   if (!mma) return MOE_OK;
+  if (p.I % 512 == 0) {
+    moe::MmaDownArgs m;
+    memset(&m, 0, sizeof(m));
+    const uint64_t rows = (uint64_t)p.E * p.W;
+    if ((s = code_map(&m.map_dq, wd_q, rows, p.I / 2, 128, "down weights")) != MOE_OK ||
+        (s = byte_map(&m.map_ds, wd_s, rows, p.I / 32, 16, 128, "down scales")) != MOE_OK)
+      return s;
+    m.h16 = d.h16; m.hscale = d.hscale; m.offsets = offsets; m.expert_list = expert_list;
+    m.y_perm = y_perm; m.status = at<int32_t>(ws, p.off_status);
+    m.W = p.W; m.I = p.I; m.E = p.E; m.R = p.R; m.min_tokens = g.min_tokens;
+    launch_pdl(moe::k_mma_down, dim3(ds.num_sms), dim3(32 * (moe::kMmaConsumers + 1)),
+               moe::mma_down_smem_bytes(), st, m);
+    return launched("expert down (tensor cores, multi-token)");
+  }
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   launch_pdl(moe::k_down_mxfp4, dim3(grid_d), dim3(32), smem, st, d);
   return launched("expert down");

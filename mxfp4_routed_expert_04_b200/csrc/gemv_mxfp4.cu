@@ -417,7 +417,8 @@ __global__ void __launch_bounds__(32) k_down_mxfp4(DownArgs a) {
 // gate/up + SwiGLU of the experts with 2+ tokens, CTA-wide TMA ring
 // block = 32 * (kMmaConsumers + 1), one CTA per SM, dynamic smem
 // mma_gateup_smem_bytes(); work item = (multi-token expert, 64-row group of
-// I); a stage holds one 512-element K slice: gate and up codes (two 128-byte
+// I), numbered group-major so that every CTA's contiguous share mixes
+// experts with many and few tokens (the MMA work grows with them); a stage holds one 512-element K slice: gate and up codes (two 128-byte
 // boxes x 64 rows each, 128-byte swizzle, the layout ldmatrix reads), their
 // scales (16 bytes x 64 rows), and the slice of every token row (f16, rows
 // 1040 bytes apart so the B-fragment loads spread over the banks). Consumer
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
       for (int s = 0; s < kMmaStages; ++s) { last_ph[s] = 0; filled[s] = false; }
       bool ok = true;
       for (long it = lo; it < hi && ok; ++it) {
-        const int e = s_list[it / groups], rg = (int)(it % groups);
+        const int e = s_list[it % n_multi], rg = (int)(it / n_multi);   // group-major: hot and cold experts mix
         const int r0 = __ldg(a.offsets + e), n_all = __ldg(a.offsets + e + 1) - r0;
         const int wrow = e * I + rg * kMgRows;
         for (int c0 = 0; c0 < n_all && ok; c0 += kMgTok) {
@@ -547,7 +548,7 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
     uint32_t ph = 0;
     bool ok = true;
     for (long it = lo; it < hi && ok; ++it) {
-      const int e = s_list[it / groups], rg = (int)(it % groups);
+      const int e = s_list[it % n_multi], rg = (int)(it / n_multi);   // group-major: hot and cold experts mix
       const int r0 = __ldg(a.offsets + e), n_all = __ldg(a.offsets + e + 1) - r0;
       const int q = rg * 4 + tt;                        // the 16-row tile (h group) index within I
       const int i0 = 32 * (q >> 1) + 4 * (q & 1);
@@ -677,6 +678,203 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
 }
 
 size_t mma_gateup_smem_bytes() { return 1024 + (size_t)kMmaStages * kMgStage + kMgRed; }
+
+// ---------------------------------------------------------------------------
+// down projection of the experts with 2+ tokens, CTA-wide TMA ring
+// block = 32 * (kMmaConsumers + 1), one CTA per SM; work item = (multi-token
+// expert, 128-row group of W), numbered group-major as in k_mma_gateup; a stage holds one 512-element K slice: the
+// down codes (two 128-byte boxes x 128 rows, 128-byte swizzle), their scales
+// (16 bytes x 128 rows), every token's h slice (f16, rows 1040 bytes apart)
+// and its 32 group scales; warp w takes the 16-row tile w over the whole
+// slice (the items are short: K = I is a few slices).
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kMdRows = 128;
+constexpr int kMdBox = kMdRows * 128;
+constexpr int kMdCodes = 2 * kMdBox;
+constexpr int kMdScales = kMdRows * 16;
+constexpr int kMdHsOff = kMdCodes + kMdScales;                   // h rows
+constexpr int kMdScOff = kMdHsOff + kMgTok * kMgXStride;         // h group scales, 128 bytes per token
+constexpr int kMdStage = (kMdScOff + kMgTok * 128 + 1023) / 1024 * 1024;
+}  // namespace
+
+__global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_down(const __grid_constant__ MmaDownArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ int16_t s_list[1024];
+  __shared__ int s_wsum[kMmaConsumers + 1];
+  __shared__ uint64_t s_bars[2 * kMmaStages];
+  __shared__ int s_abort;
+  constexpr int kWarps = kMmaConsumers + 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int W = a.W, I = a.I;
+
+  const int n_act = __ldg(a.expert_list);
+  int n_multi = 0;
+  for (int base = 0; base < n_act; base += 32 * kWarps) {
+    const int i = base + threadIdx.x;
+    int e = -1;
+    if (i < n_act) {
+      e = __ldg(a.expert_list + 1 + i);
+      if (__ldg(a.offsets + e + 1) - __ldg(a.offsets + e) < a.min_tokens) e = -1;
+    }
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, e >= 0);
+    if (lane == 0) s_wsum[warp] = __popc(m);
+    __syncthreads();
+    int before = n_multi;
+    for (int w = 0; w < warp; ++w) before += s_wsum[w];
+    if (e >= 0) s_list[before + __popc(m & ((1u << lane) - 1u))] = (int16_t)e;
+    for (int w = 0; w < kWarps; ++w) n_multi += s_wsum[w];
+    __syncthreads();
+  }
+  const int groups = W / kMdRows;
+  const long total = (long)n_multi * groups;
+  const long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+  if (lo >= hi) return;
+  uint64_t* full = s_bars;
+  uint64_t* empty = s_bars + kMmaStages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMmaStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kMmaConsumers);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort = &s_abort;
+  const int nslice = I / 512;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int slot = 0;
+      uint32_t ph = 0;
+      uint32_t last_ph[kMmaStages];
+      bool filled[kMmaStages];
+      for (int s = 0; s < kMmaStages; ++s) { last_ph[s] = 0; filled[s] = false; }
+      bool ok = true;
+      for (long it = lo; it < hi && ok; ++it) {
+        const int e = s_list[it % n_multi], rg = (int)(it / n_multi);   // group-major: hot and cold experts mix
+        const int r0 = __ldg(a.offsets + e), n_all = __ldg(a.offsets + e + 1) - r0;
+        const int wrow = e * W + rg * kMdRows;
+        for (int c0 = 0; c0 < n_all && ok; c0 += kMgTok) {
+          const int nt = min(kMgTok, n_all - c0);
+          for (int s = 0; s < nslice; ++s) {
+            if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) { ok = false; break; }
+            uint8_t* st = smem + (size_t)slot * kMdStage;
+            fence_proxy_async_smem();
+            mbar_expect_tx(&full[slot], kMdCodes + kMdScales + nt * (1024 + 128));
+            tc::tma_load_2d(st, &a.map_dq, s * 256, wrow, &full[slot]);
+            tc::tma_load_2d(st + kMdBox, &a.map_dq, s * 256 + 128, wrow, &full[slot]);
+            tc::tma_load_2d(st + kMdCodes, &a.map_ds, s * 16, wrow, &full[slot]);
+            for (int c = 0; c < nt; ++c) {
+              const size_t r = (size_t)(r0 + c0 + c);
+              bulk_g2s(st + kMdHsOff + c * kMgXStride, a.h16 + r * I + s * 512, 1024u, &full[slot]);
+              bulk_g2s(st + kMdScOff + c * 128, a.hscale + r * (I >> 4) + s * 32, 128u, &full[slot]);
+            }
+            last_ph[slot] = ph;
+            filled[slot] = true;
+            if (++slot == kMmaStages) { slot = 0; ph ^= 1u; }
+          }
+        }
+      }
+      if (*abort) {
+        for (int s = 0; s < kMmaStages; ++s)
+          if (filled[s]) mbar_wait(&full[s], last_ph[s]);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const int tt = warp - 1;                            // 16-row tile of the item
+    const int g = lane >> 2, t4 = lane & 3;
+    const int lq = lane >> 3, lr = lane & 7;
+    const int ldrow = 16 * tt + (lq & 1) * 8 + lr;
+    const int row_g = 16 * tt + g, row_g8 = row_g + 8;
+    int slot = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (long it = lo; it < hi && ok; ++it) {
+      const int e = s_list[it % n_multi], rg = (int)(it / n_multi);   // group-major: hot and cold experts mix
+      const int r0 = __ldg(a.offsets + e), n_all = __ldg(a.offsets + e + 1) - r0;
+      const int n0 = rg * kMdRows + 16 * tt;             // first output column (row of Wd) of the tile
+      for (int c0 = 0; c0 < n_all; c0 += kMgTok) {
+        const int n = min(kMgTok, n_all - c0);
+        const int ng = (n + 7) >> 3;
+        float acc[4][4];
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[gi][j] = 0.0f;
+        for (int s = 0; s < nslice; ++s) {
+          if (!tc::wait_or_abort(&full[slot], ph, abort)) { ok = false; break; }
+          const uint8_t* st = smem + (size_t)slot * kMdStage;
+          const uint32_t cod = smem_u32(st);
+          const uint8_t* wsc = st + kMdCodes;
+          const uint32_t hs0a = smem_u32(st + kMdHsOff);
+          const float* hsc = reinterpret_cast<const float*>(st + kMdScOff);
+#pragma unroll 2
+          for (int bp = 0; bp < 8; ++bp) {
+            uint32_t R[4];
+            const int ch = 2 * (bp & 3) + (lq >> 1);
+            ldmatrix_x4(R, cod + (bp >> 2) * kMdBox + ldrow * 128 + ((ch ^ (ldrow & 7)) << 4));
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+              const int b = 2 * bp + hb;
+              uint32_t a0[4], a1[4];
+              decode_block(R[2 * hb], R[2 * hb + 1], a0, a1);
+              const float ws0 = e8m0_to_f32(wsc[row_g * 16 + b]);
+              const float ws8 = e8m0_to_f32(wsc[row_g8 * 16 + b]);
+#pragma unroll
+              for (int gi = 0; gi < 4; ++gi) {
+                if (gi < ng) {
+                  const int tok = min(gi * 8 + g, n - 1);
+                  const uint4 hv = lds16(hs0a + tok * kMgXStride + (32 * b + 8 * t4) * 2);
+                  float hq0[2], hq1[2];
+#pragma unroll
+                  for (int cc = 0; cc < 2; ++cc) {
+                    const int col = min(gi * 8 + 2 * t4 + cc, n - 1);
+                    hq0[cc] = hsc[col * 32 + 2 * b];
+                    hq1[cc] = hsc[col * 32 + 2 * b + 1];
+                  }
+                  float c00[4] = {0.f, 0.f, 0.f, 0.f}, c01[4] = {0.f, 0.f, 0.f, 0.f};
+                  mma_f16(c00, a0, hv.x, hv.y);
+                  mma_f16(c01, a1, hv.z, hv.w);
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float v = fmaf(c01[j], hq1[j & 1], c00[j] * hq0[j & 1]);
+                    acc[gi][j] = fmaf(v, (j >> 1) ? ws8 : ws0, acc[gi][j]);
+                  }
+                }
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&empty[slot]);
+          if (++slot == kMmaStages) { slot = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          if (gi < ng) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int col = gi * 8 + 2 * t4 + (j & 1);
+              if (col < n) a.y_perm[(size_t)(r0 + c0 + col) * W + n0 + g + 8 * (j >> 1)] = acc[gi][j];
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) atomicOr(a.status, kStatusWaitTimeout);
+}
+
+size_t mma_down_smem_bytes() { return 1024 + (size_t)kMmaStages * kMdStage; }
 
 size_t gemv_mxfp4_smem_bytes() { return (size_t)kStages * kStageBytes; }
 

@@ -39,6 +39,23 @@ struct MmaGateUpArgs {
 };
 __global__ void k_mma_gateup(const __grid_constant__ MmaGateUpArgs a);
 size_t mma_gateup_smem_bytes();
+// Down projection of the experts with 2+ tokens, the same ring (I a multiple
+// of 512): down codes [E*W, I/2] (boxes of 128 bytes x 128 rows) and scales
+// [E*W, I/32] (16 bytes x 128 rows) by tensor maps, the tokens' h rows and h
+// group scales by bulk copies.
+struct MmaDownArgs {
+  CUtensorMap map_dq, map_ds;
+  const __half* h16;         // [R, I]
+  const float* hscale;       // [R, I/16]
+  const int32_t* offsets;
+  const int32_t* expert_list;
+  float* y_perm;             // [R, W]
+  int32_t* status;
+  int W, I, E, R;
+  int min_tokens;
+};
+__global__ void k_mma_down(const __grid_constant__ MmaDownArgs a);
+size_t mma_down_smem_bytes();
 
 struct DownArgs {
   const __half* h16;
