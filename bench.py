@@ -254,7 +254,9 @@ def run_ours(args, w):
     # SwiGLU finaliser, down), or 2 for one token on the row GEMV and for 128+
     # tokens (SwiGLU in the GEMM epilogue); routed experts 4 (bf16: two GEMV
     # pairs; 2 for one token, whose experts all have a single token) or 3
-    # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 4
+    # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 3 (the down
+    # projection rides with the router rows; its bf16 rounding, the routed sum
+    # at width L, the up-projection GEMM)
     rows_k = (1024, 2048, 4096, 8192)
     rows_path = w.T == 1 and w.H in rows_k and w.I_shared in rows_k
     # (many tokens: the sigmoid-gate row rides with the router rows as well)
@@ -263,7 +265,7 @@ def run_ours(args, w):
     # the shared down launch)
     fused_combine = rows_path and not w.L and w.I_shared <= 2048
     launches_per_step = (5 - (1 if fused_combine else 0) + shared
-                         + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (4 if w.L else 0))
+                         + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (3 if w.L else 0))
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -357,7 +359,13 @@ def run_ours(args, w):
                      "roofline_ms": max(t_mem, t_tc) * 1e3,
                      "frac_of_roofline_time": max(t_mem, t_tc) / (ffn_ms * 1e-3)})
     else:
-        kernel = "moe_expert_ffn (k_fma_gemv + k_gateup_mxfp4 + k_down_mxfp4)"
+        # single-token experts on the CUDA-core GEMV pair; experts with 2+
+        # tokens on the TMA-fed mma.sync pair (whole 512-element slices) or,
+        # for other widths, on the per-warp GEMV pair
+        multi = ("k_mma_gateup" if w.W % 512 == 0 else "k_gateup_mxfp4",
+                 "k_mma_down" if w.I % 512 == 0 else "k_down_mxfp4")
+        kernel = ("moe_expert_ffn (k_fma_gemv)" if w.T == 1
+                  else "moe_expert_ffn (k_fma_gemv + %s + %s)" % multi)
         roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peak, "unit": "GB/s",
                 "frac": hbm_gbs / peak, "peak_kind": peak_kind}
     roof = dict({"kernel": kernel}, **roof)

@@ -31,22 +31,6 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Number of K splits of a dense GEMV: enough warps to cover the GPU (about 4
-// per SM), each split a whole number of 32-element steps and at least 8 of
-// them, at most 16 splits.
-int dense_splits(int N, int T, int K) {
-  const long warps = (long)((N + 15) / 16) * ((T + 31) / 32);
-  const int ksteps = K / 32;
-  int S = 1;
-  for (int c = 1; c <= ksteps && c <= 16; ++c) {
-    if (ksteps % c) continue;
-    if (ksteps / c < 8) break;
-    S = c;
-    if (warps * c >= (long)kNumSMs * 4) break;
-  }
-  return S;
-}
-
 // Token count from which the shared expert's gate/up GEMM applies SwiGLU in its
 // epilogue (below it the gate, up and sigmoid-gate rows write split-K
 // partial sums and a finaliser applies SwiGLU).
@@ -127,19 +111,26 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
     p.S_sd = 1;
   } else {
     const long ntt = (p.T + p.Nt - 1) / p.Nt;
-    p.S_router = tc_splits((long)((p.E + 255) / 256 + 1) * ntt, p.H, (size_t)p.T * (p.E + 1) * 4);
+    // the router rows, the sigmoid-gate row and the latent down-projection
+    // rows share one pass over x (the same splits when launched alone)
+    p.S_router = tc_splits((long)((p.E + 255) / 256 + 1 + (p.L + 255) / 256) * ntt, p.H,
+                           (size_t)p.T * (p.E + 1 + p.L) * 4);
     // SwiGLU epilogue: one split, the sigmoid-gate row on the GEMV
     p.S_sgu = p.swiglu_tc ? 1
                           : tc_splits((long)(2 * ((p.Is + 255) / 256) + 1) * ntt, p.H,
                                       (size_t)p.T * (2 * p.Is + 1) * 4);
     p.S_sd = tc_splits((long)((p.H + 255) / 256) * ntt, p.Is, (size_t)p.T * p.H * 4);
   }
-  p.S_ld = p.L ? dense_splits(p.L, p.T, p.H) : 0;
-  p.S_lu = p.L ? dense_splits(p.H, p.T, p.L) : 0;
+  p.S_ld = p.L ? p.S_router : 0;
+  p.S_lu = p.L ? tc_splits((long)((p.H + 255) / 256) * ((p.T + p.Nt - 1) / p.Nt), p.L,
+                           (size_t)p.T * p.H * 4)
+               : 0;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 256); return r; };
   p.off_status = take(256);
-  p.off_router = take((size_t)p.S_router * p.T * (p.E + 1) * 4);   // + the sigmoid-gate column
+  // + the sigmoid-gate column (+ the latent down-projection columns on the
+  // tcgen05 GEMM)
+  p.off_router = take((size_t)p.S_router * p.T * (p.E + 1 + (p.rows ? 0 : p.L)) * 4);
   p.off_h16 = take((size_t)p.R * p.I * 2);
   p.off_hscale = take((size_t)p.R * (p.I / 16) * 4);
   p.off_h32 = take((size_t)p.R * p.I * 4);
@@ -150,7 +141,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.off_gl = take((size_t)p.T * 4);
   p.off_sd = take((size_t)p.S_sd * p.T * p.H * 4);
   p.off_ld = take(p.L ? (size_t)p.S_ld * p.T * p.L * 4 : 0);
-  p.off_ylat = take(p.L ? (size_t)p.T * p.L * 4 : 0);
+  p.off_ylat = take(p.L ? (size_t)p.T * p.L * 4 : 0);   // bf16 pair [2][T, L]
   p.off_lu = take(p.L ? (size_t)p.S_lu * p.T * p.H * 4 : 0);
   // MXFP4 activations: tiles of at most kTileRows rows of one expert; the sum
   // over experts of ceil(rows / kTileRows) is below R / kTileRows + (experts) + 1.
@@ -220,7 +211,7 @@ struct DeviceState {
   int num_sms = 0;
   int gemv_ctas_per_sm = 0;
   cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_lat = nullptr, ev_shared = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_shared = nullptr;
 };
 std::mutex g_mu;
 DeviceState g_dev[64];
@@ -265,7 +256,6 @@ moe_status device_state(DeviceState** out) {
     if (e == cudaSuccess && s.gemv_ctas_per_sm < 1) s.gemv_ctas_per_sm = 1;
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s.side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_lat, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.ev_shared, cudaEventDisableTiming);
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "device setup: %s", cudaGetErrorString(e));
     s.ready = true;
@@ -277,21 +267,6 @@ moe_status device_state(DeviceState** out) {
 // ---------------------------------------------------------------------------
 // launchers (arguments already validated)
 // ---------------------------------------------------------------------------
-moe_status launch_dense(const uint16_t* w0, int r0, const uint16_t* w1, int r1, const uint16_t* w2,
-                        int r2, const void* x, bool x_f32, float* part, int T, int K, int S,
-                        cudaStream_t st, const char* what, bool pdl = true) {
-  moe::DenseArgs a;
-  a.w[0] = w0; a.w[1] = w1 ? w1 : w0; a.w[2] = w2 ? w2 : w0;
-  a.rows[0] = r0; a.rows[1] = r1; a.rows[2] = r2;
-  a.N = r0 + r1 + r2;
-  a.x = x; a.x_f32 = x_f32 ? 1 : 0;
-  a.part = part;
-  a.T = T; a.K = K; a.S = S; a.kper = K / S;
-  const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (T + 31) / 32);
-  if (pdl) launch_pdl(moe::k_dense_gemv, grid, dim3(32 * moe::kDenseWarps), 0, st, a);
-  else moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, st>>>(a);
-  return launched(what);
-}
 
 // single-token row GEMV: one CTA per SM (at most max_ctas), ring depth from
 // the shared-memory budget
@@ -450,40 +425,56 @@ moe_status launch_bf16_gemm(const DeviceState& ds, moe::Bf16GemmArgs& g, cudaStr
   return launched(what);
 }
 
-// The router logits (and, when w_sgate is given, the shared expert's sigmoid
-// gate logit from the same pass over x), then top-k.
+// x_lat[t, n] = bf16(sum_s part[s, t, n]) from the latent down-projection's
+// partial sums (rows of ld floats)
+moe_status round_latent(const Plan& p, const float* part, int ld, uint16_t* x_lat, cudaStream_t st) {
+  launch_pdl(moe::k_round_bf16, dim3((p.L + moe::kFinThreads - 1) / moe::kFinThreads, p.T),
+             dim3(moe::kFinThreads), 0, st, part, p.S_ld, p.T, p.L, ld, x_lat);
+  return launched("latent round");
+}
+
+// The router logits, then top-k. The same pass over x can carry the shared
+// expert's sigmoid-gate row (w_sgate) and the latent down-projection (w_ld,
+// rounded to bf16 into x_lat after the top-k).
 moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
                     int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st,
-                    const uint16_t* w_sgate = nullptr) {
+                    const uint16_t* w_sgate = nullptr, const uint16_t* w_ld = nullptr,
+                    uint16_t* x_lat = nullptr) {
   float* part = at<float>(ws, p.off_router);
   moe_status s;
   if (p.rows) {
     moe::RowsArgs r;
     memset(&r, 0, sizeof(r));
     r.w[0] = wr; r.rows[0] = p.E; r.out[0] = part;
-    if (w_sgate) { r.w[1] = w_sgate; r.rows[1] = 1; r.out[1] = at<float>(ws, p.off_gl); }
+    int seg = 1;
+    if (w_sgate) { r.w[seg] = w_sgate; r.rows[seg] = 1; r.out[seg] = at<float>(ws, p.off_gl); ++seg; }
+    if (w_ld) { r.w[seg] = w_ld; r.rows[seg] = p.L; r.out[seg] = at<float>(ws, p.off_ld); }
     r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
     if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
     launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
                p.E, p.k, idx, w, logits, (float*)nullptr);
-    return launched("top-k");
+    if ((s = launched("top-k")) != MOE_OK) return s;
+    return w_ld ? round_latent(p, at<float>(ws, p.off_ld), p.L, x_lat, st) : MOE_OK;
   }
-  // many tokens: the router rows (and the sigmoid-gate row as a second
-  // segment, column E of the partial sums) on the tcgen05 GEMM
+  // many tokens: the router rows, then the sigmoid-gate row (column E of the
+  // partial sums) and the latent rows as further segments of the tcgen05 GEMM
   moe::Bf16GemmArgs g;
   memset(&g, 0, sizeof(g));
   if ((s = bf16_map(&g.map_a[0], wr, p.E, p.H, "router weights")) != MOE_OK ||
       (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK ||
-      (w_sgate && (s = bf16_map(&g.map_a[1], w_sgate, 1, p.H, "sigmoid-gate weights")) != MOE_OK))
+      (w_sgate && (s = bf16_map(&g.map_a[1], w_sgate, 1, p.H, "sigmoid-gate weights")) != MOE_OK) ||
+      (w_ld && (s = bf16_map(&g.map_a[2], w_ld, p.L, p.H, "latent down weights")) != MOE_OK))
     return s;
-  const int ld = w_sgate ? p.E + 1 : p.E;
+  const int lat_col = w_sgate ? p.E + 1 : p.E;
+  const int ld = lat_col + (w_ld ? p.L : 0);
   g.out = part; g.status = at<int32_t>(ws, p.off_status);
   g.mode = moe::kBf16Plain; g.K = p.H; g.T = p.T; g.S = p.S_router; g.passes = 1; g.N = p.Nt;
-  g.seg_rows[0] = p.E; g.seg_rows[1] = w_sgate ? 1 : 0; g.ld = ld;
+  g.seg_rows[0] = p.E; g.seg_rows[1] = w_sgate ? 1 : 0; g.seg_rows[2] = w_ld ? p.L : 0; g.ld = ld;
   if ((s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)")) != MOE_OK) return s;
   launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E,
              ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr);
-  return launched("top-k");
+  if ((s = launched("top-k")) != MOE_OK) return s;
+  return w_ld ? round_latent(p, part + lat_col, ld, x_lat, st) : MOE_OK;
 }
 
 // Shared expert on the tcgen05 GEMM, first half: h = silu(Wg x) * (Wu x) as
@@ -723,27 +714,46 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   return launched("expert down");
 }
 
-moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row, const float* topk_w,
-                    const uint16_t* w_lat_up, float* y, void* ws, cudaStream_t st) {
+// The latent up-projection: W_lu [H, L] times the routed sum y_lat given as a
+// bf16 pair (hi, lo), on the tcgen05 GEMM; split-K partials [S_lu, T, H].
+moe_status do_latent_up(const Plan& p, const DeviceState& ds, const uint16_t* w_lat_up, void* ws,
+                        cudaStream_t st) {
+  uint16_t* y_hi = at<uint16_t>(ws, p.off_ylat);
+  uint16_t* y_lo = y_hi + (size_t)p.T * p.L;
+  moe_status s;
+  moe::Bf16GemmArgs u;
+  memset(&u, 0, sizeof(u));
+  if ((s = bf16_map(&u.map_a[0], w_lat_up, p.H, p.L, "latent up weights")) != MOE_OK ||
+      (s = bf16_map(&u.map_b0, y_hi, p.T, p.L, "latent sum (hi)", p.Nt)) != MOE_OK ||
+      (s = bf16_map(&u.map_b1, y_lo, p.T, p.L, "latent sum (lo)", p.Nt)) != MOE_OK)
+    return s;
+  u.out = at<float>(ws, p.off_lu); u.status = at<int32_t>(ws, p.off_status);
+  u.mode = moe::kBf16Plain; u.K = p.L; u.T = p.T; u.S = p.S_lu; u.passes = 2; u.N = p.Nt;
+  u.seg_rows[0] = p.H; u.ld = p.H;
+  return launch_bf16_gemm(ds, u, st, "latent up gemm (tcgen05)");
+}
+
+moe_status do_final(const Plan& p, const DeviceState& ds, const float* y_perm, const int32_t* slot_row,
+                    const float* topk_w, const uint16_t* w_lat_up, float* y, void* ws, cudaStream_t st) {
   moe::CombineArgs c;
+  memset(&c, 0, sizeof(c));
   c.slot_row = slot_row; c.topk_w = topk_w; c.k = p.k;
   c.gate_logit = at<float>(ws, p.off_gl);
   c.T = p.T;
   if (p.L) {
-    // routed weighted sum at width L, then the up-projection, then + shared
-    c.y_perm = y_perm; c.add1 = nullptr; c.S1 = 0; c.add2 = nullptr; c.S2 = 0;
-    c.out = at<float>(ws, p.off_ylat); c.width = p.L;
+    // routed weighted sum at width L (as a bf16 pair), then the
+    // up-projection, then + shared
+    c.y_perm = y_perm;
+    c.out_hi = at<uint16_t>(ws, p.off_ylat); c.out_lo = c.out_hi + (size_t)p.T * p.L;
+    c.width = p.L;
     moe::k_combine<<<dim3((p.L / 4 + moe::kCombineThreads - 1) / moe::kCombineThreads, p.T),
                      moe::kCombineThreads, 0, st>>>(c);
     moe_status s = launched("latent combine");
-    if (s != MOE_OK) return s;
-    s = launch_dense(w_lat_up, p.H, nullptr, 0, nullptr, 0, at<float>(ws, p.off_ylat), true,
-                     at<float>(ws, p.off_lu), p.T, p.L, p.S_lu, st, "latent up gemv");
-    if (s != MOE_OK) return s;
-    c.y_perm = nullptr;
+    if (s != MOE_OK || (s = do_latent_up(p, ds, w_lat_up, ws, st)) != MOE_OK) return s;
+    c.y_perm = nullptr; c.out_hi = c.out_lo = nullptr;
     c.add1 = at<float>(ws, p.off_lu); c.S1 = p.S_lu;
   } else {
-    c.y_perm = y_perm; c.add1 = nullptr; c.S1 = 0;
+    c.y_perm = y_perm;
   }
   c.add2 = at<float>(ws, p.off_sd); c.S2 = p.S_sd;
   c.out = y; c.width = p.H;
@@ -752,16 +762,30 @@ moe_status do_final(const Plan& p, const float* y_perm, const int32_t* slot_row,
   return launched("combine");
 }
 
-moe_status do_latent_down(const Plan& p, const uint16_t* x, const uint16_t* w_ld, uint16_t* x_lat,
-                          void* ws, cudaStream_t st) {
+// The latent down-projection alone: the same GEMM geometry and split order as
+// when it rides along with the router rows, so that both give the same bits.
+moe_status do_latent_down(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* w_ld,
+                          uint16_t* x_lat, void* ws, cudaStream_t st) {
   float* part = at<float>(ws, p.off_ld);
-  moe_status s = launch_dense(w_ld, p.L, nullptr, 0, nullptr, 0, x, false, part, p.T, p.H, p.S_ld, st,
-                              "latent down gemv");
-  if (s != MOE_OK) return s;
-  launch_pdl(moe::k_round_bf16, dim3((p.L + moe::kFinThreads - 1) / moe::kFinThreads, p.T),
-             dim3(moe::kFinThreads), 0, st, (const float*)part, p.S_ld,
-             p.T, p.L, x_lat);
-  return launched("latent round");
+  moe_status s;
+  if (p.rows) {
+    moe::RowsArgs r;
+    memset(&r, 0, sizeof(r));
+    r.w[0] = w_ld; r.rows[0] = p.L; r.out[0] = part;
+    r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
+    if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "latent down gemv")) != MOE_OK) return s;
+  } else {
+    moe::Bf16GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    if ((s = bf16_map(&g.map_a[0], w_ld, p.L, p.H, "latent down weights")) != MOE_OK ||
+        (s = bf16_map(&g.map_b0, x, p.T, p.H, "tokens", p.Nt)) != MOE_OK)
+      return s;
+    g.out = part; g.status = at<int32_t>(ws, p.off_status);
+    g.mode = moe::kBf16Plain; g.K = p.H; g.T = p.T; g.S = p.S_ld; g.passes = 1; g.N = p.Nt;
+    g.seg_rows[0] = p.L; g.ld = p.L;
+    if ((s = launch_bf16_gemm(ds, g, st, "latent down gemm (tcgen05)")) != MOE_OK) return s;
+  }
+  return round_latent(p, part, p.L, x_lat, st);
 }
 
 }  // namespace
@@ -922,7 +946,7 @@ moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t*
   if (combine_in_shared_down(p))
     return do_shared_down(p, *ds, ws_down, ws, st, 0, y_perm, slot_row, topk_w, y);
   if ((s = do_shared_down(p, *ds, ws_down, ws, st)) != MOE_OK) return s;
-  return do_final(p, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
+  return do_final(p, *ds, y_perm, slot_row, topk_w, w_lat_up, y, ws, st);
 }
 
 moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16_t* w_lat_down,
@@ -933,7 +957,9 @@ moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16
   if (!p.L) return fail(MOE_ERR_INVALID_ARG, "moe_latent_down needs L > 0");
   CHECK_PTR(x); CHECK_PTR(w_lat_down); CHECK_PTR(x_lat);
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
-  return do_latent_down(p, x, w_lat_down, x_lat, ws, (cudaStream_t)stream);
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  return do_latent_down(p, *ds, x, w_lat_down, x_lat, ws, (cudaStream_t)stream);
 }
 
 moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, size_t ws_bytes,
@@ -959,20 +985,17 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   cudaError_t e = cudaEventRecord(ds->ev_fork, st);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
   // main stream first: the router's CTAs are queued before the shared expert's
-  // (one token: the sigmoid-gate row rides along with the router rows)
+  // (one token or the SwiGLU-epilogue GEMM: the sigmoid-gate row rides along
+  // with the router rows; the latent down-projection always does)
   const bool sgate_with_router = p.rows || p.swiglu_tc;
   if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st,
-                    sgate_with_router ? a->w_sgate : nullptr)) != MOE_OK)
+                    sgate_with_router ? a->w_sgate : nullptr, p.L ? a->w_lat_down : nullptr,
+                    a->x_lat)) != MOE_OK)
     return s;
-  // side stream: latent projection, then the first half of the shared expert
-  // (it streams its weights while the routing chain runs)
+  // side stream: the first half of the shared expert (it streams its weights
+  // while the routing chain runs)
   if ((e = cudaStreamWaitEvent(ds->side, ds->ev_fork, 0)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
-  if (p.L) {
-    if ((s = do_latent_down(p, a->x, a->w_lat_down, a->x_lat, ws, ds->side)) != MOE_OK) return s;
-    if ((e = cudaEventRecord(ds->ev_lat, ds->side)) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
-  }
   // (the row GEMV leaves a few SMs to the routing chain's small kernels)
   if ((s = do_shared_up(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, ws, ds->side, sgate_with_router,
                         ds->num_sms - kRowsFreeSMs)) != MOE_OK)
@@ -980,8 +1003,6 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   // main stream: dispatch, experts, combine
-  if (p.L && (e = cudaStreamWaitEvent(st, ds->ev_lat, 0)) != cudaSuccess)
-    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
   if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets,
                       a->expert_list, a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) !=
       MOE_OK)
@@ -996,7 +1017,7 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if (combine_in_shared_down(p))
     return do_shared_down(p, *ds, a->ws_down, ws, st, 0, a->y_perm, a->slot_row, a->topk_w, a->y);
   if ((s = do_shared_down(p, *ds, a->ws_down, ws, st)) != MOE_OK) return s;
-  return do_final(p, a->y_perm, a->slot_row, a->topk_w, a->w_lat_up, a->y, ws, st);
+  return do_final(p, *ds, a->y_perm, a->slot_row, a->topk_w, a->w_lat_up, a->y, ws, st);
 }
 
 }  // extern "C"

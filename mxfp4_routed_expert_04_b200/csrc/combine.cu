@@ -63,6 +63,21 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineArgs a) {
     split_sum(a.add2, a.S2, sh);
     fma4(sigmoid_f32(__ldg(a.gate_logit + t)), sh, acc);
   }
+  if (a.out_hi) {
+    // the operand pair of a bf16 tensor-core GEMM: hi + lo carries 16
+    // significant bits of the fp32 sum
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hi[i] = f32_to_bf16_rne(v[i]);
+      lo[i] = f32_to_bf16_rne(v[i] - bf16_to_f32(hi[i]));
+    }
+    const size_t o = (size_t)t * a.width + c;
+    *reinterpret_cast<uint2*>(a.out_hi + o) = make_uint2(hi[0] | hi[1] << 16, hi[2] | hi[3] << 16);
+    *reinterpret_cast<uint2*>(a.out_lo + o) = make_uint2(lo[0] | lo[1] << 16, lo[2] | lo[3] << 16);
+    return;
+  }
   *reinterpret_cast<float4*>(a.out + (size_t)t * a.width + c) = acc;
 }
 
@@ -105,16 +120,18 @@ __global__ void __launch_bounds__(kFinThreads) k_sum_column(const float* __restr
   if (t < T) out[t] = sum_splits(part + (size_t)t * ld + col, S, (size_t)T * ld);
 }
 
-// out[t, n] = bf16_rne( sum_s part[s, t, n] )   (latent down-projection)
+// out[t, n] = bf16_rne( sum_s part[s, t, n] )   (latent down-projection;
+// partial rows of ld floats)
 // grid (ceil(N/kFinThreads), T), block kFinThreads
 __global__ void __launch_bounds__(kFinThreads) k_round_bf16(const float* __restrict__ part, int S,
-                                                          int T, int N, uint16_t* __restrict__ out) {
+                                                          int T, int N, int ld,
+                                                          uint16_t* __restrict__ out) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.y;
   const int n = blockIdx.x * kFinThreads + threadIdx.x;
   if (n >= N) return;
-  const float v = sum_splits(part + (size_t)t * N + n, S, (size_t)T * N);
+  const float v = sum_splits(part + (size_t)t * ld + n, S, (size_t)T * ld);
   out[(size_t)t * N + n] = (uint16_t)f32_to_bf16_rne(v);
 }
 

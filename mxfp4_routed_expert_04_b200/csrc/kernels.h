@@ -228,7 +228,8 @@ __global__ void k_act_to_mxfp4_perm(const uint16_t* x, int W, int k, const int32
 constexpr int kFinThreads = 64;
 __global__ void k_shared_swiglu(const float* part, int S, int T, int Is, uint16_t* h_hi,
                                 uint16_t* h_lo, float* gate_logit);
-__global__ void k_round_bf16(const float* part, int S, int T, int N, uint16_t* out);
+// out[t, n] = bf16(sum_s part[(s * T + t) * ld + n]), n < N
+__global__ void k_round_bf16(const float* part, int S, int T, int N, int ld, uint16_t* out);
 __global__ void k_sum_column(const float* part, int S, int T, int ld, int col, float* out);
 
 struct CombineArgs {
@@ -241,7 +242,9 @@ struct CombineArgs {
   const float* add2;         // [S2, T, width] partials scaled by sigmoid(gate_logit[t]), or NULL
   int S2;
   const float* gate_logit;   // [T]
-  float* out;                // [T, width]
+  float* out;                // [T, width] fp32, or NULL when out_hi is set
+  uint16_t* out_hi;          // [T, width] bf16 pair hi = bf16(y), lo = bf16(y - hi), or NULL
+  uint16_t* out_lo;
   int T, width;
 };
 constexpr int kCombineThreads = 64;

@@ -35,6 +35,13 @@ WIDE = synth.MoeWorkload("wide_tc", T=260, H=640, I=256, E=6, k=2, I_shared=384,
 # the whole-row CUDA-core GEMV (E = 10 router rows: the last stage holds two;
 # the sigmoid-gate row is a segment of its own)
 ROWS_T1 = synth.MoeWorkload("rows_t1", T=1, H=2048, I=256, E=10, k=3, I_shared=1024, seed=80)
+# latent layers: one token on the row GEMV (the latent rows a third segment of
+# the router launch), and T >= 128 on the tcgen05 GEMM (router rows, the
+# sigmoid-gate row and the latent rows as three segments of one pass over x)
+ROWS_LATENT_T1 = synth.MoeWorkload("rows_latent_t1", T=1, H=1024, I=128, E=12, k=3, I_shared=1024,
+                                   L=256, seed=81)
+WIDE_LATENT = synth.MoeWorkload("wide_latent", T=130, H=512, I=128, E=6, k=2, I_shared=256, L=384,
+                                seed=82)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
@@ -42,6 +49,8 @@ CASES = [
     (LATENT_SMALL, None),
     (WIDE, None),
     (ROWS_T1, None),
+    (ROWS_LATENT_T1, None),
+    (WIDE_LATENT, None),
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
