@@ -252,8 +252,8 @@ def run_ours(args, w):
     # kernels enqueued by one moe_layer call: router 2 (logits, top-k), permute 2
     # (dispatch, activation operand), combine 1; shared expert 3 (gate/up,
     # SwiGLU finaliser, down), or 2 for one token on the row GEMV and for 128+
-    # tokens (SwiGLU in the GEMM epilogue); routed experts 4 (bf16: two GEMV
-    # pairs; 2 for one token, whose experts all have a single token) or 3
+    # tokens (SwiGLU in the GEMM epilogue); routed experts 4 or 5 (bf16: two
+    # GEMV pairs; 2 for one token, whose experts all have a single token) or 3
     # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 3 (the down
     # projection rides with the router rows; its bf16 rounding, the routed sum
     # at width L, the up-projection GEMM)
@@ -264,8 +264,11 @@ def run_ours(args, w):
     # (one token, no latent projection, I_shared <= 2048: the combine runs in
     # the shared down launch)
     fused_combine = rows_path and not w.L and w.I_shared <= 2048
+    # (several tokens, W and I multiples of 512: gate/up, h row scales, down on
+    # the TMA-ring kernels beside the two CUDA-core GEMVs)
+    routed_multi = 5 if (w.W % 512 == 0 and w.I % 512 == 0) else 4
     launches_per_step = (5 - (1 if fused_combine else 0) + shared
-                         + (3 if act == "mxfp4" else (2 if w.T == 1 else 4)) + (3 if w.L else 0))
+                         + (3 if act == "mxfp4" else (2 if w.T == 1 else routed_multi)) + (3 if w.L else 0))
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -667,10 +667,11 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   const bool mma = !(fma && p.T == 1);
   moe_status s = MOE_OK;
   if (fma && (s = launch_fma<true>(ds, f, st)) != MOE_OK) return s;
-  const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
-  if (mma && p.W % 512 == 0) {
-    // CTA-wide TMA ring (W a multiple of 512: whole 512-element slices, and
-    // scale rows a multiple of 16 bytes)
+  // experts with 2+ tokens: CTA-wide TMA rings (W and I multiples of 512:
+  // whole 512-element slices, scale rows a multiple of 16 bytes) with h as
+  // fp32 rows converted to f16 with one scale per row in between; else the
+  // per-warp rings with h in f16 with one scale per 16-element group
+  if (mma && p.W % 512 == 0 && p.I % 512 == 0) {
     moe::MmaGateUpArgs m;
     memset(&m, 0, sizeof(m));
     const uint64_t rows = (uint64_t)p.E * p.I;
@@ -680,11 +681,32 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
         (s = byte_map(&m.map_us, wu_s, rows, p.W / 32, 16, 64, "up scales")) != MOE_OK)
       return s;
     m.g = g;
+    m.h32 = f.h32;
     m.status = at<int32_t>(ws, p.off_status);
     launch_pdl(moe::k_mma_gateup, dim3(ds.num_sms), dim3(32 * (moe::kMmaConsumers + 1)),
                moe::mma_gateup_smem_bytes(), st, m);
     if ((s = launched("expert gate/up (tensor cores, multi-token)")) != MOE_OK) return s;
-  } else if (mma) {
+    float* hrs = g.hscale;                               // [R] row scales in the group-scale region
+    const int grid_h = (int)std::min<long>((p.R + 7) / 8, (long)ds.num_sms * 8);
+    launch_pdl(moe::k_h_rowscale, dim3(grid_h), dim3(256), 0, st, (const float*)f.h32, offsets, p.E,
+               p.R, p.I, g.min_tokens, g.h16, hrs);
+    if ((s = launched("expert h row scales")) != MOE_OK) return s;
+    if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
+    moe::MmaDownArgs d;
+    memset(&d, 0, sizeof(d));
+    const uint64_t drows = (uint64_t)p.E * p.W;
+    if ((s = code_map(&d.map_dq, wd_q, drows, p.I / 2, 128, "down weights")) != MOE_OK ||
+        (s = byte_map(&d.map_ds, wd_s, drows, p.I / 32, 16, 128, "down scales")) != MOE_OK)
+      return s;
+    d.h16 = g.h16; d.hrs = hrs; d.offsets = offsets; d.expert_list = expert_list;
+    d.y_perm = y_perm; d.status = at<int32_t>(ws, p.off_status);
+    d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R; d.min_tokens = g.min_tokens;
+    launch_pdl(moe::k_mma_down, dim3(ds.num_sms), dim3(32 * (moe::kMmaConsumers + 1)),
+               moe::mma_down_smem_bytes(), st, d);
+    return launched("expert down (tensor cores, multi-token)");
+  }
+  const int grid_g = (int)std::min<long>(ny * (p.I / 16), slots);
+  if (mma) {
     launch_pdl(moe::k_gateup_mxfp4, dim3(grid_g), dim3(32), smem, st, g);
     if ((s = launched("expert gate/up")) != MOE_OK) return s;
   }
@@ -695,20 +717,6 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.min_tokens = g.min_tokens;
   if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
   if (!mma) return MOE_OK;
-  if (p.I % 512 == 0) {
-    moe::MmaDownArgs m;
-    memset(&m, 0, sizeof(m));
-    const uint64_t rows = (uint64_t)p.E * p.W;
-    if ((s = code_map(&m.map_dq, wd_q, rows, p.I / 2, 128, "down weights")) != MOE_OK ||
-        (s = byte_map(&m.map_ds, wd_s, rows, p.I / 32, 16, 128, "down scales")) != MOE_OK)
-      return s;
-    m.h16 = d.h16; m.hscale = d.hscale; m.offsets = offsets; m.expert_list = expert_list;
-    m.y_perm = y_perm; m.status = at<int32_t>(ws, p.off_status);
-    m.W = p.W; m.I = p.I; m.E = p.E; m.R = p.R; m.min_tokens = g.min_tokens;
-    launch_pdl(moe::k_mma_down, dim3(ds.num_sms), dim3(32 * (moe::kMmaConsumers + 1)),
-               moe::mma_down_smem_bytes(), st, m);
-    return launched("expert down (tensor cores, multi-token)");
-  }
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
   launch_pdl(moe::k_down_mxfp4, dim3(grid_d), dim3(32), smem, st, d);
   return launched("expert down");

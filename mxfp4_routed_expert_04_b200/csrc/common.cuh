@@ -168,6 +168,23 @@ MOE_DEV float pow2_f32(int n) {
   return n >= -126 ? __uint_as_float((uint32_t)(n + 127) << 23) : __uint_as_float(1u << (n + 149));
 }
 
+// A fragments of the two k16 halves of one block from the row-g / row-g+8 words.
+MOE_DEV void decode_block(uint32_t wg, uint32_t wg8, uint32_t (&a0)[4], uint32_t (&a1)[4]) {
+  uint32_t lo[4], hi[4];
+  e2m1x8_to_f16x8(wg, lo);
+  e2m1x8_to_f16x8(wg8, hi);
+  a0[0] = lo[0]; a0[1] = hi[0]; a0[2] = lo[1]; a0[3] = hi[1];
+  a1[0] = lo[2]; a1[1] = hi[2]; a1[2] = lo[3]; a1[3] = hi[3];
+}
+
+// power-of-two scale mapping a block maximum m into [2^14, 2^15) as f16
+MOE_DEV void f16_block_scale(float m, float& scale, float& inv) {
+  if (!(m > 0.0f) || !isfinite(m)) { scale = 1.0f; inv = 1.0f; return; }
+  const int ex = max(-100, min(127, frexp_exponent(m)));   // m = f * 2^ex, f in [0.5, 1)
+  scale = pow2_f32(ex - 15);
+  inv = pow2_f32(15 - ex);
+}
+
 // Sum of S split-K partials p[0], p[stride], ... in the order s = 0, 1, ...;
 // the loads are issued sixteen at a time ahead of their additions.
 MOE_DEV float sum_splits(const float* __restrict__ p, int S, size_t stride) {

@@ -128,7 +128,12 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   // 2) this CTA's share of the units (gate/up: row pairs; down: rows)
   const long total = (long)n_single * N;
   const long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
-  if (lo >= hi) return;                                   // uniform across the CTA
+  if (lo >= hi) {                                         // uniform across the CTA
+    // no work, but the grid must not complete before the previous one: the
+    // next kernel's wait covers this grid only
+    pdl_wait();
+    return;
+  }
   uint64_t* full = s_bars;
   uint64_t* empty = s_bars + kFmaMaxStages;
   if (threadIdx.x == 0) {

@@ -25,28 +25,32 @@ struct GateUpArgs {
   int min_tokens;            // experts with fewer tokens are left to the CUDA-core path
 };
 
-// Gate/up of the experts with 2+ tokens through a CTA-wide TMA ring (W a
-// multiple of 512): codes by 2-D tensor maps over [E*I, W/2] bytes (boxes of
-// 128 bytes x 64 rows, 128-byte swizzle), scales over [E*I, W/32] bytes
-// (boxes of 16 bytes x 64 rows), token rows by bulk copies; output as in
-// k_gateup_mxfp4 (h16 + per-16-row-group scales).
-constexpr int kMmaConsumers = 8;     // consumer warps (4 row tiles x 2 K halves) plus one producer warp
+// Gate/up of the experts with 2+ tokens through a CTA-wide TMA ring (W and I
+// multiples of 512, gemv_mma.cu): codes by 2-D tensor maps over [E*I, W/2]
+// bytes (boxes of 128 bytes x 64 rows, 128-byte swizzle), scales over
+// [E*I, W/32] bytes (boxes of 16 bytes x 64 rows), token rows by bulk copies;
+// h written as fp32 rows (g.h16 / g.hscale unused).
+constexpr int kMmaConsumers = 16;    // consumer warps plus one producer warp
 constexpr int kMmaStages = 3;
 struct MmaGateUpArgs {
   CUtensorMap map_gq, map_uq, map_gs, map_us;
   GateUpArgs g;
+  float* h32;                // [R, I]
   int32_t* status;
 };
 __global__ void k_mma_gateup(const __grid_constant__ MmaGateUpArgs a);
 size_t mma_gateup_smem_bytes();
-// Down projection of the experts with 2+ tokens, the same ring (I a multiple
-// of 512): down codes [E*W, I/2] (boxes of 128 bytes x 128 rows) and scales
-// [E*W, I/32] (16 bytes x 128 rows) by tensor maps, the tokens' h rows and h
-// group scales by bulk copies.
+// h rows of the experts with >= min_tokens tokens: fp32 [R, I] -> f16 [R, I]
+// with one power-of-two scale per row (hrs [R])
+__global__ void k_h_rowscale(const float* h32, const int32_t* offsets, int E, int R, int I,
+                             int min_tokens, __half* h16, float* hrs);
+// Down projection of the experts with 2+ tokens, the same ring: down codes
+// [E*W, I/2] (boxes of 128 bytes x 128 rows) and scales [E*W, I/32] (16 bytes
+// x 128 rows) by tensor maps, the tokens' f16 h rows by bulk copies.
 struct MmaDownArgs {
   CUtensorMap map_dq, map_ds;
   const __half* h16;         // [R, I]
-  const float* hscale;       // [R, I/16]
+  const float* hrs;          // [R] h row scales
   const int32_t* offsets;
   const int32_t* expert_list;
   float* y_perm;             // [R, W]

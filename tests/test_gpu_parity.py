@@ -42,6 +42,11 @@ ROWS_LATENT_T1 = synth.MoeWorkload("rows_latent_t1", T=1, H=1024, I=128, E=12, k
                                    L=256, seed=81)
 WIDE_LATENT = synth.MoeWorkload("wide_latent", T=130, H=512, I=128, E=6, k=2, I_shared=256, L=384,
                                 seed=82)
+# W and I multiples of 512: experts with 2+ tokens on the TMA-ring tensor-core
+# kernels; more than 16 tokens per expert (several passes over the weights),
+# and a mix of single-token (CUDA-core) and multi-token experts
+MMA_MANY = synth.MoeWorkload("mma_many", T=44, H=1024, I=512, E=6, k=2, I_shared=256, seed=83)
+MMA_MIXED = synth.MoeWorkload("mma_mixed", T=24, H=1024, I=512, E=40, k=2, I_shared=256, seed=84)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
@@ -51,6 +56,8 @@ CASES = [
     (ROWS_T1, None),
     (ROWS_LATENT_T1, None),
     (WIDE_LATENT, None),
+    (MMA_MANY, None),
+    (MMA_MIXED, None),
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
