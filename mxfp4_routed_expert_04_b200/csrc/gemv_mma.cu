@@ -33,7 +33,8 @@ constexpr int kMgRows = 64;                          // weight rows per gate/up 
 constexpr int kMgBox = kMgRows * 128;                // one code box (256 K elements)
 constexpr int kMgCodes = 2 * kMgBox;                 // one matrix's codes of a stage (512 K)
 constexpr int kMgScales = kMgRows * 16;              // one matrix's scales of a stage
-constexpr int kXStride = 1040;                       // token row stride in a stage (65 x 16 bytes)
+constexpr int kXStride = 1088;                       // token row stride in a stage: 68 x 16 bytes, so the
+                                                     // fragment loads of two tokens hit disjoint banks
 constexpr int kMgXOff = 2 * kMgCodes + 2 * kMgScales;
 constexpr int kTok = 16;                             // tokens per pass over the weights
 constexpr int kNG = kTok / 8;                        // 8-token MMA column groups
@@ -76,6 +77,20 @@ MOE_DEV int multi_token_experts(const int32_t* __restrict__ expert_list, const i
   }
   return n_multi;
 }
+
+// True when no byte of w is an E8M0 code 0 or 255 (the two codes whose
+// value is not the plain power of two c << 23).
+MOE_DEV bool e8m0_plain4(uint32_t w) { return (__vcmpeq4(w, 0u) | __vcmpeq4(w, 0xFFFFFFFFu)) == 0u; }
+
+// Value of E8M0 code byte i of w: the exponent field alone on the plain path,
+// else e8m0_to_f32 (2^-127 for code 0, NaN for 255).
+template <int i>
+MOE_DEV float e8m0_byte(uint32_t w, bool plain) {
+  if (plain) return __uint_as_float((i < 3 ? (w << (23 - 8 * i)) : (w >> 1)) & 0x7F800000u);
+  return e8m0_to_f32((w >> (8 * i)) & 0xFFu);
+}
+// Value of E8M0 code c; `plain`: c is known to be neither 0 nor 255
+MOE_DEV float e8m0_value(uint32_t c, bool plain) { return plain ? __uint_as_float(c << 23) : e8m0_to_f32(c); }
 
 MOE_DEV void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
@@ -142,9 +157,6 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
         const int wrow = e * I + rg * kMgRows;
         for (int c0 = 0; c0 < n_all && ok; c0 += kTok) {
           const int nt = min(kTok, n_all - c0);
-          int tok[kTok];
-#pragma unroll
-          for (int c = 0; c < kTok; ++c) tok[c] = c < nt ? __ldg(a.row_token + r0 + c0 + c) : 0;
           for (int s = 0; s < nslice; ++s) {
             if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) { ok = false; break; }
             uint8_t* st = smem + (size_t)slot * kMgStage;
@@ -156,10 +168,9 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
             tc::tma_load_2d(st + kMgCodes + kMgBox, &A.map_uq, s * 256 + 128, wrow, &full[slot]);
             tc::tma_load_2d(st + 2 * kMgCodes, &A.map_gs, s * 16, wrow, &full[slot]);
             tc::tma_load_2d(st + 2 * kMgCodes + kMgScales, &A.map_us, s * 16, wrow, &full[slot]);
-#pragma unroll
-            for (int c = 0; c < kTok; ++c)
-              if (c < nt)
-                bulk_g2s(st + kMgXOff + c * kXStride, a.x16 + (size_t)tok[c] * W + s * 512, 1024u, &full[slot]);
+            for (int c = 0; c < nt; ++c)
+              bulk_g2s(st + kMgXOff + c * kXStride, a.x16 + (size_t)__ldg(a.row_token + r0 + c0 + c) * W + s * 512,
+                       1024u, &full[slot]);
             last_ph[slot] = ph;
             filled[slot] = true;
             if (++slot == kMmaStages) { slot = 0; ph ^= 1u; }
@@ -198,10 +209,11 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
           if (!tc::wait_or_abort(&full[slot], ph, abort)) { ok = false; break; }
           const uint8_t* st = smem + (size_t)slot * kMgStage;
           const uint32_t gq = smem_u32(st) + lda, uq = gq + kMgCodes;
-          const uint8_t* gsc = st + 2 * kMgCodes;
+          // the scales of this warp's four blocks: bytes 4 kq .. 4 kq + 3 of rows g, g + 8
+          const uint8_t* gsc = st + 2 * kMgCodes + 4 * kq;
           const uint8_t* usc = gsc + kMgScales;
           const uint32_t xs0 = smem_u32(st + kMgXOff);
-#pragma unroll
+#pragma unroll 1
           for (int bp = 0; bp < 2; ++bp) {
             const int b0 = 4 * kq + 2 * bp;                    // first block of the pair in the slice
             const int ch = (b0 & 7) + (lq >> 1);               // its 16-byte chunk in the box row
@@ -212,31 +224,31 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_gateup(cons
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
               const int b = b0 + hb;
+              const int sb = 2 * bp + hb;                      // scale byte of the block
+              const float sc[4] = {e8m0_to_f32(gsc[row_g * 16 + sb]), e8m0_to_f32(gsc[row_g8 * 16 + sb]),
+                                   e8m0_to_f32(usc[row_g * 16 + sb]), e8m0_to_f32(usc[row_g8 * 16 + sb])};
               uint32_t ag0[4], ag1[4], au0[4], au1[4];
               decode_block(Rg[2 * hb], Rg[2 * hb + 1], ag0, ag1);
               decode_block(Ru[2 * hb], Ru[2 * hb + 1], au0, au1);
-              const float sg0 = e8m0_to_f32(gsc[row_g * 16 + b]);
-              const float sg8 = e8m0_to_f32(gsc[row_g8 * 16 + b]);
-              const float su0 = e8m0_to_f32(usc[row_g * 16 + b]);
-              const float su8 = e8m0_to_f32(usc[row_g8 * 16 + b]);
 #pragma unroll
               for (int gi = 0; gi < kNG; ++gi) {
                 if (gi < ng) {
-                  const int tk = min(gi * 8 + g, n - 1);
-                  const uint4 xv = lds16(xs0 + tk * kXStride + (32 * b + 8 * t4) * 2);
+                  // columns past n read stale rows of the stage: they only
+                  // reach accumulator columns that are never stored
+                  const uint4 xv = lds16(xs0 + (gi * 8 + g) * kXStride + (32 * b + 8 * t4) * 2);
                   float cg[4] = {0.f, 0.f, 0.f, 0.f}, cu[4] = {0.f, 0.f, 0.f, 0.f};
                   mma_f16(cg, ag0, xv.x, xv.y);
                   mma_f16(cu, au0, xv.x, xv.y);
                   mma_f16(cg, ag1, xv.z, xv.w);
                   mma_f16(cu, au1, xv.z, xv.w);
-                  accG[gi][0] = fmaf(cg[0], sg0, accG[gi][0]);
-                  accG[gi][1] = fmaf(cg[1], sg0, accG[gi][1]);
-                  accG[gi][2] = fmaf(cg[2], sg8, accG[gi][2]);
-                  accG[gi][3] = fmaf(cg[3], sg8, accG[gi][3]);
-                  accU[gi][0] = fmaf(cu[0], su0, accU[gi][0]);
-                  accU[gi][1] = fmaf(cu[1], su0, accU[gi][1]);
-                  accU[gi][2] = fmaf(cu[2], su8, accU[gi][2]);
-                  accU[gi][3] = fmaf(cu[3], su8, accU[gi][3]);
+                  accG[gi][0] = fmaf(cg[0], sc[0], accG[gi][0]);
+                  accG[gi][1] = fmaf(cg[1], sc[0], accG[gi][1]);
+                  accG[gi][2] = fmaf(cg[2], sc[1], accG[gi][2]);
+                  accG[gi][3] = fmaf(cg[3], sc[1], accG[gi][3]);
+                  accU[gi][0] = fmaf(cu[0], sc[2], accU[gi][0]);
+                  accU[gi][1] = fmaf(cu[1], sc[2], accU[gi][1]);
+                  accU[gi][2] = fmaf(cu[2], sc[3], accU[gi][2]);
+                  accU[gi][3] = fmaf(cu[3], sc[3], accU[gi][3]);
                 }
               }
             }
@@ -440,32 +452,44 @@ __global__ void __launch_bounds__(32 * (kMmaConsumers + 1), 1) k_mma_down(const 
           if (!tc::wait_or_abort(&full[slot], ph, abort)) { ok = false; break; }
           const uint8_t* st = smem + (size_t)slot * kMdStage;
           const uint32_t cq = smem_u32(st) + lda;
-          const uint8_t* wsc = st + kMdCodes;
+          // the scales of this warp's eight blocks: bytes 8 kh .. 8 kh + 7 of rows g, g + 8
+          const uint8_t* wsc = st + kMdCodes + 8 * kh;
+          const uint2 w0 = *reinterpret_cast<const uint2*>(wsc + row_g * 16);
+          const uint2 w8 = *reinterpret_cast<const uint2*>(wsc + row_g8 * 16);
+          const bool plain = __all_sync(0xFFFFFFFFu, e8m0_plain4(w0.x) && e8m0_plain4(w0.y) &&
+                                                         e8m0_plain4(w8.x) && e8m0_plain4(w8.y));
           const uint32_t hs0 = smem_u32(st + kMdHOff);
 #pragma unroll 2
           for (int bp = 0; bp < 4; ++bp) {
             uint32_t R[4];
             const int ch = 2 * bp + (lq >> 1);
             ldmatrix_x4(R, cq + ((ch ^ (ldrow & 7)) << 4));
+            const uint32_t s0 = (bp < 2) ? w0.x : w0.y, s8 = (bp < 2) ? w8.x : w8.y;
+            float sc[2][2];                                   // [block][row g, row g+8]
+            if (bp & 1) {
+              sc[0][0] = e8m0_byte<2>(s0, plain); sc[0][1] = e8m0_byte<2>(s8, plain);
+              sc[1][0] = e8m0_byte<3>(s0, plain); sc[1][1] = e8m0_byte<3>(s8, plain);
+            } else {
+              sc[0][0] = e8m0_byte<0>(s0, plain); sc[0][1] = e8m0_byte<0>(s8, plain);
+              sc[1][0] = e8m0_byte<1>(s0, plain); sc[1][1] = e8m0_byte<1>(s8, plain);
+            }
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
               const int b = 8 * kh + 2 * bp + hb;                 // block in the slice
               uint32_t a0[4], a1[4];
               decode_block(R[2 * hb], R[2 * hb + 1], a0, a1);
-              const float ws0 = e8m0_to_f32(wsc[row_g * 16 + b]);
-              const float ws8 = e8m0_to_f32(wsc[row_g8 * 16 + b]);
 #pragma unroll
               for (int gi = 0; gi < kNG; ++gi) {
                 if (gi < ng) {
-                  const int tk = min(gi * 8 + g, n - 1);
-                  const uint4 hv = lds16(hs0 + tk * kXStride + (32 * b + 8 * t4) * 2);
+                  // columns past n read stale rows of the stage (never stored)
+                  const uint4 hv = lds16(hs0 + (gi * 8 + g) * kXStride + (32 * b + 8 * t4) * 2);
                   float c[4] = {0.f, 0.f, 0.f, 0.f};
                   mma_f16(c, a0, hv.x, hv.y);
                   mma_f16(c, a1, hv.z, hv.w);
-                  acc[gi][0] = fmaf(c[0], ws0, acc[gi][0]);
-                  acc[gi][1] = fmaf(c[1], ws0, acc[gi][1]);
-                  acc[gi][2] = fmaf(c[2], ws8, acc[gi][2]);
-                  acc[gi][3] = fmaf(c[3], ws8, acc[gi][3]);
+                  acc[gi][0] = fmaf(c[0], sc[hb][0], acc[gi][0]);
+                  acc[gi][1] = fmaf(c[1], sc[hb][0], acc[gi][1]);
+                  acc[gi][2] = fmaf(c[2], sc[hb][1], acc[gi][2]);
+                  acc[gi][3] = fmaf(c[3], sc[hb][1], acc[gi][3]);
                 }
               }
             }

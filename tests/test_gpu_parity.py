@@ -214,6 +214,36 @@ def test_nan_scale_poisons_only_its_outputs():
             assert np.all(np.isfinite(gpu["y_perm"][r]))
 
 
+def test_nan_scale_multi_token_kernels():
+    """The same on the TMA-ring kernels of experts with 2+ tokens (W, I multiples
+    of 512): a NaN down scale poisons one output column of its expert's rows, a
+    NaN gate scale every output of them; the other expert stays finite."""
+    w = synth.MoeWorkload("edge_mma", T=8, H=512, I=512, E=2, k=1, I_shared=128, seed=92)
+    run = GpuRun(w)
+    gpu0 = run.run_stages()
+    counts = np.diff(gpu0["offsets"][:w.E + 1])
+    e = int(np.argmax(counts))
+    assert counts[e] >= 2
+    rows_e = set(range(int(gpu0["offsets"][e]), int(gpu0["offsets"][e + 1])))
+    saved = run.dev["wd_s"][e, 7, 3].clone()
+    run.dev["wd_s"][e, 7, 3] = 255
+    gpu = run.run_stages()
+    for r in range(w.T * w.k):
+        if r in rows_e:
+            assert np.isnan(gpu["y_perm"][r, 7])
+            assert np.all(np.isfinite(np.delete(gpu["y_perm"][r], 7)))
+        else:
+            assert np.all(np.isfinite(gpu["y_perm"][r]))
+    run.dev["wd_s"][e, 7, 3] = saved
+    run.dev["wg_s"][e, 5, 3] = 255
+    gpu = run.run_stages()
+    for r in range(w.T * w.k):
+        if r in rows_e:
+            assert np.all(np.isnan(gpu["y_perm"][r]))
+        else:
+            assert np.all(np.isfinite(gpu["y_perm"][r]))
+
+
 def test_invalid_expert_index_sets_status_and_empties_routing():
     import mxfp4_routed_expert_04_b200 as M
     w = _small(T=4, E=8, k=2)
