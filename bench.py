@@ -261,9 +261,9 @@ def run_ours(args, w):
     rows_path = w.T == 1 and w.H in rows_k and w.I_shared in rows_k
     # (many tokens: the sigmoid-gate row rides with the router rows as well)
     shared = 2 if (rows_path or w.T >= 128) else 3
-    # (one token, no latent projection, I_shared <= 2048: the combine runs in
-    # the shared down launch)
-    fused_combine = rows_path and not w.L and w.I_shared <= 2048
+    # (one token, no latent projection: the combine runs in the shared down
+    # launch)
+    fused_combine = rows_path and not w.L
     # (several tokens, W and I multiples of 512: gate/up, h row scales, down on
     # the TMA-ring kernels beside the two CUDA-core GEMVs)
     routed_multi = 5 if (w.W % 512 == 0 and w.I % 512 == 0) else 4

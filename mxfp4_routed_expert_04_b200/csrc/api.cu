@@ -42,7 +42,7 @@ constexpr int kDenseSwiGLUTokens = 128;
 // 16-token tile.
 bool rows_k_ok(int K) { return K == 1024 || K == 2048 || K == 4096 || K == 8192; }
 bool rows_path_for(int T, int H, int Is) { return T == 1 && rows_k_ok(H) && rows_k_ok(Is); }
-constexpr size_t kRowsSmemBudget = 200 * 1024;
+constexpr size_t kRowsSmemBudget = 220 * 1024;
 constexpr int kRowsFreeSMs = 8;     // SMs a side-stream row GEMV leaves to the routing chain
 
 // Token tile of the tcgen05 bf16 GEMM: the MMA's N, a multiple of 16 up to 128.
@@ -272,13 +272,17 @@ moe_status device_state(DeviceState** out) {
 // the shared-memory budget
 moe_status launch_rows(const DeviceState& ds, moe::RowsArgs& r, bool swiglu, bool x_f32, int max_ctas,
                        cudaStream_t st, const char* what, bool pdl = true) {
-  r.nst = moe::rows_stages(r.K, kRowsSmemBudget);
-  if (!r.nst) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: K=%d too long for the row GEMV", what, r.K);
   const long units = swiglu ? r.rows[0] : (long)r.rows[0] + r.rows[1] + r.rows[2];
-  const long slots = moe::kRowsConsumers / moe::rows_warps_per_row(r.K);
-  const long per = swiglu ? slots / 2 : slots;
-  const int grid = (int)std::max<long>(1, std::min<long>((units + per - 1) / per, max_ctas));
-  const size_t smem = (size_t)r.nst * moe::rows_stage_bytes(r.K);
+  const int grid = (int)std::max<long>(1, std::min<long>(units, max_ctas));
+  // slots of a stage: the units of a CTA rounded up to a power of two (at
+  // most 16 MMA rows), so that a CTA's few rows come in whole-row stages
+  const long per = (units + grid - 1) / grid;
+  int pp = 1;
+  while (pp < per && pp < (swiglu ? 8 : 16)) pp <<= 1;
+  r.slots = swiglu ? 2 * pp : pp;
+  r.nst = moe::rows_stages(r.K, r.slots, x_f32, kRowsSmemBudget);
+  if (!r.nst) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: K=%d too long for the row GEMV", what, r.K);
+  const size_t smem = (size_t)r.nst * moe::rows_stage_bytes(r.K, r.slots) + moe::rows_act_bytes(r.K, x_f32);
   void (*kern)(moe::RowsArgs) = swiglu ? moe::k_rows_bf16<true, false>
                                        : (x_f32 ? moe::k_rows_bf16<false, true> : moe::k_rows_bf16<false, false>);
   const dim3 block(32 * (moe::kRowsConsumers + 1));
@@ -551,10 +555,9 @@ moe_status do_shared_up(const Plan& p, const DeviceState& ds, const uint16_t* x,
 
 // Shared expert, second half: the down GEMM over both halves of h (split-K
 // partial sums for the combine).
-// One token on the row GEMV with the shared down rows whole per warp
-// (I_shared <= 2048) and no latent projection: the shared down launch also
-// finishes the combine (same order of operations as k_combine).
-bool combine_in_shared_down(const Plan& p) { return p.rows && p.L == 0 && p.Is <= 2048; }
+// One token on the row GEMV and no latent projection: the shared down launch
+// also finishes the combine (same order of operations as k_combine).
+bool combine_in_shared_down(const Plan& p) { return p.rows && p.L == 0; }
 
 // comb (combine_in_shared_down): y_perm, slot_row, topk_w of the routed
 // experts and the layer output y
@@ -592,10 +595,20 @@ moe_status do_shared_down(const Plan& p, const DeviceState& ds, const uint16_t* 
 // MXFP4 activations: gate/up (+ SwiGLU, h quantised to MXFP4) and down on the
 // tensor cores, one persistent CTA per SM each; the tile list and the token
 // operand come from moe_permute (inside x_op), weight scales are tiled.
+// Make `st` wait for `ev` (NULL: nothing) before the next launch.
+moe_status join_before(cudaEvent_t ev, cudaStream_t st) {
+  if (!ev) return MOE_OK;
+  const cudaError_t e = cudaStreamWaitEvent(st, ev, 0);
+  return e == cudaSuccess ? MOE_OK : fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
+}
+
+// `join` (or NULL): an event the down projection waits for (moe_layer joins
+// the shared expert's stream there, well after that work is done, so that the
+// join never delays a launch)
 moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* x_op,
                               const uint8_t* wg_q, const uint8_t* wg_s, const uint8_t* wu_q,
                               const uint8_t* wu_s, const uint8_t* wd_q, const uint8_t* wd_s,
-                              float* y_perm, void* ws, cudaStream_t st) {
+                              float* y_perm, void* ws, cudaStream_t st, cudaEvent_t join = nullptr) {
   void* xop = const_cast<void*>(x_op);
   const int4* tiles = at<int4>(xop, p.xop_tiles_off);
   const int32_t* n_tiles = at<int32_t>(xop, p.xop_ntiles_off);
@@ -630,6 +643,7 @@ moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* 
   d.y = y_perm;
   d.status = g.status;
   d.K = p.I; d.M = p.W;
+  if ((s = join_before(join, st)) != MOE_OK) return s;
   moe::k_mxf4_gemm<false><<<ds.num_sms, threads, moe::mxf4_gemm_smem_bytes(false), st>>>(d);
   return launched("expert down (tcgen05)");
 }
@@ -638,9 +652,10 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const int32_t* offsets, const int32_t* expert_list,
                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
-                         const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st) {
+                         const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st,
+                         cudaEvent_t join = nullptr) {
   if (p.mode == MOE_ACT_MXFP4)
-    return do_expert_ffn_mxf4(p, ds, x_op, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st);
+    return do_expert_ffn_mxf4(p, ds, x_op, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st, join);
   const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
   moe::GateUpArgs g;
   g.x16 = static_cast<const __half*>(x_op);
@@ -691,6 +706,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
     launch_pdl(moe::k_h_rowscale, dim3(grid_h), dim3(256), 0, st, (const float*)f.h32, offsets, p.E,
                p.R, p.I, g.min_tokens, g.h16, hrs);
     if ((s = launched("expert h row scales")) != MOE_OK) return s;
+    if ((s = join_before(join, st)) != MOE_OK) return s;
     if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
     moe::MmaDownArgs d;
     memset(&d, 0, sizeof(d));
@@ -715,6 +731,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   d.wd_q = wd_q; d.wd_s = wd_s; d.y_perm = y_perm;
   d.W = p.W; d.I = p.I; d.E = p.E; d.R = p.R;
   d.min_tokens = g.min_tokens;
+  if ((s = join_before(join, st)) != MOE_OK) return s;
   if (fma && (s = launch_fma<false>(ds, f, st)) != MOE_OK) return s;
   if (!mma) return MOE_OK;
   const int grid_d = (int)std::min<long>(ny * (p.W / 32), slots);
@@ -1015,13 +1032,15 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
                       a->expert_list, a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) !=
       MOE_OK)
     return s;
-  // the routed experts start once the shared expert's first half is done, so
-  // that they have every SM from their first stage on
-  if ((e = cudaStreamWaitEvent(st, ds->ev_shared, 0)) != cudaSuccess)
-    return fail(MOE_ERR_CUDA, "join: %s", cudaGetErrorString(e));
+  // the routed experts follow the dispatch directly (their CTAs take the SMs
+  // the shared expert's first half leaves); the shared stream joins before the
+  // shared down projection, the first reader of its output (a joined launch
+  // loses the early start of programmatic serialisation, a few microseconds,
+  // wherever the join sits)
   if ((s = do_expert_ffn(p, *ds, a->x_op, a->offsets, a->expert_list, a->row_token, a->wg_q,
                          a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
     return s;
+  if ((s = join_before(ds->ev_shared, st)) != MOE_OK) return s;
   if (combine_in_shared_down(p))
     return do_shared_down(p, *ds, a->ws_down, ws, st, 0, a->y_perm, a->slot_row, a->topk_w, a->y);
   if ((s = do_shared_down(p, *ds, a->ws_down, ws, st)) != MOE_OK) return s;

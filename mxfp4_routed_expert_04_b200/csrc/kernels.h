@@ -132,10 +132,9 @@ template <bool kGateUp> __global__ void k_mxf4_gemm(const __grid_constant__ Mxf4
 size_t mxf4_gemm_smem_bytes(bool gate_up);
 int mxf4_gemm_threads();
 
-// --- single-token bf16 GEMV on the CUDA cores (whole rows per CTA) ---------
+// --- single-token bf16 GEMV (contiguous row ranges per CTA, mma.sync) ------
 constexpr int kRowsConsumers = 16;   // consumer warps (plus one producer warp)
 constexpr int kRowsMaxStages = 8;
-constexpr int kRowsMaxChunks = 8;    // 8-element chunks per lane (2048 elements per warp)
 struct RowsArgs {
   const uint16_t* w[3];      // bf16 [rows[i], K]; SwiGLU: w[0] gate, w[1] up
   int rows[3];               // plain: segment rows (0: unused); SwiGLU: rows[0] = row pairs
@@ -143,7 +142,8 @@ struct RowsArgs {
   const void* x;             // [K] bf16, or fp32 (k_rows_bf16<*, true>)
   int32_t* status;
   int K, nst;
-  // optional combine of one token (plain mode, K <= 2048): instead of
+  int slots;                 // row slots of a stage: 1..16 (plain), 2..16 (SwiGLU), a power of two
+  // optional combine of one token (plain mode): instead of
   // out[0][row], y[row] = sum_j topk_w[j] * y_perm[slot_row[j], row]
   //                      + sigmoid(gate_logit[0]) * (Wx)[row]
   float* y;                  // [rows[0]] or NULL
@@ -154,13 +154,17 @@ struct RowsArgs {
   int k;
 };
 template <bool kSwiGLU, bool kXF32> __global__ void k_rows_bf16(RowsArgs a);
-// K a power of two in 1024..8192: warps per row K/2048 (at least 1), a stage
-// of 16 / that many rows
-__host__ __device__ constexpr int rows_warps_per_row(int K) { return K > 2048 ? K / 2048 : 1; }
-__host__ __device__ constexpr size_t rows_stage_bytes(int K) {
-  return (size_t)(kRowsConsumers / rows_warps_per_row(K)) * K * 2;
+// K a power of two in 1024..8192: a stage holds `slots` row slots (plain:
+// rows; SwiGLU: half gate, half up rows) of a K chunk of about 64 KB over the
+// slots, each slot 16 bytes longer than the chunk (conflict-free ldmatrix);
+// after the ring the activation (bf16 x [K], or the bf16 hi/lo pair [2][K]
+// of fp32 x)
+__host__ __device__ constexpr int rows_chunk(int K, int slots) { return K < 32768 / slots ? K : 32768 / slots; }
+__host__ __device__ constexpr size_t rows_stage_bytes(int K, int slots) {
+  return (size_t)slots * ((size_t)rows_chunk(K, slots) * 2 + 16);
 }
-int rows_stages(int K, size_t smem_budget);
+__host__ __device__ constexpr size_t rows_act_bytes(int K, bool x_f32) { return (size_t)K * (x_f32 ? 4 : 2); }
+int rows_stages(int K, int slots, bool x_f32, size_t smem_budget);
 
 // --- dense bf16 GEMM on tcgen05 -----------------------------------------------
 // Weights [rows, K] and tokens [T, K] bf16 through 2-D tensor maps (weights:
