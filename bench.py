@@ -267,7 +267,10 @@ def run_ours(args, w):
     # (several tokens, W and I multiples of 512: gate/up, h row scales, down on
     # the TMA-ring kernels beside the two CUDA-core GEMVs)
     routed_multi = 5 if (w.W % 512 == 0 and w.I % 512 == 0) else 4
-    launches_per_step = (5 - (1 if fused_combine else 0) + shared
+    # (one token, bf16 activations, no latent projection: the top-k launch also
+    # writes the dispatch and the activation operand)
+    fused_dispatch = w.T == 1 and act == "bf16" and not w.L
+    launches_per_step = (5 - (1 if fused_combine else 0) - (2 if fused_dispatch else 0) + shared
                          + (3 if act == "mxfp4" else (2 if w.T == 1 else routed_multi)) + (3 if w.L else 0))
 
     def timed(fn, steps):

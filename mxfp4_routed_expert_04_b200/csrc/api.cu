@@ -440,10 +440,13 @@ moe_status round_latent(const Plan& p, const float* part, int ld, uint16_t* x_la
 // The router logits, then top-k. The same pass over x can carry the shared
 // expert's sigmoid-gate row (w_sgate) and the latent down-projection (w_ld,
 // rounded to bf16 into x_lat after the top-k).
+// (fuse: one token in bf16 mode, the top-k launch also writes the dispatch
+// and the activation operand; moe_permute is then skipped)
 moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
                     int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st,
                     const uint16_t* w_sgate = nullptr, const uint16_t* w_ld = nullptr,
-                    uint16_t* x_lat = nullptr) {
+                    uint16_t* x_lat = nullptr, const moe::TopkFuse* fuse = nullptr) {
+  const moe::TopkFuse tf = fuse ? *fuse : moe::TopkFuse{};
   float* part = at<float>(ws, p.off_router);
   moe_status s;
   if (p.rows) {
@@ -456,7 +459,7 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
     r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
     if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
     launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
-               p.E, p.k, idx, w, logits, (float*)nullptr);
+               p.E, p.k, idx, w, logits, (float*)nullptr, tf);
     if ((s = launched("top-k")) != MOE_OK) return s;
     return w_ld ? round_latent(p, at<float>(ws, p.off_ld), p.L, x_lat, st) : MOE_OK;
   }
@@ -476,7 +479,7 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
   g.seg_rows[0] = p.E; g.seg_rows[1] = w_sgate ? 1 : 0; g.seg_rows[2] = w_ld ? p.L : 0; g.ld = ld;
   if ((s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)")) != MOE_OK) return s;
   launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E,
-             ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr);
+             ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr, tf);
   if ((s = launched("top-k")) != MOE_OK) return s;
   return w_ld ? round_latent(p, part + lat_col, ld, x_lat, st) : MOE_OK;
 }
@@ -1013,9 +1016,19 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   // (one token or the SwiGLU-epilogue GEMM: the sigmoid-gate row rides along
   // with the router rows; the latent down-projection always does)
   const bool sgate_with_router = p.rows || p.swiglu_tc;
+  // one token, bf16 activations, no latent projection: the top-k launch also
+  // writes the dispatch and the activation operand (what moe_permute writes)
+  const bool fused_dispatch = p.T == 1 && p.mode == MOE_ACT_BF16 && p.L == 0;
+  moe::TopkFuse tf{};
+  if (fused_dispatch) {
+    tf.counts = a->counts; tf.offsets = a->offsets; tf.expert_list = a->expert_list;
+    tf.row_token = a->row_token; tf.row_slot = a->row_slot; tf.slot_row = a->slot_row;
+    tf.x = a->x; tf.W = p.W;
+    tf.x16 = static_cast<__half*>(a->x_op); tf.xscale = at<float>(a->x_op, p.xop_scale_off);
+  }
   if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st,
                     sgate_with_router ? a->w_sgate : nullptr, p.L ? a->w_lat_down : nullptr,
-                    a->x_lat)) != MOE_OK)
+                    a->x_lat, fused_dispatch ? &tf : nullptr)) != MOE_OK)
     return s;
   // side stream: the first half of the shared expert (it streams its weights
   // while the routing chain runs)
@@ -1028,9 +1041,9 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));
   // main stream: dispatch, experts, combine
-  if ((s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets,
-                      a->expert_list, a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) !=
-      MOE_OK)
+  if (!fused_dispatch &&
+      (s = do_permute(p, a->topk_idx, p.L ? a->x_lat : a->x, a->counts, a->offsets, a->expert_list,
+                      a->row_token, a->row_slot, a->slot_row, a->x_op, ws, st)) != MOE_OK)
     return s;
   // the routed experts follow the dispatch directly (their CTAs take the SMs
   // the shared expert's first half leaves); the shared stream joins before the

@@ -316,15 +316,18 @@ __global__ void __launch_bounds__(256) k_h_rowscale(const float* __restrict__ h3
                                                     float* __restrict__ hrs) {
   pdl_wait();
   pdl_trigger();
+  __shared__ int s_off[1025];                             // offsets[0..E], E <= 1024
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = __ldg(offsets + i);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < R; r += gridDim.x * 8) {
     // the expert of row r: offsets[e] <= r < offsets[e + 1]
     int lo = 0, hi = E;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (__ldg(offsets + mid) <= r) lo = mid; else hi = mid;
+      if (s_off[mid] <= r) lo = mid; else hi = mid;
     }
-    if (__ldg(offsets + lo + 1) - __ldg(offsets + lo) < min_tokens) continue;
+    if (s_off[lo + 1] - s_off[lo] < min_tokens) continue;
     const float4* src = reinterpret_cast<const float4*>(h32 + (size_t)r * I);
     float m = 0.0f;
     for (int i = lane; i < I / 4; i += 32) {

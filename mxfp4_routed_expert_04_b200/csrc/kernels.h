@@ -216,10 +216,21 @@ constexpr int kDenseWarps = 4;   // warps (16-row tiles) per CTA
 
 // --- router tail ------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
+// One token with bf16 activations: k_topk can also write what k_permute and
+// k_act_to_f16 write for it (the dispatch of its k experts and the f16 row
+// with its power-of-two scale); x == NULL: top-k only.
+struct TopkFuse {
+  int32_t *counts, *offsets, *expert_list, *row_token, *row_slot, *slot_row;
+  const uint16_t* x;         // [W] bf16
+  int W;                     // a multiple of 8
+  __half* x16;               // [W]
+  float* xscale;             // [1]
+};
 // part [S, T, ld] router partial sums (ld >= E); with gate_logit set, column E
-// holds the sigmoid-gate row's partials and gate_logit[t] gets their sum
+// holds the sigmoid-gate row's partials and gate_logit[t] gets their sum;
+// f.x set: T == 1 and the fused dispatch above
 __global__ void k_topk(const float* part, int S, int T, int E, int ld, int k, int32_t* idx, float* w,
-                       float* logits, float* gate_logit);
+                       float* logits, float* gate_logit, TopkFuse f);
 
 // --- permutation and activation operands ------------------------------------
 __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,

@@ -23,12 +23,17 @@ namespace moe {
 // 3) the experts above it are taken, then experts equal to it by ascending
 //    index until k are taken;
 // 4) warp 0 orders the k by descending logit, equal logits by ascending index,
-//    and computes the renormalised weights.
+//    and computes the renormalised weights;
+// with f.x set (one token): step 3 also writes the dispatch (expert e's row =
+// its rank among the selected by index, as k_permute places a lone token's
+// pairs) and step 4 the slot <-> row maps, while warps 1..31 write the f16
+// activation row with its power-of-two scale (the arithmetic of
+// k_act_to_f16).
 __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__ part, int S, int T,
                                                      int E, int ld, int k, int32_t* __restrict__ idx,
                                                      float* __restrict__ w,
                                                      float* __restrict__ logits,
-                                                     float* __restrict__ gate_logit) {
+                                                     float* __restrict__ gate_logit, TopkFuse f) {
   pdl_wait();
   pdl_trigger();
   __shared__ int s_cnt[kTopkThreads / 32];
@@ -68,15 +73,62 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   __syncthreads();
   if (lane == 0) s_cnt[warp] = __popc(sel_m);
   __syncthreads();
+  int pos = __popc(sel_m & lt_mask);                     // selected experts below e
+  for (int w2 = 0; w2 < warp; ++w2) pos += s_cnt[w2];
   if (sel) {
-    int pos = __popc(sel_m & lt_mask);
-    for (int w2 = 0; w2 < warp; ++w2) pos += s_cnt[w2];
     s_key[pos] = key;
     s_exp[pos] = e;
     s_val[pos] = v;
   }
+  const bool fuse = f.x != nullptr;
+  if (fuse) {
+    if (live) {
+      f.counts[e] = sel ? 1 : 0;
+      f.offsets[e] = pos;
+      if (sel) f.expert_list[1 + pos] = e;
+    }
+    if (e == 0) {
+      f.offsets[E] = k;
+      f.expert_list[0] = k;
+    }
+  }
   __syncthreads();
-  if (warp != 0) return;
+  if (warp != 0) {
+    if (fuse) {
+      // the activation operand: the row's largest magnitude, then f16 with
+      // the power-of-two scale that maps it into [2^14, 2^15)
+      __shared__ float s_max[kTopkThreads / 32];
+      const int tid = threadIdx.x - 32, nthr = kTopkThreads - 32;
+      float m = 0.0f;
+      for (int i = tid * 8; i < f.W; i += nthr * 8) {
+        const uint4 xv = ldg16(f.x + i);
+        const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16lo(wv[j])), fabsf(bf16hi(wv[j]))));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      if (lane == 0) s_max[warp] = m;
+      asm volatile("bar.sync 1, %0;\n" ::"n"(kTopkThreads - 32) : "memory");
+      m = s_max[1];
+      for (int w2 = 2; w2 < kTopkThreads / 32; ++w2) m = fmaxf(m, s_max[w2]);
+      float scale, inv;
+      f16_block_scale(m, scale, inv);
+      for (int i = tid * 8; i < f.W; i += nthr * 8) {
+        const uint4 xv = ldg16(f.x + i);
+        const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(bf16lo(wv[j]) * inv, bf16hi(wv[j]) * inv);
+          o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(f.x16 + i) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      if (tid == 0) f.xscale[0] = scale;
+    }
+    return;
+  }
   // lane i < k: its rank among the k taken (descending key, then ascending index)
   uint32_t ki = 0;
   int ei = 0;
@@ -89,6 +141,11 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
     rank += (kj > ki || (kj == ki && ej < ei)) ? 1 : 0;
   }
   __syncwarp();
+  if (fuse && lane < k) {          // row `lane` (ascending expert) holds slot `rank`
+    f.row_token[lane] = 0;
+    f.row_slot[lane] = rank;
+    f.slot_row[rank] = lane;
+  }
   if (lane < k) { s_exp[rank] = ei; s_val[rank] = vi; }
   __syncwarp();
   // lane r now holds the r-th selection

@@ -106,7 +106,7 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x,
   const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (a.T + 31) / 32);
   moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, cs>>>(a);
   moe::k_topk<<<dims->T, moe::kTopkThreads, 0, cs>>>(part, S, dims->T, dims->E, dims->E, dims->k, topk_idx,
-                                                     topk_w, logits, nullptr);
+                                                     topk_w, logits, nullptr, moe::TopkFuse{});
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return moe::record_error(MOE_ERR_CUDA, cudaGetErrorString(e));
   return MOE_OK;

@@ -152,6 +152,16 @@ def test_fused_layer_matches_stages_bitwise(case):
     w, sample, run, gpu = case
     y = run.run_layer()
     np.testing.assert_array_equal(y, gpu["y"])
+    # the layer's routing, dispatch and activation operand (written by fused
+    # launches for one token) equal the step calls' as well
+    L = run.layer
+    for name, t in (("idx", L.topk_idx), ("counts", L.counts), ("offsets", L.offsets),
+                    ("row_token", L.row_token), ("row_slot", L.row_slot), ("slot_row", L.slot_row),
+                    ("x_op", L.x_op)):
+        np.testing.assert_array_equal(t.cpu().numpy(), gpu[name], err_msg=name)
+    n = int(gpu["expert_list"][0])
+    np.testing.assert_array_equal(L.expert_list.cpu().numpy()[:1 + n], gpu["expert_list"][:1 + n])
+    np.testing.assert_array_equal(L.topk_w.cpu().numpy().astype(np.float64), gpu["w"])
     y2 = run.run_layer()
     np.testing.assert_array_equal(y2, y)
 
