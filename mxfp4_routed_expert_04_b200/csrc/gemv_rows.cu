@@ -182,27 +182,38 @@ __global__ void __launch_bounds__(32 * (kRowsConsumers + 1), 1) k_rows_bf16(Rows
       // the routed values of output row w for the combine, loaded ahead of the group
       float v = 0.0f;
       if (!kSwiGLU && a.y && w < n && lane < a.k) v = __ldg(a.y_perm + (size_t)sr * a.rows[0] + r + w);
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulators (even and odd k16 steps; fp32 x: the hi and the lo
+      // halves) halve the chain of dependent MMAs; added at the group's end
+      float d[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
       for (int kc = 0; kc < nkc; ++kc) {
         if (!tc::wait_or_abort(&full[slot], ph, abort)) { ok = false; break; }
         const uint32_t ab = smem_u32(smem + (size_t)slot * stage_bytes) + lrow * slot_bytes + (kw0 + lcol) * 2;
         const uint32_t xb = xa + (uint32_t)(kc * KC + kw0 + 2 * t4) * 2u;
-        for (int s = 0; s < steps; ++s) {
-          uint32_t A[4];
-          ldmatrix_x4(A, ab + 32u * s);
-          mma_bf16(d, A, lds32(xb + 32u * s), lds32(xb + 32u * s + 16u));
-          if (kXF32)
-            mma_bf16(d, A, lds32(xb + (uint32_t)K * 2u + 32u * s), lds32(xb + (uint32_t)K * 2u + 32u * s + 16u));
+        if (kXF32) {
+          for (int s = 0; s < steps; ++s) {
+            uint32_t A[4];
+            ldmatrix_x4(A, ab + 32u * s);
+            mma_bf16(d, A, lds32(xb + 32u * s), lds32(xb + 32u * s + 16u));
+            mma_bf16(d2, A, lds32(xb + (uint32_t)K * 2u + 32u * s), lds32(xb + (uint32_t)K * 2u + 32u * s + 16u));
+          }
+        } else {
+          for (int s = 0; s < steps; s += 2) {       // steps is even (KC >= 512)
+            uint32_t A[4], B[4];
+            ldmatrix_x4(A, ab + 32u * s);
+            ldmatrix_x4(B, ab + 32u * s + 32u);
+            mma_bf16(d, A, lds32(xb + 32u * s), lds32(xb + 32u * s + 16u));
+            mma_bf16(d2, B, lds32(xb + 32u * s + 32u), lds32(xb + 32u * s + 48u));
+          }
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&empty[slot]);   // this warp is done with the slot
         if (++slot == nst) { slot = 0; ph ^= 1u; }
       }
       if (!ok) break;
-      // every column of the fragment holds the same sums: rows g (d[0]) and g + 8 (d[2])
+      // every column of the fragment holds the same sums: rows g ([0]) and g + 8 ([2])
       if (t4 == 0) {
-        s_red[gp][w][g] = d[0];
-        s_red[gp][w][g + 8] = d[2];
+        s_red[gp][w][g] = d[0] + d2[0];
+        s_red[gp][w][g + 8] = d[2] + d2[2];
       }
       consumer_barrier();
       if (w < n) {
