@@ -95,7 +95,10 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   __shared__ int s_abort;
   __shared__ float2 s_part[2][kFmaConsumers / 2][2];   // gate/up partial sums [stage&1][pair][half]
   constexpr int kWarps = kFmaConsumers + 1;
-  constexpr int P = kGateUp ? kFmaConsumers / 2 : kFmaConsumers * RPS;   // units per stage
+  // gate/up with K > 2048: two warps per row pair, each over half of K; with
+  // shorter rows one warp per pair (twice the pairs per stage, no exchange)
+  constexpr bool kSplit = kGateUp && BPL > 2;
+  constexpr int P = kGateUp ? (kSplit ? kFmaConsumers / 2 : kFmaConsumers) : kFmaConsumers * RPS;   // units per stage
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int K = kGateUp ? a.W : a.I;
   const int KB = K >> 5;
@@ -243,14 +246,15 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
     }
   } else {
     // ---------------- consumers ----------------
-    // gate/up: warps 2p and 2p+1 share row pair p of a stage, each over one
-    // half of K (half the activation registers), and combine their partial
-    // sums through shared memory; down: warp w takes rows RPS*w ... of a stage
+    // gate/up, K > 2048: warps 2p and 2p+1 share row pair p of a stage, each
+    // over one half of K (half the activation registers), and combine their
+    // partial sums through shared memory; K <= 2048: warp w takes row pair w;
+    // down: warp w takes rows RPS*w ... of a stage
     pdl_wait();                             // the previous grid's outputs (xscale)
     const int w = warp - 1;
-    constexpr int BW = kGateUp ? (BPL + 1) / 2 : BPL;    // blocks per lane of this warp
-    const int half = kGateUp ? (w & 1) : 0;
-    const int KBw = kGateUp ? KB / 2 : KB;                // blocks of this warp's K range
+    constexpr int BW = kSplit ? (BPL + 1) / 2 : BPL;     // blocks per lane of this warp
+    const int half = kSplit ? (w & 1) : 0;
+    const int KBw = kSplit ? KB / 2 : KB;                 // blocks of this warp's K range
     const int kb0 = half * KBw;                           // its first block
     uint32_t xr[BW][16];
     float bsc[BW];                                        // down: per-block scale of h
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       // rows of this warp: gate/up -> row 0 = gate, row 1 = up of pair w/2;
       // down -> rows RPS*w ... (codes qrow apart, scales srow apart)
       constexpr int NR = kGateUp ? 2 : RPS;
-      const int u0 = kGateUp ? (w >> 1) : RPS * w;
+      const int u0 = kGateUp ? (kSplit ? (w >> 1) : w) : RPS * w;
       float acc[NR];
 #pragma unroll
       for (int rr = 0; rr < NR; ++rr) acc[rr] = 0.0f;
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
             }
           }
         }
-        if (kGateUp) {
+        if (kSplit) {
           const float gs = warp_sum(acc[0]), us = warp_sum(acc[1]);
           float2* part = s_part[k & 1][u0];
           if (lane == 0) part[half] = make_float2(gs, us);
@@ -387,6 +391,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
             const float2 o = part[1];
             a.h32[(size_t)r0 * a.I + r + u0] = silu_f32((gs + o.x) * xs) * ((us + o.y) * xs);
           }
+        } else if (kGateUp) {
+          const float gs = warp_sum(acc[0]), us = warp_sum(acc[1]);
+          if (lane == 0) a.h32[(size_t)r0 * a.I + r + u0] = silu_f32(gs * xs) * (us * xs);
         } else {
 #pragma unroll
           for (int rr = 0; rr < NR; ++rr) {
@@ -411,7 +418,8 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 
 // Geometry for reduction length K (host side): rows per consumer warp in a
 // down stage rps = max(1, 8 / BPL); a stage holds kFmaConsumers / 2 row pairs
-// (gate/up: the gate rows, then the up rows, then the two E8M0 spans) or
+// (kFmaConsumers for K <= 2048; gate/up: the gate rows, then the up rows, then
+// the two E8M0 spans) or
 // kFmaConsumers * rps rows (down: codes, then their span); every span with 32
 // bytes of alignment slack; after the ring the activation buffer (gate/up: an
 // f16 token row of K; down: an fp32 h row of K, its f16 copy and K/32 fp32
@@ -422,7 +430,7 @@ FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget) {
   const int bpl = (K + 1023) / 1024;
   if (bpl > 8) return g;
   const int rps = gate_up ? 1 : (bpl > 4 ? 1 : bpl > 2 ? 2 : bpl > 1 ? 4 : 8);
-  const int units = gate_up ? kFmaConsumers / 2 : kFmaConsumers * rps;
+  const int units = gate_up ? (bpl > 2 ? kFmaConsumers / 2 : kFmaConsumers) : kFmaConsumers * rps;
   g.rps = rps;
   g.units = units;
   g.code_bytes = (uint32_t)((units * qrow + 127) / 128 * 128);
