@@ -36,10 +36,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // partial sums and a finaliser applies SwiGLU).
 constexpr int kDenseSwiGLUTokens = 128;
 
-// One token: the router and the shared expert stream whole weight rows on the
-// CUDA cores (k_rows_bf16) when both reduction lengths (H, I_shared) are
-// powers of two in 1024..8192; otherwise they take the tcgen05 GEMM with a
-// 16-token tile.
+// One token: the router and the shared expert stream contiguous ranges of
+// weight rows through the tensor-core row GEMV (k_rows_bf16, no split-K) when
+// both reduction lengths (H, I_shared) are powers of two in 1024..8192;
+// otherwise they take the tcgen05 GEMM with a 16-token tile.
 bool rows_k_ok(int K) { return K == 1024 || K == 2048 || K == 4096 || K == 8192; }
 bool rows_path_for(int T, int H, int Is) { return T == 1 && rows_k_ok(H) && rows_k_ok(Is); }
 constexpr size_t kRowsSmemBudget = 220 * 1024;

@@ -201,7 +201,7 @@ __host__ __device__ constexpr int bf16_stages(int N, int passes) {
 size_t bf16_gemm_smem_bytes(int N, int passes);
 int bf16_gemm_threads();
 
-// --- dense bf16 GEMV with split-K partial sums -----------------------------
+// --- dense bf16 GEMV with split-K partial sums (moe_route_noalloc's router) -
 struct DenseArgs {
   const uint16_t* w[3];      // row segments of the weight matrix, each [rows, K]
   int rows[3];
