@@ -247,9 +247,10 @@ moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16
  * Every buffer of the calls above in one struct; moe_layer enqueues the same
  * arithmetic as route -> (latent_down) -> permute -> expert_ffn -> combine
  * (bit for bit: the latent down-projection rows ride in the router's pass over
- * x with the same splits as the stand-alone call), with the first half of the
- * shared expert on a second stream forked from and joined back into `stream`
- * (capturable in a CUDA graph).
+ * x with the same splits as the stand-alone call; for one token in bf16 mode
+ * without a latent projection the top-k launch also writes what moe_permute
+ * writes), with the first half of the shared expert on a second stream forked
+ * from and joined back into `stream` (capturable in a CUDA graph).
  */
 typedef struct {
   const uint16_t* x;

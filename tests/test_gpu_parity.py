@@ -46,6 +46,9 @@ WIDE_LATENT = synth.MoeWorkload("wide_latent", T=130, H=512, I=128, E=6, k=2, I_
 # kernels; more than 16 tokens per expert (several passes over the weights),
 # and a mix of single-token (CUDA-core) and multi-token experts
 MMA_MANY = synth.MoeWorkload("mma_many", T=44, H=1024, I=512, E=6, k=2, I_shared=256, seed=83)
+# one token with H off the row GEMV's lengths: router and shared expert on the
+# tcgen05 GEMM (16-token tile), dispatch and operand from the top-k launch
+TC_T1 = synth.MoeWorkload("tc_t1", T=1, H=640, I=256, E=12, k=3, I_shared=384, seed=85)
 MMA_MIXED = synth.MoeWorkload("mma_mixed", T=24, H=1024, I=512, E=40, k=2, I_shared=256, seed=84)
 
 CASES = [
@@ -58,6 +61,7 @@ CASES = [
     (WIDE_LATENT, None),
     (MMA_MANY, None),
     (MMA_MIXED, None),
+    (TC_T1, None),
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], [0, 17]),      # sampled tokens at full size
