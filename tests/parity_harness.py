@@ -17,7 +17,7 @@ TOL = 1e-2            # max |gpu - oracle| <= TOL * RMS(oracle), per output tens
 NEAR_TIE = 1e-5
 
 
-class GpuRun:
+class DeviceRun:
     """Uploads a workload, runs it stage by stage, keeps host copies of every output."""
 
     def __init__(self, w: synth.MoeWorkload, act_mode=M.ACT_BF16, dense=None):

@@ -26,7 +26,7 @@ import mxfp4_routed_expert_04_b200 as M
 import oracle as O
 from mxfp4_routed_expert_04_b200 import synth
 
-from parity_harness import TOL, GpuRun, check_permutation, check_routing, expert_getter, max_rel_err
+from parity_harness import TOL, DeviceRun, check_permutation, check_routing, expert_getter, max_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +104,7 @@ def _unpack(packed):
 @pytest.fixture(scope="module", params=CASES, ids=lambda c: c[0].name)
 def case(request):
     w, sample = request.param
-    run = GpuRun(w, act_mode=M.ACT_MXFP4)
+    run = DeviceRun(w, act_mode=M.ACT_MXFP4)
     gpu = run.run_stages()
     gpu.update(_mxf4_operands(run, gpu))
     assert M.moe_device_status(run.layer.ws) == 0

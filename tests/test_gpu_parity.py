@@ -22,7 +22,7 @@ from mxfp4_routed_expert_04_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-from parity_harness import (TOL, GpuRun, check_permutation, check_routing, check_x_op_f16,  # noqa: E402
+from parity_harness import (TOL, DeviceRun, check_permutation, check_routing, check_x_op_f16,  # noqa: E402
                             expert_getter, max_rel_err)
 
 MEDIUM = synth.MoeWorkload("medium_ragged", T=70, H=640, I=384, E=6, k=3, I_shared=256, seed=77)
@@ -76,7 +76,7 @@ def _free():
 @pytest.fixture(scope="module", params=CASES, ids=lambda c: c[0].name)
 def case(request):
     w, sample = request.param
-    run = GpuRun(w)
+    run = DeviceRun(w)
     gpu = run.run_stages()
     yield w, sample, run, gpu
     del run
@@ -182,7 +182,7 @@ def test_zero_input_ties_go_to_lowest_index():
     w = _small()
     d = synth.dense_inputs(w)
     d["x"] = np.zeros_like(d["x"])
-    run = GpuRun(w, dense=d)
+    run = DeviceRun(w, dense=d)
     gpu = run.run_stages()
     assert np.all(gpu["logits"] == 0)
     np.testing.assert_array_equal(gpu["idx"], np.tile(np.arange(w.k), (w.T, 1)))
@@ -193,7 +193,7 @@ def test_zero_input_ties_go_to_lowest_index():
 
 def test_all_experts_selected():
     w = _small(T=3, E=4, k=4)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     gpu = run.run_stages()
     assert np.all(gpu["counts"] == 3)
     ref = O.moe_layer(run.dense, w.k, expert_getter(w))
@@ -203,7 +203,7 @@ def test_all_experts_selected():
 
 def test_single_token_single_expert():
     w = _small(T=1, E=1, k=1)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     gpu = run.run_stages()
     ref = O.moe_layer(run.dense, 1, expert_getter(w))
     assert gpu["w"][0, 0] == 1.0
@@ -213,7 +213,7 @@ def test_single_token_single_expert():
 
 def test_nan_scale_poisons_only_its_outputs():
     w = _small(T=4, E=2, k=1)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     gpu0 = run.run_stages()
     e = int(gpu0["idx"][0, 0])
     # E8M0 code 255 (NaN) in one scale of one gate row of expert e
@@ -233,7 +233,7 @@ def test_nan_scale_multi_token_kernels():
     of 512): a NaN down scale poisons one output column of its expert's rows, a
     NaN gate scale every output of them; the other expert stays finite."""
     w = synth.MoeWorkload("edge_mma", T=8, H=512, I=512, E=2, k=1, I_shared=128, seed=92)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     gpu0 = run.run_stages()
     counts = np.diff(gpu0["offsets"][:w.E + 1])
     e = int(np.argmax(counts))
@@ -261,7 +261,7 @@ def test_nan_scale_multi_token_kernels():
 def test_invalid_expert_index_sets_status_and_empties_routing():
     import mxfp4_routed_expert_04_b200 as M
     w = _small(T=4, E=8, k=2)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     L = run.layer
     M.moe_workspace_init(run.dims, L.ws)
     bad = torch.tensor([[0, 1], [2, 8], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
