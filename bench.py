@@ -205,6 +205,24 @@ def _dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), n
 
 
+def max_over_ranks(value, world, device):
+    """The largest of the ranks' values (every rank calls this in the same
+    order; world == 1: the value itself)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank, world, step_ms):
+    """Whole-job throughput of N replicas: every rank's tokens over the slowest
+    rank's step time."""
+    return tokens_per_rank * world / (step_ms * 1e-3)
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -308,11 +326,7 @@ def run_ours(args, w):
         soak(0.7)
     torch.cuda.synchronize()
     barrier()
-    step_ms = sum(ms) / len(ms)
-    if world > 1:
-        t = torch.tensor([step_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(sum(ms) / len(ms), world, "cuda")
 
     # dominant call alone: moe_expert_ffn on the routing of the captured step
     lw = layer.w      # the layer's weights (tiled scales for mxfp4 activations)
@@ -333,11 +347,7 @@ def run_ours(args, w):
         graph.replay()
         y_host.copy_(layer.y, non_blocking=True)
     timed(e2e_step, 3)
-    e2e_ms = statistics.mean(timed(e2e_step, args.steps))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(statistics.mean(timed(e2e_step, args.steps)), world, "cuda")
 
     if rank != 0:
         if world > 1:
@@ -377,10 +387,9 @@ def run_ours(args, w):
     roof = dict({"kernel": kernel}, **roof)
     roof.update({"bytes_per_launch": fb, "flops_per_launch": ff, "ms_per_launch": ffn_ms,
                  "traffic": _traffic(w.name)})
-    tokens = w.T * world
     out = {
         "metric": METRIC,
-        "value": tokens / (step_ms * 1e-3),
+        "value": job_tokens_per_s(w.T, world, step_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -401,7 +410,7 @@ def run_ours(args, w):
                   "tflops": layer_flops(w) / (step_ms * 1e-3) / 1e12},
         "roofline": roof,
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(w.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
                 "ms_per_step": e2e_ms},
         "clocks": clk.summary(),
