@@ -86,3 +86,18 @@ def test_rank_environment():
                 os.environ.pop(k, None)
             else:
                 os.environ[k] = v
+
+
+def test_reference_arm_line_on_rank_0(monkeypatch):
+    """The reference arm's JSON line (the fp64 oracle on the host cores)."""
+    b = _bench()
+    for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE"):
+        monkeypatch.delenv(k, raising=False)
+    from mxfp4_routed_expert_04_b200 import synth
+    args = types.SimpleNamespace(steps=2, warmup=3, act=None)
+    out = b.run_reference(args, synth.WORKLOADS["tiny"])
+    assert out["impl"] == "reference" and out["unit"] == "tokens/s" and out["value"] > 0
+    assert out["warmup"] == 3 and 1 <= out["steps"] <= 2 and out["n_gpus"] == 1
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["value"] == out["value"]
+    assert out["higher_is_better"] is True and out["metric"] == b.METRIC
