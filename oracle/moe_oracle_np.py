@@ -1,4 +1,9 @@
-"""fp64 CPU oracle of the routed MXFP4 MoE FFN layer.
+"""Independent numpy restatement of the fp64 oracle (cross-check of the C++ one).
+
+The oracle proper is the plain C++ implementation in oracle/moe_oracle.cpp;
+this module states the same definitions with numpy primitives (matmul,
+stable sorts) so that tests can check the two implementations against each
+other on random layers.
 
 TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
@@ -128,9 +133,9 @@ def topk_route(logits, k: int, near_tie: float = 1e-5):
     softmax over all E experts; the full denominator cancels, so this is
     exp(l_j - m) / sum_sel exp(l_i - m) with m the largest logit.
 
-    near-tie flag: a token is flagged when two adjacent logits among its k+1
-    largest differ by less than ``near_tie`` (the set boundary, or the order of
-    slots inside the set, then depends on rounding).
+    near-tie flag: a token is flagged when its k-th and (k+1)-th largest
+    logits differ by less than ``near_tie`` (the selected set then depends on
+    rounding).
 
     Returns idx [T, k] int32, w [T, k] float64, flagged [T] bool.
     """
@@ -146,8 +151,7 @@ def topk_route(logits, k: int, near_tie: float = 1e-5):
         idx[t] = sel
         ex = np.exp(logits[t, sel] - logits[t, sel[0]])
         w[t] = ex / ex.sum()
-        ranked = logits[t, order[:min(k + 1, E)]]
-        if len(ranked) > 1 and np.min(ranked[:-1] - ranked[1:]) < near_tie:
+        if k < E and logits[t, order[k - 1]] - logits[t, order[k]] < near_tie:
             flagged[t] = True
     return idx, w, flagged
 
@@ -271,7 +275,6 @@ def expert_ffn(x_rows, wg, wu, wd, act: str = "exact"):
     act: where the activations are rounded before a matmul
       "exact"  no rounding (decode: bf16 x is exact, h stays unrounded)
       "mxfp4"  x and h are MXFP4-quantised per 32-block (prefill, MXFP4 acts)
-      "bf16"   h is rounded to bf16 (prefill, bf16 acts)
     Returns (y [n, W], h [n, I]) with h as it entered the down projection.
 
     Reading: the expert activation is SwiGLU (silu(gate) * up), silu(z) =
@@ -288,8 +291,6 @@ def expert_ffn(x_rows, wg, wu, wd, act: str = "exact"):
     if act == "mxfp4":
         c, s = mxfp4_quantize(h)
         h = mxfp4_values(c, s)
-    elif act == "bf16":
-        h = bf16_to_f64(round_to_bf16_bits(h))
     return h @ wd.T, h
 
 

@@ -4,14 +4,12 @@ except where a test says it evaluates the oracle on the GPU's own routing
 choice for a near-tie token)."""
 from __future__ import annotations
 
-import functools
-
 import numpy as np
 import torch
 
 import mxfp4_routed_expert_04_b200 as M
 import oracle as O
-from mxfp4_routed_expert_04_b200 import synth
+import synth
 
 TOL = 1e-2            # max |gpu - oracle| <= TOL * RMS(oracle), per output tensor
 NEAR_TIE = 1e-5
@@ -59,17 +57,17 @@ class DeviceRun:
         return L.y.cpu().numpy().astype(np.float64)
 
 
-@functools.lru_cache(maxsize=None)
-def _expert_cached(w, e):
-    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
-    g = synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
-    u = synth.expert_matrix(w.seed, "up", e, Ng, Kg)
-    d = synth.expert_matrix(w.seed, "down", e, Nd, Kd)
-    return g + u + d
-
-
 def expert_getter(w):
-    return lambda e: _expert_cached(w, int(e))
+    """e -> the six MXFP4 arrays of expert e, regenerated from the seed on each
+    call (nothing cached: full-size layers hold gigabytes of experts)."""
+    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
+
+    def get(e):
+        e = int(e)
+        return (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
+                + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
+    return get
 
 
 def max_rel_err(got, want):
@@ -77,25 +75,47 @@ def max_rel_err(got, want):
     return float(np.max(np.abs(got - want))) / rms, rms
 
 
-def check_routing(gpu, ref_logits, k, near_tie=NEAR_TIE):
-    """Compare the GPU router against the oracle; returns the oracle's near-tie flags."""
-    idx, w, flagged = O.topk_route(ref_logits, k, near_tie)
+def check_routing(gpu, ref_logits, k, near_tie=NEAR_TIE, **route_kw):
+    """Compare the GPU router against the oracle; returns the tokens whose
+    selected SET is a near tie (the k-th and (k+1)-th selection scores, or the
+    last kept and first dropped group scores, closer than near_tie), where the
+    GPU's choice is checked for validity instead and used as the reference.
+
+    Elsewhere the set is bit-exact; the slot order is bit-exact too unless two
+    selected scores are a near tie (then it must be a valid order). Weights
+    are compared with the weights of the GPU's own selection, within a bound
+    derived from the logit error."""
+    idx, w, flags = O.route(ref_logits, k, near_tie=near_tie, **route_kw)
+    set_tie = (flags & (O.TIE_SET | O.TIE_GROUP)) != 0
+    order_tie = (flags & O.TIE_ORDER) != 0
     scale = max(1.0, float(np.abs(ref_logits).max()))
     assert np.max(np.abs(gpu["logits"] - ref_logits)) <= 1e-5 * scale * 10
-    ok = ~flagged
-    np.testing.assert_array_equal(gpu["idx"][ok], idx[ok])
-    # w_j = exp(l_j - m) / sum_sel exp(l - m): d log w_j / d l_i = [i == j] - w_i, so
-    # |log w_gpu - log w| <= 2 max_sel |l_gpu - l| (+ fp32 rounding of exp and divide)
-    dl = np.abs(np.take_along_axis(gpu["logits"] - ref_logits, idx.astype(np.int64), axis=1))
-    bound = w * (np.expm1(2 * dl.max(axis=1, keepdims=True)) + 1e-6) + 1e-9
-    assert np.all(np.abs(gpu["w"][ok] - w[ok]) <= bound[ok])
-    # near-tie tokens: the GPU choice must be a valid top-k within the tie window
-    for t in np.nonzero(flagged)[0]:
-        sel = ref_logits[t, gpu["idx"][t]]
-        kth = np.sort(ref_logits[t])[::-1][k - 1]
-        assert np.all(sel >= kth - near_tie) and len(set(gpu["idx"][t])) == k
-    np.testing.assert_allclose(gpu["w"].sum(axis=1), 1.0, atol=1e-6)
-    return flagged
+    ok = ~set_tie
+    g_idx = gpu["idx"]
+    np.testing.assert_array_equal(np.sort(g_idx[ok], axis=1), np.sort(idx[ok], axis=1))
+    exact = ok & ~order_tie
+    np.testing.assert_array_equal(g_idx[exact], idx[exact])
+    assert np.all([len(set(r)) == k for r in g_idx])
+    # selection scores of the oracle, to check the validity of tied choices
+    sel_score = ref_logits if route_kw.get("score_fn", O.SOFTMAX) == O.SOFTMAX else \
+        O.sigmoid(ref_logits) + (0.0 if route_kw.get("bias") is None else route_kw["bias"])
+    for t in np.nonzero(order_tie & ok)[0]:
+        s = sel_score[t, g_idx[t]]
+        assert np.all(np.diff(s) <= near_tie), (t, s)
+    for t in np.nonzero(set_tie & ((flags & O.TIE_GROUP) == 0))[0]:
+        s = sel_score[t, g_idx[t]]
+        kth = np.sort(sel_score[t])[::-1][k - 1]
+        assert np.all(s >= kth - near_tie)
+    # weights of the GPU's selection under the oracle's rule:
+    # d log w_j / d l_i = [i == j] c_j - w_i c_i with 0 <= c <= 1 (softmax:
+    # c = 1; sigmoid: c = 1 - s), so |log w_gpu - log w| <= 2 max_sel |dl|
+    # (+ fp32 rounding of exp and divide)
+    w_sel = O.route(ref_logits, k, near_tie=near_tie, idx_in=g_idx, **route_kw)[1]
+    dl = np.abs(np.take_along_axis(gpu["logits"] - ref_logits, g_idx.astype(np.int64), axis=1))
+    bound = np.abs(w_sel) * (np.expm1(2 * dl.max(axis=1, keepdims=True)) + 1e-6) + 1e-9
+    assert np.all(np.abs(gpu["w"] - w_sel) <= bound)
+    np.testing.assert_allclose(gpu["w"].sum(axis=1), route_kw.get("scale", 1.0), rtol=1e-6)
+    return set_tie
 
 
 def check_permutation(gpu, E):

@@ -24,7 +24,7 @@ import torch
 
 import mxfp4_routed_expert_04_b200 as M
 import oracle as O
-from mxfp4_routed_expert_04_b200 import synth
+import synth
 
 from parity_harness import TOL, DeviceRun, check_permutation, check_routing, expert_getter, max_rel_err
 
@@ -45,7 +45,10 @@ CASES = [
     (MEDIUM, None),
     (SKEWED, None),
     (ODD_H, None),
-    (synth.WORKLOADS["prefill4096"], [0, 1, 2047, 4095]),
+    # sampled tokens at full size: fixed ones plus, chosen from the GPU's routing,
+    # a token of the hottest expert in its last tile and one in the ragged last
+    # tile of an expert with several tiles
+    (synth.WORKLOADS["prefill4096"], [0, 1, 2047, 4095, "hot", "ragged"]),
 ]
 
 
@@ -113,10 +116,30 @@ def case(request):
     _free()
 
 
-def _rows_of(w, gpu, sample):
+def _sample_tokens(w, gpu, sample):
+    """Token ids of a sample; "hot" and "ragged" pick tokens from the GPU's
+    routing (validated separately against the oracle)."""
     if sample is None:
-        return np.arange(w.T * w.k)
-    return np.concatenate([gpu["slot_row"][t] for t in sample])
+        return np.arange(w.T)
+    counts = np.diff(gpu["offsets"])
+    tr = int(gpu["tile_rows"])
+    out = []
+    for s in sample:
+        if s == "hot":
+            e = int(np.argmax(counts))
+            out.append(int(gpu["row_token"][gpu["offsets"][e + 1] - 1]))
+        elif s == "ragged":
+            multi = np.nonzero((counts > tr) & (counts % tr != 0))[0]
+            assert len(multi), "no expert with a ragged last tile"
+            e = int(multi[np.argmax(counts[multi])])
+            out.append(int(gpu["row_token"][gpu["offsets"][e + 1] - 1]))
+        else:
+            out.append(int(s))
+    return np.unique(np.array(out))
+
+
+def _rows_of(w, gpu, sample):
+    return np.concatenate([gpu["slot_row"][t] for t in _sample_tokens(w, gpu, sample)])
 
 
 def test_routing_and_permutation(case):
@@ -190,7 +213,7 @@ def _oracle_rows(w, run, gpu, rows):
     """h64 and the reference h / y_perm of permuted rows `rows` (GPU permutation,
     validated by test_routing_and_permutation)."""
     get = expert_getter(w)
-    xq = O.mxfp4_values(*O.mxfp4_quantize(O.bf16_to_f64(run.dense["x"])))
+    x64 = O.bf16_to_f64(run.dense["x"])
     off = gpu["offsets"]
     ex = np.searchsorted(off, rows, side="right") - 1
     h_ref = np.zeros((len(rows), w.I))
@@ -200,14 +223,13 @@ def _oracle_rows(w, run, gpu, rows):
         sel = np.nonzero(ex == e)[0]
         rr = rows[sel]
         wg_q, wg_s, wu_q, wu_s, wd_q, wd_s = get(int(e))
-        x_rows = xq[gpu["row_token"][rr]]
-        g = x_rows @ O.mxfp4_dequant(wg_q, wg_s).T
-        u = x_rows @ O.mxfp4_dequant(wu_q, wu_s).T
-        h64 = O.silu(g) * u
+        # h before its quantisation (the oracle's expert with MXFP4 activations)
+        _, _, h64 = O.expert_ffn(x64[gpu["row_token"][rr]], wg_q, wg_s, wu_q, wu_s, wd_q, wd_s,
+                                 act="mxfp4", h_raw=True)
         href, t = _reference_h(h64, gpu["h_codes"][rr], gpu["h_scales"][rr])
         taken += t
         h_ref[sel] = href
-        y_ref[sel] = href @ O.mxfp4_dequant(wd_q, wd_s).T
+        y_ref[sel] = O.mxfp4_matmul(wd_q, wd_s, href)
     return h_ref, y_ref, taken
 
 
@@ -237,26 +259,39 @@ def test_layer_output(case, rows_ref):
     w, sample, run, gpu = case
     rows, h_ref, y_ref, taken = rows_ref
     d = run.dense
-    tokens = np.arange(w.T) if sample is None else np.array(sample)
-    # the oracle's routing weights; at near-tie tokens, the weights of the
-    # GPU's (validated) selection, whose rows y_ref holds
+    tokens = _sample_tokens(w, gpu, sample)
+    # the oracle's weights of the GPU's selection (equal to the oracle's own
+    # selection as a set wherever that is not a near tie:
+    # test_routing_and_permutation), whose rows y_ref holds
     logits = O.router_logits(d["x"][tokens], d["w_router"])
-    idx_o, _, flagged = O.topk_route(logits, w.k)
-    idx_use = np.where(flagged[:, None], gpu["idx"][tokens], idx_o)
-    np.testing.assert_array_equal(idx_use, gpu["idx"][tokens])
-    w_ref = O.selection_weights(logits, idx_use)
+    w_ref = O.selection_weights(logits, gpu["idx"][tokens])
     y_perm = np.zeros((w.T * w.k, w.W))
     y_perm[rows] = y_ref
     shared, _ = O.shared_expert(d["x"][tokens], d["ws_gate"], d["ws_up"], d["ws_down"], d["w_sgate"])
     ref = O.combine(y_perm, gpu["slot_row"][tokens], w_ref, shared)
     err, rms = max_rel_err(gpu["y"][tokens], ref)
     assert err <= TOL, (err, rms)
+    # the fused moe_layer path against the same reference
+    y_layer = run.run_layer()
+    err, rms = max_rel_err(y_layer[tokens], ref)
+    assert err <= TOL, ("moe_layer", err, rms)
 
 
 def test_fused_layer_matches_stages_bitwise(case):
     w, sample, run, gpu = case
     y = run.run_layer()
     np.testing.assert_array_equal(y, gpu["y"])
+
+
+def test_sample_covers_hot_and_ragged_tiles(case):
+    w, sample, run, gpu = case
+    if sample is None:
+        pytest.skip("every token is checked")
+    tokens = _sample_tokens(w, gpu, sample)
+    counts = np.diff(gpu["offsets"])
+    experts = set(gpu["idx"][tokens].ravel().tolist())
+    assert int(np.argmax(counts)) in experts
+    assert counts.max() > 2 * int(gpu["tile_rows"])
 
 
 def test_tile_scales_matches_the_tiled_layout():

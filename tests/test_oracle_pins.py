@@ -15,7 +15,7 @@ import scipy.special
 import torch
 
 import oracle as O
-from mxfp4_routed_expert_04_b200 import synth
+import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -206,12 +206,14 @@ def test_selection_weights_of_any_choice_equal_renormalised_full_softmax():
                                rtol=1e-13)
 
 
-def test_topk_near_tie_flag():
-    logits = np.array([[3.0, 2.0, 1.0, 1.0 - 5e-6, 0.0],
-                       [3.0, 2.0, 1.0, 0.5, 0.0],
-                       [3.0, 3.0 - 1e-6, 1.0, 0.5, 0.0]])
+def test_topk_near_tie_flags_split_set_boundary_from_slot_order():
+    logits = np.array([[3.0, 2.0, 1.0, 1.0 - 5e-6, 0.0],     # k-th vs (k+1)-th: the set
+                       [3.0, 2.0, 1.0, 0.5, 0.0],            # no tie
+                       [3.0, 3.0 - 1e-6, 1.0, 0.5, 0.0]])    # inside the set: the order only
     _, _, flagged = O.topk_route(logits, 3)
-    assert list(flagged) == [True, False, True]
+    assert list(flagged) == [True, False, False]
+    _, _, flags = O.route(logits, 3)
+    assert list(flags) == [O.TIE_SET, 0, O.TIE_ORDER]
 
 
 def test_router_logits_against_torch():
@@ -348,20 +350,130 @@ def test_latent_identity_reduces_to_plain_layer():
 
 
 def test_mxfp4_activation_mode_quantises_both_operands():
-    # with act="mxfp4" the layer equals the exact layer run on pre-quantised x,
-    # with h quantised before the down projection
+    # with act="mxfp4" the expert equals the exact expert run on pre-quantised x,
+    # with h quantised before the down projection (products in torch float64)
     w, d, ex, get = _tiny_layer_inputs(E=1, k=1, T=3)
-    wg = O.mxfp4_dequant(ex["wg_q"][0], ex["wg_s"][0])
-    wu = O.mxfp4_dequant(ex["wu_q"][0], ex["wu_s"][0])
-    wd = O.mxfp4_dequant(ex["wd_q"][0], ex["wd_s"][0])
+    wg = _torch_decode(ex["wg_q"][0], ex["wg_s"][0])
+    wu = _torch_decode(ex["wu_q"][0], ex["wu_s"][0])
+    wd = _torch_decode(ex["wd_q"][0], ex["wd_s"][0])
     x = O.bf16_to_f64(d["x"])
-    y, h = O.expert_ffn(x, wg, wu, wd, act="mxfp4")
-    xq = O.mxfp4_values(*O.mxfp4_quantize(x))
-    h_ref = O.silu(xq @ wg.T) * (xq @ wu.T)
+    y, h, h_raw = O.expert_ffn(x, *get(0), act="mxfp4", h_raw=True)
+    xq = torch.from_numpy(O.mxfp4_values(*O.mxfp4_quantize(x)))
+    h_ref = (torch.nn.functional.silu(xq @ wg.T) * (xq @ wu.T)).numpy()
+    np.testing.assert_allclose(h_raw, h_ref, rtol=1e-12, atol=1e-300)
     hq = O.mxfp4_values(*O.mxfp4_quantize(h_ref))
     np.testing.assert_array_equal(h, hq)
-    np.testing.assert_allclose(y, hq @ wd.T, rtol=1e-14)
-    assert not np.array_equal(xq, x)
+    np.testing.assert_allclose(y, (torch.from_numpy(hq) @ wd.T).numpy(), rtol=1e-12)
+    assert not np.array_equal(xq.numpy(), x)
+    # and act="exact" leaves both unrounded
+    y0, h0 = O.expert_ffn(x, *get(0))
+    xt = torch.from_numpy(x)
+    np.testing.assert_allclose(y0, _torch_dense_swiglu(x, wg.numpy(), wu.numpy(), wd.numpy()).numpy(),
+                               rtol=1e-11, atol=1e-12 * np.abs(y0).max())
+    np.testing.assert_allclose(h0, (torch.nn.functional.silu(xt @ wg.T) * (xt @ wu.T)).numpy(),
+                               rtol=1e-11, atol=1e-300)
+
+
+def test_mxfp4_matmul_against_torch():
+    rng = np.random.default_rng(12)
+    q = rng.integers(0, 256, (24, 48), dtype=np.uint8)
+    s = rng.integers(115, 135, (24, 3), dtype=np.uint8)
+    x = rng.standard_normal((5, 96))
+    want = (torch.from_numpy(x) @ _torch_decode(q, s).T).numpy()
+    np.testing.assert_allclose(O.mxfp4_matmul(q, s, x), want, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# latent layers (L != H)
+# ---------------------------------------------------------------------------
+
+def _latent_inputs(T=4, H=96, L=64, I=64, E=6, k=2, seed=21):
+    w = synth.MoeWorkload("lat", T=T, H=H, I=I, E=E, k=k, I_shared=32, L=L, seed=seed)
+    d = synth.dense_inputs(w)
+    ex = synth.expert_weights(w, range(E))
+    get = lambda e: tuple(ex[n][e] for n in ("wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s"))
+    return w, d, ex, get
+
+
+def _torch_latent_layer(d, ex, idx, wts, x_lat):
+    """The latent layer in torch float64 from a given routing and expert input x_lat [T, L]."""
+    bf = lambda a: torch.from_numpy(O.bf16_to_f64(d[a]))
+    xl = torch.as_tensor(x_lat, dtype=torch.float64)
+    T, k = idx.shape
+    acc = torch.zeros(T, xl.shape[1], dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            wg, wu, wd = (_torch_decode(ex[a][e], ex[b][e])
+                          for a, b in (("wg_q", "wg_s"), ("wu_q", "wu_s"), ("wd_q", "wd_s")))
+            h = torch.nn.functional.silu(xl[t] @ wg.T) * (xl[t] @ wu.T)
+            acc[t] += float(wts[t, j]) * (h @ wd.T)
+    x = bf("x")
+    shared = torch.sigmoid(x @ bf("w_sgate"))[:, None] * (
+        (torch.nn.functional.silu(x @ bf("ws_gate").T) * (x @ bf("ws_up").T)) @ bf("ws_down").T)
+    return (acc @ bf("w_lat_up").T + shared).numpy()
+
+
+def test_latent_down_against_torch_with_random_projection():
+    w, d, ex, get = _latent_inputs()
+    x = torch.from_numpy(O.bf16_to_f64(d["x"]))
+    prod = (x @ torch.from_numpy(O.bf16_to_f64(d["w_lat_down"])).T).numpy()
+    got = O.latent_down(d["x"], d["w_lat_down"])
+    # torch rounds float64 -> bfloat16 through float32; that double rounding can
+    # differ from one rounding only where the float32 value lands on a bf16 tie
+    want = torch.from_numpy(prod).float().to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    f32 = prod.astype(np.float32).view(np.uint32)
+    on_tie = (f32 & 0xFFFF) == 0x8000
+    assert np.array_equal(got[~on_tie], want[~on_tie])
+    assert got.shape == (w.T, w.L)
+
+
+def test_latent_layer_against_torch_and_rounding_point_matters():
+    w, d, ex, get = _latent_inputs()
+    out = O.moe_layer(d, w.k, get)
+    x_lat = O.bf16_to_f64(out["x_lat"])
+    ref = _torch_latent_layer(d, ex, out["idx"], out["w"], x_lat)
+    scale = np.abs(ref).max()
+    np.testing.assert_allclose(out["y"], ref, rtol=0, atol=1e-12 * scale)
+    # the bf16 rounding of x_lat changes the input bits, and an oracle without
+    # that rounding point would be far outside the bound above
+    prod = (torch.from_numpy(O.bf16_to_f64(d["x"]))
+            @ torch.from_numpy(O.bf16_to_f64(d["w_lat_down"])).T).numpy()
+    assert np.mean(x_lat != prod) > 0.9
+    unrounded = _torch_latent_layer(d, ex, out["idx"], out["w"], prod)
+    assert np.abs(unrounded - out["y"]).max() > 1e-6 * scale
+    # the routing sees the full-width x, not x_lat
+    np.testing.assert_array_equal(out["idx"], O.topk_route(O.router_logits(d["x"], d["w_router"]),
+                                                           w.k)[0])
+
+
+# ---------------------------------------------------------------------------
+# the C++ oracle against the independent numpy restatement
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["plain", "latent", "mxfp4", "skewed"])
+def test_cpp_oracle_matches_numpy_restatement(kind):
+    from oracle import moe_oracle_np as N
+    if kind == "latent":
+        w, d, ex, get = _latent_inputs(T=5, E=7, k=3, seed=31)
+    elif kind == "skewed":
+        w = synth.MoeWorkload("sk", T=9, H=128, I=64, E=16, k=4, I_shared=32, skew="hot64",
+                              seed=33)
+        d = synth.dense_inputs(w)
+        ex = synth.expert_weights(w, range(w.E))
+        get = lambda e: tuple(ex[n][e] for n in ("wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s"))
+    else:
+        w, d, ex, get = _tiny_layer_inputs(E=8, k=3, T=6, seed=32)
+    act = "mxfp4" if kind == "mxfp4" else "exact"
+    a = O.moe_layer(d, w.k, get, act=act)
+    b = N.moe_layer(d, w.k, get, act=act)
+    for name in ("idx", "counts", "offsets", "row_token", "row_slot", "slot_row", "flagged"):
+        np.testing.assert_array_equal(a[name], b[name], err_msg=name)
+    if kind == "latent":
+        np.testing.assert_array_equal(a["x_lat"], b["x_lat"])
+    for name in ("logits", "w", "y_perm", "shared", "gate", "y"):
+        scale = max(np.abs(b[name]).max(), 1e-300)
+        np.testing.assert_allclose(a[name], b[name], rtol=0, atol=1e-12 * scale, err_msg=name)
 
 
 def test_silu_sigmoid_match_torch_including_extremes():
