@@ -1,6 +1,7 @@
 """Benchmark of the routed MXFP4 MoE layer on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                [--extra NAMES | --no-extra]
 
 One step = one pass of the whole layer (route, permute, routed experts, gated
 shared expert, combine) over one batch of synthetic input, weights resident in
@@ -15,12 +16,18 @@ Activations: decode workloads keep bf16 activations (exact f16 operand of the
 grouped GEMVs); prefill workloads quantise them to MXFP4 for the tcgen05
 block-scaled GEMMs (``--act`` overrides).
 
+The printed line is the decode1 workload (T=1 H=8192 I=2048 E=512 k=10,
+I_shared=2048); by default the same measurement of decode32, latent16 and
+prefill4096 rides in the same line under ``workloads`` (``--extra`` /
+``--no-extra`` change that; extras time min(steps, 10) steps).
+
 Extra keys: ``roofline`` for the routed-expert call (moe_expert_ffn), timed
 alone in its own loop with the same flushing, against HBM bandwidth or, when
-its FLOPs take longer than its bytes at peak, the FP4 tensor peak; ``cpu_baseline`` (the fp64 oracle on the host cores, rank 0 only);
-``e2e`` (the same metric through moe_layer with the step's x copied in from
-pinned host memory and y copied back, inside the timed region); ``clocks``
-(nvidia-smi samples taken during the timed region).
+its FLOPs take longer than its bytes at peak, the FP4 tensor peak;
+``cpu_baseline`` (the C++ fp64 oracle on the host cores, all threads and one
+thread, rank 0 only); ``e2e`` (the same metric through moe_layer with the
+step's x copied in from pinned host memory and y copied back, inside the
+timed region); ``clocks`` (nvidia-smi samples taken during the timed region).
 """
 from __future__ import annotations
 
@@ -39,6 +46,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill MXF4 TFLOPS as % of roofline"
+DATA = ("synthetic, seeded: x ~ N(0,1) and bf16 weights ~ N(0,0.02) rounded to bf16; routed "
+        "MXFP4 codes uniform over 0..15, E8M0 scale codes uniform over 120..127; skewed routing "
+        "(decode32: 60% of tokens Zipf(1.1) over a hot set of 64; prefill: Zipf(1.1) over all "
+        "experts); random-init weights, no checkpoint")
+EXTRA_DEFAULT = ("decode32", "latent16", "prefill4096")
 EXPERT_BYTES_PER_ROW_BLOCK = 17   # 16 packed bytes + 1 E8M0 code per 32 weights
 
 
@@ -67,14 +79,25 @@ def layer_bytes(w, n_active):
 
 
 def ffn_bytes(w, n_active, act="bf16"):
-    """Algorithmic bytes of one moe_expert_ffn call: routed weights read once,
-    the activation operand read once, y_perm written once; with MXFP4
-    activations also h (codes + scales) written by gate/up and read by down."""
+    """Algorithmic bytes of one moe_expert_ffn call: the active experts' weights
+    read once, the activation operand read once (bf16 rows, or MXFP4 codes +
+    scales per (token, slot) row), and the routed output at its algorithmic
+    size T x W fp32. Intermediates this implementation chose (per-slot fp32
+    y_perm rows, h written by gate/up and read by down) are not counted; see
+    ffn_intermediate_bytes."""
     R = w.T * w.k
-    if act == "mxfp4":
-        return (n_active * expert_bytes(w) + w.T * w.W * 17 // 32 + R * w.W * 4
-                + 2 * R * w.I * 17 // 32)
-    return n_active * expert_bytes(w) + w.T * w.W * 2 + R * w.W * 4
+    x_op = R * w.W * 17 // 32 if act == "mxfp4" else w.T * w.W * 2
+    return n_active * expert_bytes(w) + x_op + w.T * w.W * 4
+
+
+def ffn_intermediate_bytes(w, act="bf16"):
+    """DRAM bytes of this implementation's intermediates per call (not in the
+    roofline): y_perm rows [T*k, W] fp32 written (the per-slot output beyond
+    the T x W counted above) and h written + read (fp32 in bf16 mode, MXFP4 in
+    MXFP4 mode)."""
+    R = w.T * w.k
+    h = 2 * R * w.I * (17 / 32 if act == "mxfp4" else 4)
+    return int((R - w.T) * w.W * 4 + h)
 
 
 def ffn_flops(w):
@@ -223,20 +246,18 @@ def job_tokens_per_s(tokens_per_rank, world, step_ms):
     return tokens_per_rank * world / (step_ms * 1e-3)
 
 
-def run_ours(args, w):
+def measure(args, w, steps, rank, local_rank, world, act=None):
+    """Time one workload on this rank (every rank runs the same collective
+    steps in the same order); returns the workload's result dict on rank 0,
+    None elsewhere."""
     import torch
     import torch.distributed as dist
 
     import mxfp4_routed_expert_04_b200 as M
-    from mxfp4_routed_expert_04_b200 import synth
+    import synth
 
-    rank, local_rank, world = _dist_env()
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = synth.to_device(w)
-    act = args.act or default_act(w)
+    act = act or default_act(w)
     dims = M.MoeDims.of(w, M.ACT_MXFP4 if act == "mxfp4" else M.ACT_BF16)
     layer = M.MoeLayer(dims, {k: v for k, v in dev.items() if k != "x"})
     x = dev["x"]
@@ -322,7 +343,7 @@ def run_ours(args, w):
 
     with ClockSampler(local_rank) as clk:
         soak(0.7)
-        ms = timed(graph.replay, args.steps)
+        ms = timed(graph.replay, steps)
         soak(0.7)
     torch.cuda.synchronize()
     barrier()
@@ -336,7 +357,7 @@ def run_ours(args, w):
                          lw["wg_s"], lw["wu_q"], lw["wu_s"], lw["wd_q"], lw["wd_s"],
                          layer.y_perm, layer.ws, stream)
     timed(ffn, 3)
-    ffn_ms = statistics.mean(timed(ffn, max(5, args.steps)))
+    ffn_ms = statistics.mean(timed(ffn, max(5, steps)))
 
     # end to end through moe_layer with host buffers
     x_host = x.cpu().pin_memory()
@@ -347,12 +368,10 @@ def run_ours(args, w):
         graph.replay()
         y_host.copy_(layer.y, non_blocking=True)
     timed(e2e_step, 3)
-    e2e_ms = max_over_ranks(statistics.mean(timed(e2e_step, args.steps)), world, "cuda")
-
+    e2e_ms = max_over_ranks(statistics.mean(timed(e2e_step, steps)), world, "cuda")
+    clocks = clk.summary()
+    del graph
     if rank != 0:
-        if world > 1:
-            del graph
-            dist.destroy_process_group()
         return None
     peak, peak_kind = _peaks()
     fb = ffn_bytes(w, n_active, act)
@@ -386,21 +405,18 @@ def run_ours(args, w):
                 "frac": hbm_gbs / peak, "peak_kind": peak_kind}
     roof = dict({"kernel": kernel}, **roof)
     roof.update({"bytes_per_launch": fb, "flops_per_launch": ff, "ms_per_launch": ffn_ms,
+                 "intermediate_bytes_per_launch": ffn_intermediate_bytes(w, act),
+                 "bytes_rule": "active experts' weights once + activation operand once + "
+                               "routed output T x W fp32",
                  "traffic": _traffic(w.name)})
     out = {
-        "metric": METRIC,
         "value": job_tokens_per_s(w.T, world, step_ms),
         "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
+        "steps": steps,
         "ms_per_step": step_ms,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
         "dtype": ("mxfp4 weights x mxfp4 activations (tcgen05 kind::mxf4), fp32 accumulate"
                   if act == "mxfp4" else "mxfp4 weights x f16 activations, fp32 accumulate"),
-        "data": "synthetic (seeded; BASELINE distributions)",
+        "data": DATA,
         "config": {"workload": workload_label(w), "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB write, then 512 MiB read of another "
                          "buffer, outside the events)",
@@ -409,103 +425,159 @@ def run_ours(args, w):
                   "hbm_frac": lb / (step_ms * 1e-3) / 1e9 / peak,
                   "tflops": layer_flops(w) / (step_ms * 1e-3) / 1e12},
         "roofline": roof,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * steps,
         "e2e": {"value": job_tokens_per_s(w.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 4,
                 "ms_per_step": e2e_ms},
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "clocks_note": "nvidia-smi every 200 ms over the timed steps plus 0.7 s of the same "
                        "flushed step on either side",
     }
-    if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, act=act)
-    if world > 1:
-        del graph
-        dist.destroy_process_group()
     return out
 
 
-def _oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+def run_ours(args, w):
+    """The headline workload plus the extra workloads, one after the other on
+    the same GPU(s); rank 0 returns the JSON line's dict."""
+    import gc
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+
+    rank, local_rank, world = _dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    head = measure(args, w, args.steps, rank, local_rank, world, args.act)
+    extras = {}
+    for name in args.extra:
+        if name == w.name:
+            continue
+        gc.collect()
+        torch.cuda.empty_cache()
+        r = measure(args, synth.WORKLOADS[name], min(args.steps, 10), rank, local_rank, world)
+        if r is not None:
+            extras[name] = r
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    out = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None}
+    out.update({k: v for k, v in head.items() if k not in out and k != "steps"})
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, act=args.act or default_act(w))
+    if extras:
+        out["workloads"] = extras
+    return out
+
+
+def _oracle_getter(w):
+    import synth
+    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
+    cache = {}
+
+    def get(e):
+        # regenerated from the seed once per expert (weights resident, as on the GPU)
+        if e not in cache:
+            cache[e] = (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
+                        + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
+                        + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
+        return cache[e]
+    return get
 
 
 def _oracle_token_pass(w, t, dense, getter, act="bf16"):
+    """One token of the batch through the oracle's whole layer (moe_o_layer)."""
     import oracle as O
     sub = dict(dense, x=dense["x"][t:t + 1])
     return O.moe_layer(sub, w.k, getter, act="mxfp4" if act == "mxfp4" else "exact")
 
 
-def cpu_baseline(w, budget_s: float = 20.0, act: str = "bf16"):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
-    tokens of the same batch, one at a time, until about ``budget_s`` seconds."""
-    from mxfp4_routed_expert_04_b200 import synth
+def _time_tokens(w, dense, getter, act, budget_s, first=0):
+    """Single-token layer passes until about budget_s seconds (at least one);
+    each token's experts are generated before its timed pass."""
+    import oracle as O
+    n, total = 0, 0.0
+    while n < w.T and (n == 0 or total < budget_s):
+        t = (first + n) % w.T
+        sel = O.topk_route(O.router_logits(dense["x"][t:t + 1], dense["w_router"]), w.k)[0]
+        for e in np.unique(sel):
+            getter(int(e))
+        t0 = time.perf_counter()
+        _oracle_token_pass(w, t, dense, getter, act)
+        total += time.perf_counter() - t0
+        n += 1
+    return n, total
+
+
+def cpu_baseline(w, budget_s: float = 12.0, act: str = "bf16"):
+    """The C++ fp64 oracle, as it stands, on a bounded sample of the workload:
+    whole tokens of the same batch through the whole layer, one at a time,
+    with all host threads and then with one thread. Weight generation is not
+    timed (the weights are resident, as on the GPU)."""
+    import oracle as O
+    import synth
 
     dense = synth.dense_inputs(w)
-    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
-
-    def getter(e):
-        return (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
-                + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
-                + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
-
-    t0 = time.perf_counter()
-    n = 0
-    while n < w.T and (n == 0 or time.perf_counter() - t0 < budget_s):
-        _oracle_token_pass(w, n, dense, getter, act)
-        n += 1
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{n} token(s) of {w.name}, each a full layer pass (routing, its k experts "
-                      f"decoded to fp64, shared expert, combine), {dt:.1f} s"}
+    getter = _oracle_getter(w)
+    O.set_threads(0)
+    cores = O.threads()
+    n, dt = _time_tokens(w, dense, getter, act, budget_s)
+    O.set_threads(1)
+    try:
+        n1, dt1 = _time_tokens(w, dense, getter, act, budget_s)
+    finally:
+        O.set_threads(0)
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "single_thread": {"value": n1 / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n1} token(s), {dt1:.1f} s"},
+            "sample": f"{n} token(s) of {w.name}, each a full layer pass of the C++ oracle "
+                      f"(routing, its k experts decoded to fp64, shared expert, combine) on "
+                      f"{cores} threads, {dt:.1f} s"}
 
 
 def run_reference(args, w):
-    """The reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    """The reference arm: the C++ fp64 oracle on the host cores (rank 0 only)."""
     rank, _, world = _dist_env()
     if rank != 0:
         return None
-    from mxfp4_routed_expert_04_b200 import synth
+    import oracle as O
+    import synth
 
     dense = synth.dense_inputs(w)
-    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
-
-    def getter(e):
-        return (synth.expert_matrix(w.seed, "gate", e, Ng, Kg)
-                + synth.expert_matrix(w.seed, "up", e, Ng, Kg)
-                + synth.expert_matrix(w.seed, "down", e, Nd, Kd))
-
+    getter = _oracle_getter(w)
     act = args.act or default_act(w)
+    O.set_threads(0)
+    cores = O.threads()
     # each step is one token's full layer pass; keep the whole run within a few minutes
     warmup = max(1, args.warmup)
-    t0 = time.perf_counter()
-    _oracle_token_pass(w, 0, dense, getter, act)       # the first warm-up pass also sizes the run
-    per = time.perf_counter() - t0
+    _, per = _time_tokens(w, dense, getter, act, 0.0)   # the first warm-up pass sizes the run
     for i in range(1, warmup):
-        _oracle_token_pass(w, i % w.T, dense, getter, act)
-    steps = max(1, min(args.steps, int(200.0 / max(per, 1e-3))))
+        _time_tokens(w, dense, getter, act, 0.0, first=i)
+    steps = max(1, min(args.steps, int(150.0 / max(per, 1e-3))))
     times = []
     for i in range(steps):
-        t0 = time.perf_counter()
-        _oracle_token_pass(w, i % w.T, dense, getter, act)
-        times.append(time.perf_counter() - t0)
+        _, dt = _time_tokens(w, dense, getter, act, 0.0, first=i)
+        times.append(dt)
     step = statistics.mean(times)
     v = 1.0 / step
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": warmup, "ms_per_step": step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; BASELINE distributions)",
+        "data": DATA,
         "config": {"workload": workload_label(w), "parallelism": "host cores, rank 0",
                    "act_mode": act, "step": "one token of the batch through the whole layer"},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _oracle_threads(),
-                         "kind": "oracle",
-                         "sample": f"{steps} single-token layer passes of {w.name} "
-                                   f"(steps capped so the run stays near 200 s)"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{steps} single-token layer passes of {w.name} through "
+                                   f"the C++ oracle on {cores} threads (steps capped so the "
+                                   f"run stays near 150 s; weight generation untimed)"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -518,6 +590,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode1")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated workloads measured after the headline one and "
+                         "reported under 'workloads' (default with the decode1 headline: "
+                         + ",".join(EXTRA_DEFAULT) + ")")
+    ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--act", choices=["bf16", "mxfp4"], default=None,
                     help="activation operand of the routed experts (default: mxfp4 for "
                          "prefill workloads, bf16 otherwise)")
@@ -529,12 +606,21 @@ def main():
     args = ap.parse_args()
     import dataclasses
 
-    from mxfp4_routed_expert_04_b200 import synth
+    import synth
     w = synth.WORKLOADS[args.workload]
     if args.experts:
         w = dataclasses.replace(w, E=args.experts, name=f"{w.name}-E{args.experts}")
     if args.tokens:
         w = dataclasses.replace(w, T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    if args.no_extra or args.experts or args.tokens:
+        args.extra = []
+    elif args.extra is None:
+        args.extra = list(EXTRA_DEFAULT) if args.workload == "decode1" else []
+    else:
+        args.extra = [n for n in args.extra.split(",") if n]
+        for n in args.extra:
+            if n not in synth.WORKLOADS:
+                ap.error(f"unknown workload {n}")
     res = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if res is not None:
         print(json.dumps(res), flush=True)

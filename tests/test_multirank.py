@@ -10,6 +10,8 @@ import datetime
 import importlib.util
 import os
 import socket
+import subprocess
+import sys
 import types
 
 import pytest
@@ -66,7 +68,7 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("LOCAL_RANK", "1")
     monkeypatch.setenv("WORLD_SIZE", "2")
-    from mxfp4_routed_expert_04_b200 import synth
+    import synth
     args = types.SimpleNamespace(steps=3, warmup=3, act=None)
     assert b.run_reference(args, synth.WORKLOADS["tiny"]) is None
 
@@ -93,7 +95,7 @@ def test_reference_arm_line_on_rank_0(monkeypatch):
     b = _bench()
     for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE"):
         monkeypatch.delenv(k, raising=False)
-    from mxfp4_routed_expert_04_b200 import synth
+    import synth
     args = types.SimpleNamespace(steps=2, warmup=3, act=None)
     out = b.run_reference(args, synth.WORKLOADS["tiny"])
     assert out["impl"] == "reference" and out["unit"] == "tokens/s" and out["value"] > 0
@@ -101,3 +103,23 @@ def test_reference_arm_line_on_rank_0(monkeypatch):
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["value"] == out["value"]
     assert out["higher_is_better"] is True and out["metric"] == b.METRIC
+
+
+def test_reference_arm_never_maps_the_product_library(repo_root):
+    """The reference arm (the oracle on the host) runs in a process that never
+    imports the product package nor maps its CUDA library."""
+    code = (
+        "import sys, types, bench, synth\n"
+        "args = types.SimpleNamespace(steps=1, warmup=1, act=None)\n"
+        "out = bench.run_reference(args, synth.WORKLOADS['tiny'])\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print('mapped' if 'libmoe_mxfp4' in maps else 'clean',\n"
+        "      'imported' if 'mxfp4_routed_expert_04_b200' in sys.modules else 'clean',\n"
+        "      'oracle' if 'libmoe_oracle' in maps else 'no-oracle')\n")
+    env = dict(os.environ)
+    for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE"):
+        env.pop(k, None)
+    res = subprocess.run([sys.executable, "-c", code], cwd=repo_root, env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr
+    assert res.stdout.split() == ["clean", "clean", "oracle"], res.stdout
