@@ -72,8 +72,10 @@ typedef enum {
 typedef enum {
   /* bf16 activations. x is carried exactly (as f16 times one power-of-two
    * scale per token row); h = silu(g)*u enters the down projection as f16
-   * with a power-of-two scale per group of 16 elements (relative rounding
-   * <= 2^-11). Decode path: a tensor-core grouped GEMV. */
+   * times a power of two per group (32 elements on the single-token path, a
+   * whole row on the multi-token TMA-ring path, 16 elements on the per-warp
+   * path): relative rounding <= 2^-11 for every element within 2^-28 of its
+   * group's largest magnitude. Decode path: grouped MXFP4 GEMVs. */
   MOE_ACT_BF16 = 0,
   /* MXFP4 activations: x rows and h are quantised to OCP MXFP4 (32-element
    * blocks, OCP MX v1.0 section 6.3 conversion) and the experts run as
@@ -112,12 +114,20 @@ size_t moe_x_op_size(const moe_dims* dims);
 moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream);
 
 /* Wait for `stream`, then copy the device status word into *host_status
- * (HOST pointer; 0 = no data error). Returns MOE_ERR_DEVICE_STATUS when the
- * word is non-zero, MOE_OK otherwise. Bit 0: an expert index outside [0, E);
- * bit 1: an expert repeated within one token. */
+ * (HOST pointer; 0 = no error). Returns MOE_ERR_DEVICE_STATUS when the word is
+ * non-zero, MOE_OK otherwise. Bits (OR-ed by every call that sees them, kept
+ * until moe_workspace_init clears them):
+ *   1 (bit 0)  an expert index outside [0, E) (the dispatch is emptied);
+ *   2 (bit 1)  an expert repeated within one token (the dispatch is emptied);
+ *   4 (bit 2)  a bounded device wait gave up: a kernel waited for a shared-
+ *              memory stage (a TMA or bulk copy, or another role of its CTA)
+ *              for about five seconds without it arriving; that kernel
+ *              stopped early, so the outputs of the call are incomplete. */
 moe_status moe_device_status(const void* ws, int32_t* host_status, void* stream);
 
 /* --- a1-a2: router ---------------------------------------------------------
+ * (rabbit README, model table row "MoE routing": softmax top-10 of 512; the
+ * lowest-index tie-break and the renormalisation are readings of it.)
  * logits[t, e] = sum_h x[t, h] Wr[e, h] (bf16 products are exact, fp32
  * accumulation), p = softmax(logits[t]) in fp32, the k largest logits are
  * selected (equal logits: lower expert index first; slots ordered by
@@ -132,20 +142,27 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
 
 /* --- router without a workspace ---------------------------------------------
  * (No counterpart in the pages: an interface convenience of this library.)
- * The same computation and outputs as moe_route, for callers that cannot
- * supply device scratch memory (a plug-in given only its input and output
- * tensors, or a runtime whose memory plan allows no extra buffer): the
- * split-K partial sums go to a 4 MiB device array built into the library.
- * Shapes needing more than 4 MiB of partials (S * T * E fp32 values, S the
- * K-split count of moe_route) return MOE_ERR_UNSUPPORTED_SHAPE. The array is
- * shared by every call on a device: calls that overlap on the GPU race on
- * it. The first call on each device looks up the array's address; make it
- * before capturing a stream into a CUDA graph. Nothing is allocated.
+ * The router step of moe_route (same inputs, outputs, selection and weight
+ * rule) for callers that cannot supply device scratch memory: a plug-in given
+ * only its input and output tensors, or a runtime whose memory plan allows no
+ * extra buffer. Its split-K partial sums go to a 4 MiB device array built
+ * into the library. It does not run moe_route's logit kernels: its logits
+ * come from a split-K CUDA-core GEMV summed in another order, so they agree
+ * with moe_route's to fp32 rounding; the selected experts are the same
+ * except at near ties of two router logits (every call on the same inputs
+ * gives the same bits). Shapes needing more than 4 MiB of partials (S * T * E
+ * fp32 values, S = its K-split count, up to 16) return
+ * MOE_ERR_UNSUPPORTED_SHAPE before anything is enqueued. The array is shared
+ * by every call on a device: calls that overlap on the GPU race on it. The
+ * first call on each device looks up the array's address; make it before
+ * capturing a stream into a CUDA graph. Nothing is allocated.
  */
 moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
                              int32_t* topk_idx, float* topk_w, float* logits, void* stream);
 
 /* --- a3-a4: permutation ----------------------------------------------------
+ * (The pages do not describe the dispatch; grouping the routed (token, slot)
+ * pairs by expert is what running each expert once on its own tokens needs.)
  * Groups the T*k (token, slot) pairs by expert: counts[e] pairs per expert,
  * offsets = exclusive prefix sum (E+1 entries), permuted rows ordered by
  * expert and, inside an expert, by ascending token; expert_list[0] = number
@@ -183,6 +200,9 @@ moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint
                        void* ws, size_t ws_bytes, void* stream);
 
 /* --- a5-a7: routed experts (the "expert matmul") ----------------------------
+ * (rabbit README: the "expert matmul" phase of its decode-step breakdown, on
+ * routed experts read as OCP MXFP4, model table row "native quantization
+ * read"; the SwiGLU activation is a reading.)
  * For every permuted row r of expert e (offsets[e] <= r < offsets[e+1]) and
  * its token t = row_token[r]:
  *   y_perm[r] = Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) )      [W] fp32
@@ -225,6 +245,8 @@ typedef struct {
 moe_status moe_mxf4_layout_of(const moe_dims* dims, moe_mxf4_layout* out);
 
 /* --- a8-a9 (+a10 up): shared expert and combine ------------------------------
+ * (rabbit README, model table row "MoE routing": "+ gated shared expert"; the
+ * per-token sigmoid gate is a reading.)
  *   s_t = sigmoid(w_sgate . x_t) * Ws_down (silu(Ws_gate x_t) * (Ws_up x_t))
  *   y_t = [W_lu] (sum_j topk_w[t, j] * y_perm[slot_row[t, j]]) + s_t
  * W_lu is applied only for latent layers (w_lat_up non-NULL iff L > 0).
@@ -238,10 +260,32 @@ moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t*
                        void* ws, size_t ws_bytes, void* stream);
 
 /* --- a10: latent down-projection (latent layers only) ------------------------
+ * ("Ran Moonshot's 2.8T-parameter Kimi K3 on a GPU-less mini-PC", architecture
+ * paragraph: Stable LatentMoE, routed experts in a narrower latent width; the
+ * dense bf16 projection and the bf16 rounding point are readings.)
  * x_lat[t] = bf16_rne( W_ld x_t ),  W_ld [L, H] bf16, x_lat [T, L] bf16 (out).
  */
 moe_status moe_latent_down(const moe_dims* dims, const uint16_t* x, const uint16_t* w_lat_down,
                            uint16_t* x_lat, void* ws, size_t ws_bytes, void* stream);
+
+/* --- diagnostics: the bounded device waits ----------------------------------
+ * (No counterpart in the pages: a check of this library's failure handling.)
+ * Every stage-ring kernel waits for its shared-memory stages with a bounded
+ * wait; when a stage's bytes do not arrive in time it raises an abort flag,
+ * every role of the CTA stops, and bit 2 (value 4) of the status word is set
+ * (see moe_device_status). This call runs one CTA that uses the same waits
+ * on one 512-byte stage, with `limit` tries (1..4096; about 20 us each at
+ * most) instead of the multi-second default:
+ *   deliver != 0: the stage is filled by a bulk copy from `src` (a 16-byte
+ *     aligned DEVICE buffer of 512 bytes); the waits succeed and *status is
+ *     left unchanged;
+ *   deliver == 0: nothing delivers the stage's bytes; both waits give up, the
+ *     kernel returns and ORs 4 into *status (a DEVICE int32).
+ * No copy is in flight when a wait gives up, so the context stays usable.
+ * Enqueued on `stream`; invalid arguments return an error and enqueue nothing.
+ */
+moe_status moe_selftest_bounded_wait(int32_t* status, const void* src, int deliver,
+                                     uint32_t limit, void* stream);
 
 /* --- the whole layer ---------------------------------------------------------
  * Every buffer of the calls above in one struct; moe_layer enqueues the same

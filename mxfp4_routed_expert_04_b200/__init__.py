@@ -17,8 +17,13 @@ __all__ = [
     "MoeError", "MoeDims", "MoeLayerArgs", "ACT_BF16", "ACT_MXFP4", "library_path",
     "moe_status_string", "moe_workspace_size", "moe_x_op_size", "moe_workspace_init",
     "moe_device_status", "moe_route", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
-    "moe_latent_down", "moe_layer", "moe_mxf4_layout_of", "moe_tile_scales", "MoeLayer",
+    "moe_latent_down", "moe_layer", "moe_mxf4_layout_of", "moe_tile_scales",
+    "moe_selftest_bounded_wait", "STATUS_BAD_EXPERT", "STATUS_REPEATED_EXPERT",
+    "STATUS_WAIT_TIMEOUT", "MoeLayer",
 ]
+
+# bits of the device status word (moe_device_status)
+STATUS_BAD_EXPERT, STATUS_REPEATED_EXPERT, STATUS_WAIT_TIMEOUT = 1, 2, 4
 
 ACT_BF16 = 0
 ACT_MXFP4 = 1
@@ -83,6 +88,7 @@ _sigs = {
     "moe_layer": [_D, ctypes.POINTER(MoeLayerArgs), _P, _Z, _P],
     "moe_mxf4_layout_of": [_D, ctypes.c_void_p],
     "moe_tile_scales": [_P, ctypes.c_int64, ctypes.c_int32, _P, _P],
+    "moe_selftest_bounded_wait": [_P, _P, ctypes.c_int, ctypes.c_uint32, _P],
 }
 for _n, _a in _sigs.items():
     getattr(_lib, _n).argtypes = _a
@@ -146,6 +152,14 @@ def moe_mxf4_layout_of(dims) -> MoeMxf4Layout:
 def moe_tile_scales(src, rows: int, K: int, dst, stream=None):
     """Canonical E8M0 scales [rows, K/32] -> the tiled layout of the tensor-core path."""
     _check(_lib.moe_tile_scales(_ptr(src), int(rows), int(K), _ptr(dst), _stream(stream)))
+
+
+def moe_selftest_bounded_wait(status, src, deliver: bool, limit: int, stream=None):
+    """One CTA waits (bounded, ``limit`` tries) for a stage that a bulk copy
+    from ``src`` fills (deliver) or that nothing fills; a timeout ORs
+    STATUS_WAIT_TIMEOUT into the device int32 ``status``."""
+    _check(_lib.moe_selftest_bounded_wait(_ptr(status), _ptr(src), 1 if deliver else 0,
+                                          int(limit), _stream(stream)))
 
 
 def moe_workspace_init(dims, ws, stream=None):

@@ -318,12 +318,12 @@ MOE_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 }
 
 // Bounded wait for phase `parity` of `bar`: false when it did not complete
-// within the iteration limit (the caller reports it and leaves). Each
-// try_wait may suspend the thread for up to 20 us until the phase completes,
-// so a waiting warp does not spin on the issue slots; the bound is about 5 s.
-MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// within `limit` tries (the caller reports it and leaves). Each try_wait may
+// suspend the thread for up to 20 us until the phase completes, so a waiting
+// warp does not spin on the issue slots; the default bound is about 5 s.
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = 1u << 18) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0; it < (1u << 18); ++it) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"

@@ -7,8 +7,14 @@
 // allowed or would break a memory plan fixed in advance. This entry point
 // needs nothing beyond its inputs and outputs: the router's split-K partial
 // sums live in the file-scope device array below instead of the caller's
-// workspace. It enqueues the same two kernels as moe_route, with the same
-// split of K, so its results are identical to moe_route's.
+// workspace. It computes what moe_route computes, but not with the same
+// kernels: the logits come from a split-K CUDA-core GEMV of its own
+// (k_dense_gemv, K split as router_splits below decides), and only the top-k
+// launch (k_topk) is shared with moe_route. moe_route sums the logits on
+// other kernels (a tensor-core row GEMV for one token, the tcgen05 GEMM for
+// more), in another order, so the two agree to fp32 rounding of the logits:
+// the selected experts are the same except where two router logits are a
+// near tie, and the weights agree to the same rounding.
 //
 // Limits and rules:
 // * the scratch holds kNoAllocScratchFloats fp32 values (4 MiB); shapes whose
@@ -58,9 +64,10 @@ moe_status scratch_address(float** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// K splits of the router GEMV: the rule moe_route uses (enough warps to cover
-// 148 SMs at about 4 per SM, whole 32-element steps, at least 8 per split, at
-// most 16 splits), so both entry points sum the same partials in the same order.
+// K splits of this entry point's router GEMV: enough warps to cover 148 SMs at
+// about 4 per SM, whole 32-element steps, at least 8 per split, at most 16
+// splits. The split-K partials are summed by k_topk in split order, so every
+// call on the same inputs gives the same bits.
 int router_splits(int N, int T, int K) {
   const long warps = (long)((N + 15) / 16) * ((T + 31) / 32);
   const int ksteps = K / 32;

@@ -136,10 +136,12 @@ MOE_DEV void mbar_arrive(uint64_t* bar) {
 
 // Bounded wait on phase `parity` of `bar` that also gives up as soon as
 // another role of the CTA has raised `*abort`. Returns false when it gave up
-// (raising `*abort` itself on a timeout of about four seconds).
-MOE_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// (raising `*abort` itself after `limit` tries: about four seconds by
+// default).
+MOE_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                           uint32_t limit = 1u << 22) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0; it < (1u << 22); ++it) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"

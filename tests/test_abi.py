@@ -140,3 +140,12 @@ def test_tile_scales_rejects_bad_shapes(rows, K):
 def test_tile_scales_rejects_null_and_misaligned():
     assert M._lib.moe_tile_scales(None, 128, 128, 1 << 20, None) == 1
     assert M._lib.moe_tile_scales((1 << 20) + 4, 128, 128, 1 << 20, None) == 3
+
+
+def test_selftest_bounded_wait_validates_arguments():
+    lib = M._lib
+    assert lib.moe_selftest_bounded_wait(None, None, 0, 16, None) == 1          # no status word
+    assert lib.moe_selftest_bounded_wait(FAKE, None, 1, 16, None) == 3          # deliver, no source
+    assert lib.moe_selftest_bounded_wait(FAKE, FAKE + 4, 1, 16, None) == 3      # misaligned source
+    assert lib.moe_selftest_bounded_wait(FAKE, None, 0, 0, None) == 1           # limit 0
+    assert lib.moe_selftest_bounded_wait(FAKE, None, 0, 5000, None) == 1        # limit too large
