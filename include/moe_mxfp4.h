@@ -83,6 +83,20 @@ typedef enum {
   MOE_ACT_MXFP4 = 1
 } moe_act_mode;
 
+/* How the router scores experts (rabbit README, model table row "MoE
+ * routing": "softmax top-10 of 512" for Qwen3.8-Max, "noaux_tc sigmoid" for
+ * GLM-5.2, "grouped routing" for Kimi Linear; the pages name the last two
+ * only, so their definitions here are readings). */
+typedef enum {
+  /* softmax: experts ranked by logit; w = the softmax renormalised over the
+   * selected experts (times route_scale). */
+  MOE_SCORE_SOFTMAX = 0,
+  /* sigmoid: s_e = sigmoid(logit_e); experts ranked by s_e + e_bias[e] (the
+   * bias steers the selection only; NULL = 0); w_j = s_j / sum of the
+   * selected s (times route_scale). */
+  MOE_SCORE_SIGMOID = 1
+} moe_score_fn;
+
 typedef struct {
   int32_t T;         /* tokens */
   int32_t H;         /* hidden width */
@@ -92,6 +106,18 @@ typedef struct {
   int32_t I_shared;  /* shared-expert intermediate width */
   int32_t L;         /* latent width of the routed experts; 0 = none (W = H) */
   int32_t act_mode;  /* moe_act_mode */
+  /* router variant (all zero: the softmax router) */
+  int32_t score_fn;     /* moe_score_fn */
+  int32_t n_group;      /* 0 or 1: no groups. 2..64: group-limited selection: the
+                           E experts form n_group groups of E / n_group
+                           consecutive ids; a group scores the sum of its two
+                           largest expert scores (the softmax probability, or
+                           the biased sigmoid score); the topk_group best groups
+                           are kept (ties: lower group); top-k among their
+                           experts. Needs E % n_group == 0 and
+                           topk_group * E / n_group >= k. */
+  int32_t topk_group;   /* groups kept, 1..n_group (ignored without groups) */
+  float route_scale;    /* multiplies the routing weights; 0 means 1 */
 } moe_dims;
 
 /* One-line description of a status code (static storage). */
@@ -139,6 +165,15 @@ moe_status moe_device_status(const void* ws, int32_t* host_status, void* stream)
 moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
                      int32_t* topk_idx, float* topk_w, float* logits,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* moe_route with the router's per-expert selection bias e_bias [E] fp32
+ * (device; used by MOE_SCORE_SIGMOID, ignored by the softmax router; NULL =
+ * no bias). The selection and weight rules are those of dims->score_fn,
+ * n_group, topk_group and route_scale (see moe_dims). moe_route is this call
+ * with e_bias = NULL. */
+moe_status moe_route_biased(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
+                            const float* e_bias, int32_t* topk_idx, float* topk_w, float* logits,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /* --- router without a workspace ---------------------------------------------
  * (No counterpart in the pages: an interface convenience of this library.)
@@ -311,6 +346,7 @@ typedef struct {
   void* x_op;          /* moe_x_op_size() bytes */
   float* y_perm;       /* [T*k, W] */
   float* y;            /* [T, H] */
+  const float* e_bias; /* [E] router selection bias (MOE_SCORE_SIGMOID), or NULL */
 } moe_layer_args;
 
 moe_status moe_layer(const moe_dims* dims, const moe_layer_args* args,

@@ -16,10 +16,10 @@ import torch
 __all__ = [
     "MoeError", "MoeDims", "MoeLayerArgs", "ACT_BF16", "ACT_MXFP4", "library_path",
     "moe_status_string", "moe_workspace_size", "moe_x_op_size", "moe_workspace_init",
-    "moe_device_status", "moe_route", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
+    "moe_device_status", "moe_route", "moe_route_biased", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_latent_down", "moe_layer", "moe_mxf4_layout_of", "moe_tile_scales",
     "moe_selftest_bounded_wait", "STATUS_BAD_EXPERT", "STATUS_REPEATED_EXPERT",
-    "STATUS_WAIT_TIMEOUT", "MoeLayer",
+    "STATUS_WAIT_TIMEOUT", "SCORE_SOFTMAX", "SCORE_SIGMOID", "MoeLayer",
 ]
 
 # bits of the device status word (moe_device_status)
@@ -47,13 +47,23 @@ def _load():
 _lib = _load()
 
 
+SCORE_SOFTMAX = 0
+SCORE_SIGMOID = 1
+
+
 class MoeDims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("T", "H", "I", "E", "k", "I_shared", "L", "act_mode")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "H", "I", "E", "k", "I_shared", "L", "act_mode",
+                                              "score_fn", "n_group", "topk_group")] + \
+               [("route_scale", ctypes.c_float)]
 
     @classmethod
     def of(cls, w, act_mode: int = ACT_BF16) -> "MoeDims":
-        """Dims of a workload (anything with T, H, I, E, k, I_shared, L)."""
-        return cls(w.T, w.H, w.I, w.E, w.k, w.I_shared, w.L, act_mode)
+        """Dims of a workload (anything with T, H, I, E, k, I_shared, L and,
+        optionally, the router variant: score_fn, n_group, topk_group,
+        route_scale)."""
+        return cls(w.T, w.H, w.I, w.E, w.k, w.I_shared, w.L, act_mode,
+                   getattr(w, "score_fn", 0), getattr(w, "n_group", 0),
+                   getattr(w, "topk_group", 0), getattr(w, "route_scale", 1.0))
 
 
 _P = ctypes.c_void_p
@@ -64,7 +74,7 @@ class MoeLayerArgs(ctypes.Structure):
         "x", "w_router", "wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s", "w_sgate",
         "ws_gate", "ws_up", "ws_down", "w_lat_down", "w_lat_up", "topk_idx", "topk_w",
         "counts", "offsets", "expert_list", "row_token", "row_slot", "slot_row", "x_lat", "x_op",
-        "y_perm", "y")]
+        "y_perm", "y", "e_bias")]
 
 
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -80,6 +90,7 @@ _sigs = {
     "moe_workspace_init": [_D, _P, _Z, _P],
     "moe_device_status": [_P, ctypes.POINTER(ctypes.c_int32), _P],
     "moe_route": [_D, _P, _P, _P, _P, _P, _P, _Z, _P],
+    "moe_route_biased": [_D, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_route_noalloc": [_D, _P, _P, _P, _P, _P, _P],
     "moe_permute": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
     "moe_expert_ffn": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P],
@@ -185,6 +196,12 @@ def moe_route(dims, x, w_router, topk_idx, topk_w, logits, ws, stream=None):
                           _ptr(topk_w), _ptr(logits), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
+def moe_route_biased(dims, x, w_router, e_bias, topk_idx, topk_w, logits, ws, stream=None):
+    _check(_lib.moe_route_biased(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(e_bias),
+                                 _ptr(topk_idx), _ptr(topk_w), _ptr(logits), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)))
+
+
 def moe_route_noalloc(dims, x, w_router, topk_idx, topk_w, logits, stream=None):
     """moe_route without a workspace (partials in the library's static device array)."""
     _check(_lib.moe_route_noalloc(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(topk_idx),
@@ -232,7 +249,8 @@ class MoeLayer:
 
     ``weights``: dict of device tensors (x excluded) named like the C ABI
     (w_router, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, w_sgate, ws_gate, ws_up,
-    ws_down and, for latent layers, w_lat_down, w_lat_up); bf16 tensors as
+    ws_down and, for latent layers, w_lat_down, w_lat_up; optionally e_bias,
+    the router's fp32 selection bias [E]); bf16 tensors as
     int16/uint16 bit patterns or torch.bfloat16. Scales in the canonical
     layout; for ACT_MXFP4 the layer keeps tiled copies (moe_tile_scales) in
     ``self.w``, the weights every call uses.
@@ -284,7 +302,7 @@ class MoeLayer:
             expert_list=_ptr(self.expert_list),
             row_token=_ptr(self.row_token), row_slot=_ptr(self.row_slot),
             slot_row=_ptr(self.slot_row), x_lat=_ptr(self.x_lat), x_op=_ptr(self.x_op),
-            y_perm=_ptr(self.y_perm), y=_ptr(self.y))
+            y_perm=_ptr(self.y_perm), y=_ptr(self.y), e_bias=g("e_bias"))
 
     def __call__(self, x, stream=None):
         """Whole layer (moe_layer); returns the fp32 output tensor [T, H]."""
@@ -295,7 +313,8 @@ class MoeLayer:
         """The same layer through the four step calls (route, [latent], permute,
         expert_ffn, combine); also fills self.logits."""
         d, w = self.dims, self.w
-        moe_route(d, x, w["w_router"], self.topk_idx, self.topk_w, self.logits, self.ws, stream)
+        moe_route_biased(d, x, w["w_router"], w.get("e_bias"), self.topk_idx, self.topk_w,
+                         self.logits, self.ws, stream)
         xin = x
         if d.L:
             moe_latent_down(d, x, w["w_lat_down"], self.x_lat, self.ws, stream)

@@ -63,6 +63,7 @@ int tc_splits(long units, int K, size_t split_bytes) {
 
 struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
+  moe::RouteCfg rc;          // router variant (bias pointer filled per call)
   int S_router, S_sgu, S_sd, S_ld, S_lu;
   int Nt;                    // token tile of the tcgen05 bf16 GEMMs
   bool swiglu_tc;            // shared gate/up GEMM applies SwiGLU in its epilogue
@@ -92,6 +93,22 @@ moe_status check_dims(const moe_dims* d) {
   }
   if ((long)d->T * d->k > (1L << 24))
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T*k=%ld above 2^24", (long)d->T * d->k);
+  if (d->score_fn != MOE_SCORE_SOFTMAX && d->score_fn != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "score_fn %d is not a moe_score_fn", d->score_fn);
+  if (!(d->route_scale >= 0.0f) || d->route_scale > 1e30f)
+    return fail(MOE_ERR_INVALID_ARG, "route_scale must be finite and >= 0");
+  if (d->n_group > 1) {
+    if (d->n_group > moe::kMaxGroups || d->E % d->n_group != 0)
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_group=%d must divide E=%d and be <= %d", d->n_group,
+                  d->E, moe::kMaxGroups);
+    if (d->topk_group < 1 || d->topk_group > d->n_group ||
+        (long)d->topk_group * (d->E / d->n_group) < d->k)
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                  "topk_group=%d: needs 1 <= topk_group <= n_group and topk_group*E/n_group >= k",
+                  d->topk_group);
+  } else if (d->n_group < 0) {
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_group=%d is negative", d->n_group);
+  }
   return MOE_OK;
 }
 
@@ -102,6 +119,11 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
   p.W = d->L ? d->L : d->H;
   p.R = d->T * d->k;
   p.mode = d->act_mode;
+  p.rc.bias = nullptr;
+  p.rc.score_fn = d->score_fn;
+  p.rc.n_group = d->n_group > 1 ? d->n_group : 1;
+  p.rc.topk_group = d->n_group > 1 ? d->topk_group : 1;
+  p.rc.scale = d->route_scale == 0.0f ? 1.0f : d->route_scale;
   p.Nt = tc_tile_tokens(p.T);
   p.swiglu_tc = p.T >= kDenseSwiGLUTokens;
   p.rows = rows_path_for(p.T, p.H, p.Is);
@@ -443,10 +465,13 @@ moe_status round_latent(const Plan& p, const float* part, int ld, uint16_t* x_la
 // (fuse: one token in bf16 mode, the top-k launch also writes the dispatch
 // and the activation operand; moe_permute is then skipped)
 moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
-                    int32_t* idx, float* w, float* logits, void* ws, cudaStream_t st,
-                    const uint16_t* w_sgate = nullptr, const uint16_t* w_ld = nullptr,
-                    uint16_t* x_lat = nullptr, const moe::TopkFuse* fuse = nullptr) {
+                    const float* e_bias, int32_t* idx, float* w, float* logits, void* ws,
+                    cudaStream_t st, const uint16_t* w_sgate = nullptr,
+                    const uint16_t* w_ld = nullptr, uint16_t* x_lat = nullptr,
+                    const moe::TopkFuse* fuse = nullptr) {
   const moe::TopkFuse tf = fuse ? *fuse : moe::TopkFuse{};
+  moe::RouteCfg rc = p.rc;
+  rc.bias = e_bias;
   float* part = at<float>(ws, p.off_router);
   moe_status s;
   if (p.rows) {
@@ -459,7 +484,7 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
     r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
     if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
     launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
-               p.E, p.k, idx, w, logits, (float*)nullptr, tf);
+               p.E, p.k, idx, w, logits, (float*)nullptr, tf, rc);
     if ((s = launched("top-k")) != MOE_OK) return s;
     return w_ld ? round_latent(p, at<float>(ws, p.off_ld), p.L, x_lat, st) : MOE_OK;
   }
@@ -479,7 +504,7 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
   g.seg_rows[0] = p.E; g.seg_rows[1] = w_sgate ? 1 : 0; g.seg_rows[2] = w_ld ? p.L : 0; g.ld = ld;
   if ((s = launch_bf16_gemm(ds, g, st, "router gemm (tcgen05)")) != MOE_OK) return s;
   launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, p.S_router, p.T, p.E,
-             ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr, tf);
+             ld, p.k, idx, w, logits, w_sgate ? at<float>(ws, p.off_gl) : (float*)nullptr, tf, rc);
   if ((s = launched("top-k")) != MOE_OK) return s;
   return w_ld ? round_latent(p, part + lat_col, ld, x_lat, st) : MOE_OK;
 }
@@ -917,7 +942,22 @@ moe_status moe_route(const moe_dims* dims, const uint16_t* x, const uint16_t* w_
   if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
   DeviceState* ds;
   if ((s = device_state(&ds)) != MOE_OK) return s;
-  return do_route(p, *ds, x, w_router, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
+  return do_route(p, *ds, x, w_router, nullptr, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_route_biased(const moe_dims* dims, const uint16_t* x, const uint16_t* w_router,
+                            const float* e_bias, int32_t* topk_idx, float* topk_w, float* logits,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  CHECK_PTR(x); CHECK_PTR(w_router); CHECK_PTR(topk_idx); CHECK_PTR(topk_w);
+  if (e_bias && !aligned16(e_bias)) return fail(MOE_ERR_ALIGNMENT, "e_bias not 16-byte aligned");
+  if (logits && !aligned16(logits)) return fail(MOE_ERR_ALIGNMENT, "logits not 16-byte aligned");
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  return do_route(p, *ds, x, w_router, e_bias, topk_idx, topk_w, logits, ws, (cudaStream_t)stream);
 }
 
 moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint16_t* x_in,
@@ -1026,7 +1066,8 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
     tf.x = a->x; tf.W = p.W;
     tf.x16 = static_cast<__half*>(a->x_op); tf.xscale = at<float>(a->x_op, p.xop_scale_off);
   }
-  if ((s = do_route(p, *ds, a->x, a->w_router, a->topk_idx, a->topk_w, nullptr, ws, st,
+  if (a->e_bias && !aligned16(a->e_bias)) return fail(MOE_ERR_ALIGNMENT, "e_bias not 16-byte aligned");
+  if ((s = do_route(p, *ds, a->x, a->w_router, a->e_bias, a->topk_idx, a->topk_w, nullptr, ws, st,
                     sgate_with_router ? a->w_sgate : nullptr, p.L ? a->w_lat_down : nullptr,
                     a->x_lat, fused_dispatch ? &tf : nullptr)) != MOE_OK)
     return s;

@@ -226,11 +226,27 @@ struct TopkFuse {
   __half* x16;               // [W]
   float* xscale;             // [1]
 };
+// How k_topk scores and selects (the default is the softmax router):
+// score_fn 0: softmax (selection by logit, weights the softmax renormalised
+//   over the selected experts);
+// score_fn 1: sigmoid (s = sigmoid(logit); selection by s + bias[e] with
+//   bias nullable; weights s / sum of the selected s);
+// n_group > 1: group-limited selection (E / n_group consecutive experts per
+//   group, a group scored by the sum of its two largest expert scores, the
+//   softmax probability or the biased sigmoid score; the topk_group best
+//   groups kept, ties to the lower group; top-k among their experts);
+// the weights are multiplied by scale.
+struct RouteCfg {
+  const float* bias;         // [E] or nullptr
+  float scale;
+  int score_fn, n_group, topk_group;
+};
+constexpr int kMaxGroups = 64;
 // part [S, T, ld] router partial sums (ld >= E); with gate_logit set, column E
 // holds the sigmoid-gate row's partials and gate_logit[t] gets their sum;
 // f.x set: T == 1 and the fused dispatch above
 __global__ void k_topk(const float* part, int S, int T, int E, int ld, int k, int32_t* idx, float* w,
-                       float* logits, float* gate_logit, TopkFuse f);
+                       float* logits, float* gate_logit, TopkFuse f, RouteCfg rc);
 
 // --- permutation and activation operands ------------------------------------
 __global__ void k_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,

@@ -1,5 +1,10 @@
 // Router tail: softmax top-k with renormalised weights (rabbit README, model
-// table row "MoE routing": softmax top-10 of 512).
+// table row "MoE routing": softmax top-10 of 512), and the two other routers
+// the same table names: "noaux_tc sigmoid" (GLM-5.2; read as sigmoid scores,
+// a per-expert bias that steers the selection only, weights renormalised over
+// the unbiased scores and scaled) and "grouped routing" (Kimi Linear; read as
+// group-limited selection: the experts' groups ranked by the sum of their two
+// best scores, top-k inside the best groups).
 //
 // One CTA per token, one thread per expert. The router logits arrive as
 // split-K partial sums [S, T, E] from the router GEMM and are summed in a
@@ -33,7 +38,8 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
                                                      int E, int ld, int k, int32_t* __restrict__ idx,
                                                      float* __restrict__ w,
                                                      float* __restrict__ logits,
-                                                     float* __restrict__ gate_logit, TopkFuse f) {
+                                                     float* __restrict__ gate_logit, TopkFuse f,
+                                                     RouteCfg rc) {
   pdl_wait();
   pdl_trigger();
   __shared__ int s_cnt[kTopkThreads / 32];
@@ -50,17 +56,77 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   }
   if (gate_logit && e == E) gate_logit[tok] = sum_splits(part + (size_t)tok * ld + E, S, (size_t)T * ld);
   // a NaN logit never wins; -0 ranks equal to +0
-  const float v = (live && !isnan(acc)) ? (acc == 0.0f ? 0.0f : acc) : -INFINITY;
-  const uint32_t u = __float_as_uint(v);
+  const bool finite_in = live && !isnan(acc);
+  const float v = finite_in ? (acc == 0.0f ? 0.0f : acc) : -INFINITY;
+  // selection score (`choice`) and the value the weights use (`wval`):
+  // softmax: the logit for both; sigmoid: s + bias and s
+  float choice = v, wval = v;
+  if (rc.score_fn == 1) {
+    const float sg = finite_in ? 1.0f / (1.0f + expf(-acc)) : 0.0f;
+    float c = finite_in ? sg + (rc.bias ? rc.bias[e] : 0.0f) : -INFINITY;
+    if (isnan(c)) c = -INFINITY;
+    choice = c == 0.0f ? 0.0f : c;
+    wval = sg;
+  }
+  bool elig = live;
+  if (rc.n_group > 1) {
+    // group scores: the sum of the two largest expert scores of each group
+    // (the softmax probability up to its common denominator, exp(l - l_max),
+    // or the biased sigmoid score); then the rank of this expert's group
+    __shared__ float s_gv[kTopkThreads];
+    __shared__ float s_red[kTopkThreads / 32];
+    __shared__ float s_gscore[kMaxGroups];
+    float gv = choice;
+    if (rc.score_fn == 0) {
+      float m = v;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      if (lane == 0) s_red[warp] = m;
+      __syncthreads();
+      m = s_red[0];
+      for (int w2 = 1; w2 < kTopkThreads / 32; ++w2) m = fmaxf(m, s_red[w2]);
+      gv = finite_in ? expf(v - m) : 0.0f;
+    }
+    s_gv[e] = live ? gv : -INFINITY;
+    __syncthreads();
+    const int gsize = E / rc.n_group;
+    for (int g = warp; g < rc.n_group; g += kTopkThreads / 32) {
+      float m1 = -INFINITY, m2 = -INFINITY;
+      for (int i = lane; i < gsize; i += 32) {
+        const float x = s_gv[g * gsize + i];
+        if (x > m1) { m2 = m1; m1 = x; } else if (x > m2) { m2 = x; }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float o1 = __shfl_xor_sync(0xFFFFFFFFu, m1, off);
+        const float o2 = __shfl_xor_sync(0xFFFFFFFFu, m2, off);
+        m2 = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+        m1 = fmaxf(m1, o1);
+      }
+      if (lane == 0) s_gscore[g] = gsize > 1 ? m1 + m2 : m1;
+    }
+    __syncthreads();
+    if (live) {
+      const int g = e / gsize;
+      const float sg = s_gscore[g];
+      int grank = 0;
+      for (int j = 0; j < rc.n_group; ++j) {
+        const float sj = s_gscore[j];
+        grank += (sj > sg || (sj == sg && j < g)) ? 1 : 0;
+      }
+      elig = grank < rc.topk_group;
+    }
+  }
+  const uint32_t u = __float_as_uint(choice);
   const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 
-  // largest thr with #{key >= thr} >= k: the k-th largest key
+  // largest thr with #{key >= thr} >= k among the eligible: the k-th largest key
   uint32_t thr = 0;
   for (int b = 31; b >= 0; --b) {
     const uint32_t c = thr | (1u << b);
-    if (__syncthreads_count(live && key >= c) >= k) thr = c;
+    if (__syncthreads_count(elig && key >= c) >= k) thr = c;
   }
-  const bool gt = live && key > thr, eq = live && key == thr;
+  const bool gt = elig && key > thr, eq = elig && key == thr;
   const int n_gt = __syncthreads_count(gt);
   const uint32_t lt_mask = (1u << lane) - 1u;
   const unsigned eq_m = __ballot_sync(0xFFFFFFFFu, eq);
@@ -78,7 +144,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   if (sel) {
     s_key[pos] = key;
     s_exp[pos] = e;
-    s_val[pos] = v;
+    s_val[pos] = wval;
   }
   const bool fuse = f.x != nullptr;
   if (fuse) {
@@ -151,14 +217,16 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   // lane r now holds the r-th selection
   const float selv = (lane < k) ? s_val[lane] : 0.0f;
   const int sele = (lane < k) ? s_exp[lane] : 0;
+  // softmax: exp(l - l_top) over the selected (l_top = slot 0's logit, the
+  // largest selected); sigmoid: the unbiased scores themselves
   const float m = __shfl_sync(0xFFFFFFFFu, selv, 0);
-  const float ex = (lane < k) ? expf(selv - m) : 0.0f;
+  const float ex = (lane < k) ? (rc.score_fn == 1 ? selv : expf(selv - m)) : 0.0f;
   float den = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, off);
   if (lane < k) {
     idx[(size_t)tok * k + lane] = sele;
-    w[(size_t)tok * k + lane] = ex / den;
+    w[(size_t)tok * k + lane] = ex / den * rc.scale;
   }
 }
 

@@ -112,8 +112,14 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x,
   a.T = dims->T; a.K = dims->H; a.S = S; a.kper = dims->H / S;
   const dim3 grid((a.N + 16 * moe::kDenseWarps - 1) / (16 * moe::kDenseWarps), S, (a.T + 31) / 32);
   moe::k_dense_gemv<<<grid, 32 * moe::kDenseWarps, 0, cs>>>(a);
+  moe::RouteCfg rc;
+  rc.bias = nullptr;
+  rc.score_fn = dims->score_fn;
+  rc.n_group = dims->n_group > 1 ? dims->n_group : 1;
+  rc.topk_group = dims->n_group > 1 ? dims->topk_group : 1;
+  rc.scale = dims->route_scale == 0.0f ? 1.0f : dims->route_scale;
   moe::k_topk<<<dims->T, moe::kTopkThreads, 0, cs>>>(part, S, dims->T, dims->E, dims->E, dims->k, topk_idx,
-                                                     topk_w, logits, nullptr, moe::TopkFuse{});
+                                                     topk_w, logits, nullptr, moe::TopkFuse{}, rc);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return moe::record_error(MOE_ERR_CUDA, cudaGetErrorString(e));
   return MOE_OK;

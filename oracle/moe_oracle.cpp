@@ -306,9 +306,12 @@ void moe_o_router_logits(const uint16_t* x, const uint16_t* wr, int T, int H, in
 // Both: w is multiplied by `scale` (1 for the plain softmax router).
 // Group-limited selection (reading of "grouped routing"; n_group > 1): the E
 // experts form n_group consecutive groups of E / n_group; a group's score is
-// the sum of the two largest selection scores in it (the one score when a
-// group has one expert); the topk_group best groups are kept (ties: lower
-// group first) and the top k is taken among their experts only.
+// the sum of the two largest expert scores in it (the one score when a group
+// has one expert), the expert score being the softmax probability (softmax;
+// computed as exp(l_e - max_e' l_e'), the common denominator dropped) or the
+// biased sigmoid score s_e + bias[e] (sigmoid); the topk_group best groups
+// are kept (ties: lower group first) and the top k is taken among their
+// experts only, ranked as above.
 // Near-tie flags: kTieSet when the k-th and (k+1)-th selection scores among
 // the eligible experts differ by less than near_tie (the selected SET then
 // depends on rounding); kTieOrder when two adjacent selected scores do (only
@@ -333,11 +336,15 @@ int moe_o_route(const double* logits, const double* bias, int T, int E, int k, i
     uint8_t f = 0;
     std::vector<char> eligible(E, 1);
     if (n_group > 1) {
+      std::vector<double> gval(E);
+      double lmax = -INFINITY;
+      for (int e = 0; e < E; ++e) lmax = std::max(lmax, l[e]);
+      for (int e = 0; e < E; ++e) gval[e] = score_fn == 0 ? std::exp(l[e] - lmax) : choice[e];
       std::vector<double> gscore(n_group);
       std::vector<int> ord;
       for (int g = 0; g < n_group; ++g) {
-        rank_desc(choice.data() + (int64_t)g * gsize, gsize, ord);
-        gscore[g] = choice[g * gsize + ord[0]] + (gsize > 1 ? choice[g * gsize + ord[1]] : 0.0);
+        rank_desc(gval.data() + (int64_t)g * gsize, gsize, ord);
+        gscore[g] = gval[g * gsize + ord[0]] + (gsize > 1 ? gval[g * gsize + ord[1]] : 0.0);
       }
       std::vector<int> gord;
       rank_desc(gscore.data(), n_group, gord);

@@ -13,6 +13,7 @@ ones the workload descriptions state):
 * routed MXFP4 weights: element codes uniform over the 16 E2M1 codes (so each
   packed byte is uniform over 0..255) and E8M0 scale codes uniform over
   120..127 (block scales 2^-7 .. 2^0)
+* router-variant workloads: a per-expert fp32 selection bias ~ N(0, bias_std)
 * skewed routing (small-batch decode and prefill workloads): each skewed token
   receives a set S_t of k distinct experts drawn without replacement with
   probability proportional to rank^-1.1 (Zipf 1.1 over a seeded ranking), and
@@ -48,6 +49,14 @@ class MoeWorkload:
     L: int = 0      # latent width (0: routed experts run at width H)
     skew: str = "none"   # "none" | "hot64" | "zipf"
     seed: int = 1000
+    # router variant (default: softmax top-k): score function 0 softmax /
+    # 1 sigmoid, expert groups and groups kept, weight scale, and the standard
+    # deviation of a seeded per-expert selection bias (0: none)
+    score_fn: int = 0
+    n_group: int = 0
+    topk_group: int = 0
+    route_scale: float = 1.0
+    bias_std: float = 0.0
 
     @property
     def W(self) -> int:
@@ -69,6 +78,7 @@ WORKLOADS = {
 # stream ids
 _S_X, _S_ROUTER, _S_SG, _S_SU, _S_SD, _S_SGATE, _S_LD, _S_LU = 1, 2, 3, 4, 5, 6, 7, 8
 _S_SKEW = 9
+_S_BIAS = 10
 _S_WG, _S_WU, _S_WD = 20, 21, 22
 
 
@@ -158,6 +168,9 @@ def dense_inputs(w: MoeWorkload) -> dict:
     if w.L:
         d["w_lat_down"] = _normal_bf16(s, _S_LD, (w.L, w.H), 0.02)
         d["w_lat_up"] = _normal_bf16(s, _S_LU, (w.H, w.L), 0.02)
+    if w.bias_std > 0:
+        d["e_bias"] = (_rng(s, _S_BIAS).standard_normal(w.E, dtype=np.float32)
+                       * np.float32(w.bias_std))
     x = _rng(s, _S_X).standard_normal((w.T, w.H), dtype=np.float32)
     if w.skew != "none":
         x = x + _skew_boost(w, bf16_bits_to_f32(d["w_router"]))
@@ -219,7 +232,8 @@ def to_device(w: MoeWorkload, dense: dict | None = None, device="cuda", chunk: i
     dense = dense_inputs(w) if dense is None else dense
     out = {}
     for name, arr in dense.items():
-        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16))
+        arr = np.ascontiguousarray(arr)
+        t = torch.from_numpy(arr if arr.dtype == np.float32 else arr.view(np.int16))
         out[name] = t.to(device)
     (Ng, Kg), (Nd, Kd) = expert_shapes(w)
     shapes = {"wg_q": (Ng, Kg // 2), "wg_s": (Ng, Kg // 32), "wu_q": (Ng, Kg // 2),

@@ -70,6 +70,20 @@ def expert_getter(w):
     return get
 
 
+def route_kw(w, dense):
+    """The oracle's router configuration of a workload (score function,
+    selection bias, groups, weight scale), for O.route / check_routing."""
+    return dict(score_fn=w.score_fn, bias=dense.get("e_bias"), n_group=max(1, w.n_group),
+                topk_group=max(1, w.topk_group), scale=w.route_scale)
+
+
+def layer_kw(w, dense):
+    """The same configuration in O.moe_layer's keyword names."""
+    r = route_kw(w, dense)
+    return dict(score_fn=r["score_fn"], e_bias=r["bias"], n_group=r["n_group"],
+                topk_group=r["topk_group"], route_scale=r["scale"])
+
+
 def max_rel_err(got, want):
     rms = float(np.sqrt(np.mean(np.square(want))))
     return float(np.max(np.abs(got - want))) / rms, rms

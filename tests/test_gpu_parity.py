@@ -23,7 +23,7 @@ import synth
 pytestmark = pytest.mark.gpu
 
 from parity_harness import (TOL, DeviceRun, check_permutation, check_routing, check_x_op_f16,  # noqa: E402
-                            expert_getter, max_rel_err)
+                            expert_getter, layer_kw, max_rel_err, route_kw)
 
 MEDIUM = synth.MoeWorkload("medium_ragged", T=70, H=640, I=384, E=6, k=3, I_shared=256, seed=77)
 LATENT_SMALL = synth.MoeWorkload("latent_small", T=5, H=384, I=128, E=12, k=3, I_shared=128, L=256,
@@ -50,6 +50,22 @@ MMA_MANY = synth.MoeWorkload("mma_many", T=44, H=1024, I=512, E=6, k=2, I_shared
 # tcgen05 GEMM (16-token tile), dispatch and operand from the top-k launch
 TC_T1 = synth.MoeWorkload("tc_t1", T=1, H=640, I=256, E=12, k=3, I_shared=384, seed=85)
 MMA_MIXED = synth.MoeWorkload("mma_mixed", T=24, H=1024, I=512, E=40, k=2, I_shared=256, seed=84)
+# router variants (rabbit README, model table row "MoE routing"): sigmoid scores
+# with a selection bias and a weight scale ("noaux_tc sigmoid"), group-limited
+# selection ("grouped routing") with sigmoid and with softmax scores, one token
+# at full decode size (the top-k launch writes the dispatch), and 130 tokens
+# (router on the tcgen05 GEMM)
+NOAUX = synth.MoeWorkload("noaux_sigmoid", T=6, H=512, I=256, E=32, k=4, I_shared=128, seed=86,
+                          score_fn=1, bias_std=0.05, route_scale=2.5)
+GROUPED = synth.MoeWorkload("grouped_sigmoid", T=5, H=512, I=256, E=64, k=6, I_shared=128, seed=87,
+                            score_fn=1, n_group=8, topk_group=4, bias_std=0.02)
+GROUPED_SM = synth.MoeWorkload("grouped_softmax", T=9, H=512, I=256, E=48, k=4, I_shared=128,
+                               seed=88, n_group=6, topk_group=2)
+GROUPED_WIDE = synth.MoeWorkload("grouped_wide", T=130, H=512, I=128, E=64, k=4, I_shared=256,
+                                 seed=89, n_group=4, topk_group=2, score_fn=1, bias_std=0.03)
+DECODE1_GROUPED = synth.MoeWorkload("decode1_grouped", T=1, H=8192, I=2048, E=512, k=10,
+                                    I_shared=2048, seed=90, score_fn=1, n_group=8, topk_group=4,
+                                    bias_std=0.05, route_scale=2.5)
 
 CASES = [
     (synth.WORKLOADS["tiny"], None),
@@ -65,6 +81,11 @@ CASES = [
     (synth.WORKLOADS["latent16"], None),
     (synth.WORKLOADS["decode1"], None),
     (synth.WORKLOADS["decode32"], None),
+    (NOAUX, None),
+    (GROUPED, None),
+    (GROUPED_SM, None),
+    (GROUPED_WIDE, None),
+    (DECODE1_GROUPED, None),
 ]
 
 
@@ -103,16 +124,17 @@ def ref(case):
     d = run.dense
     tokens = np.arange(w.T) if sample is None else np.array(sample)
     sub = dict(d, x=d["x"][tokens])
-    idx_o, _, flags = O.route(O.router_logits(sub["x"], d["w_router"]), w.k)
+    idx_o, _, flags = O.route(O.router_logits(sub["x"], d["w_router"]), w.k, **route_kw(w, d))
     tied = flags != 0
     override = np.where(tied[:, None], gpu["idx"][tokens], idx_o) if np.any(tied) else None
-    return tokens, O.moe_layer(sub, w.k, expert_getter(w), idx_override=override)
+    return tokens, O.moe_layer(sub, w.k, expert_getter(w), idx_override=override,
+                               **layer_kw(w, d))
 
 
 def test_routing_and_permutation(case):
     w, sample, run, gpu, layer = case
     ref_logits = O.router_logits(run.dense["x"], run.dense["w_router"])
-    check_routing(gpu, ref_logits, w.k)
+    check_routing(gpu, ref_logits, w.k, **route_kw(w, run.dense))
     check_permutation(gpu, w.E)
 
 
@@ -321,3 +343,15 @@ def test_bounded_wait_gives_up_and_sets_the_status_bit():
     ref = O.moe_layer(run.dense, w.k, expert_getter(w))
     err, _ = max_rel_err(gpu["y"], ref["y"])
     assert err <= TOL
+
+
+def test_router_variant_selection_differs_from_softmax():
+    """The variant cases really exercise other selections: the biased and
+    group-limited routers pick other experts than plain softmax top-k on the
+    same logits for some tokens (so a kernel ignoring the variant fails)."""
+    for w in (NOAUX, GROUPED, GROUPED_SM):
+        d = synth.dense_inputs(w)
+        lg = O.router_logits(d["x"], d["w_router"])
+        plain = O.route(lg, w.k)[0]
+        var = O.route(lg, w.k, **route_kw(w, d))[0]
+        assert not np.array_equal(np.sort(plain, axis=1), np.sort(var, axis=1)), w.name

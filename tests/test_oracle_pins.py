@@ -482,3 +482,107 @@ def test_silu_sigmoid_match_torch_including_extremes():
                                rtol=1e-14, atol=1e-300)
     np.testing.assert_allclose(O.sigmoid(z), torch.sigmoid(torch.from_numpy(z)).numpy(),
                                rtol=1e-14, atol=1e-300)
+
+
+# ---------------------------------------------------------------------------
+# router variants: sigmoid scores with a selection bias ("noaux_tc sigmoid"),
+# group-limited selection ("grouped routing")
+# ---------------------------------------------------------------------------
+
+def test_sigmoid_router_without_bias_selects_like_softmax():
+    # sigmoid and softmax are both monotone in the logit: same experts, same order
+    rng = np.random.default_rng(41)
+    logits = rng.standard_normal((25, 32)) * 1.8
+    a, _, _ = O.route(logits, 6)
+    b, w, _ = O.route(logits, 6, score_fn=O.SIGMOID, scale=2.5)
+    np.testing.assert_array_equal(a, b)
+    s = scipy.special.expit(np.take_along_axis(logits, b.astype(np.int64), axis=1))
+    np.testing.assert_allclose(w, 2.5 * s / s.sum(axis=1, keepdims=True), rtol=1e-14)
+
+
+def test_sigmoid_router_with_bias_brute_force():
+    rng = np.random.default_rng(42)
+    logits = rng.standard_normal((30, 12)) * 1.8
+    bias = np.round(rng.standard_normal(12) * 0.2, 3)
+    idx, w, _ = O.route(logits, 4, score_fn=O.SIGMOID, bias=bias)
+    for t in range(30):
+        s = [1.0 / (1.0 + math.exp(-v)) for v in logits[t]]
+        order = sorted(range(12), key=lambda e: (-(s[e] + bias[e]), e))[:4]
+        assert list(idx[t]) == order
+        tot = sum(s[e] for e in order)
+        np.testing.assert_allclose(w[t], [s[e] / tot for e in order], rtol=1e-14)
+    # the bias changes the selection somewhere, and not the weight rule
+    plain, _, _ = O.route(logits, 4, score_fn=O.SIGMOID)
+    assert not np.array_equal(np.sort(plain, axis=1), np.sort(idx, axis=1))
+
+
+def test_softmax_router_ignores_the_selection_bias():
+    rng = np.random.default_rng(43)
+    logits = rng.standard_normal((10, 16))
+    a = O.route(logits, 3)
+    b = O.route(logits, 3, bias=rng.standard_normal(16))
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_grouped_sigmoid_router_hand_worked():
+    # 8 experts in 4 groups of 2, keep 2 groups, top-3, weights x 2.5.
+    # logits 0 except expert 6 (ln 3): sigmoid scores 0.5, and 0.75 for expert 6;
+    # with the bias, selection scores
+    #   [0.625, 0.5 | 0.875, 0.1875 | 0.5625, 0.5 | 0.75, 0.8125]
+    # group scores (sum of the two largest): 1.125, 1.0625, 1.0625, 1.5625
+    # -> keep groups 3 and 0; expert 2 (0.875, the best overall) is excluded;
+    # top-3 of {0, 1, 6, 7}: 7 (0.8125), 6 (0.75), 0 (0.625);
+    # weights 2.5 * [0.5, 0.75, 0.5] / 1.75 from the unbiased scores
+    logits = np.zeros((1, 8))
+    logits[0, 6] = math.log(3.0)
+    bias = np.array([0.125, 0, 0.375, -0.3125, 0.0625, 0, 0, 0.3125])
+    idx, w, flags = O.route(logits, 3, score_fn=O.SIGMOID, bias=bias, n_group=4, topk_group=2,
+                            scale=2.5)
+    assert list(idx[0]) == [7, 6, 0]
+    np.testing.assert_allclose(w[0], 2.5 * np.array([0.5, 0.75, 0.5]) / 1.75, rtol=1e-14)
+    assert flags[0] == 0
+    # without groups expert 2 wins
+    idx2, _, _ = O.route(logits, 3, score_fn=O.SIGMOID, bias=bias)
+    assert list(idx2[0]) == [2, 7, 6]
+
+
+def test_grouped_softmax_router_hand_worked():
+    # 8 experts in 4 groups of 2, keep 2 groups, top-3; group scores on the
+    # probabilities (exp(l - 3)): g0 = e^-1 + e^-1.1 = 0.7008,
+    # g1 = 1 + e^-8 = 1.0003, g2 = 2 e^-3 = 0.0996, g3 = e^-0.5 + e^-3 = 0.6563
+    # -> keep g1, g0; expert 6 (logit 2.5, second overall) is excluded;
+    # top-3 of {0, 1, 2, 3}: 2, 0, 1; weights = softmax renormalised over them
+    logits = np.array([[2.0, 1.9, 3.0, -5.0, 0.0, 0.0, 2.5, 0.0]])
+    idx, w, flags = O.route(logits, 3, n_group=4, topk_group=2)
+    assert list(idx[0]) == [2, 0, 1]
+    e = np.array([1.0, math.exp(-1.0), math.exp(-1.1)])
+    np.testing.assert_allclose(w[0], e / e.sum(), rtol=1e-14)
+    assert flags[0] == 0
+    assert list(O.route(logits, 3)[0][0]) == [2, 6, 0]
+
+
+def test_grouped_router_reduces_to_plain_routing():
+    rng = np.random.default_rng(44)
+    logits = rng.standard_normal((20, 24)) * 1.8
+    bias = rng.standard_normal(24) * 0.1
+    for fn, b in ((O.SOFTMAX, None), (O.SIGMOID, bias)):
+        plain = O.route(logits, 5, score_fn=fn, bias=b)
+        # every group kept
+        allg = O.route(logits, 5, score_fn=fn, bias=b, n_group=4, topk_group=4)
+        # one expert per group, k groups kept: the group scores rank like the experts
+        single = O.route(logits, 5, score_fn=fn, bias=b, n_group=24, topk_group=5)
+        for other in (allg, single):
+            np.testing.assert_array_equal(plain[0], other[0])
+            np.testing.assert_allclose(plain[1], other[1], rtol=1e-15)
+
+
+def test_grouped_router_group_near_tie_flag_and_rejections():
+    logits = np.zeros((1, 8))
+    bias = np.array([0.25, 0.25, 0.25, 0.25, 0.0, 0.0, 0.0, 0.0])
+    _, _, flags = O.route(logits, 2, score_fn=O.SIGMOID, bias=bias, n_group=4, topk_group=1)
+    assert flags[0] & O.TIE_GROUP        # groups 0 and 1 tie exactly
+    with pytest.raises(ValueError):
+        O.route(logits, 2, n_group=3, topk_group=1)       # 8 experts do not split in 3
+    with pytest.raises(ValueError):
+        O.route(logits, 3, n_group=4, topk_group=1)       # one group of 2 cannot give 3
