@@ -80,13 +80,18 @@ MOE_DEV float warp_max(float v) {
 // block = 32 * (kFmaConsumers + 1) threads (warp 0: producer); one CTA per SM;
 // dynamic shared memory = g.smem_bytes (the ring, then the activation buffer
 // at g.act_off).
-// The producer waits for the previous kernel (griddepcontrol.wait) only before
-// it copies an activation row (x from the dispatch, h from the gate/up
-// kernel), which goes out ahead of the weights of its first stage.
+// The kernel lets its dependants launch at once (griddepcontrol.launch_
+// dependents), then waits for the previous kernel (griddepcontrol.wait)
+// before it reads anything: for one token the previous kernel is the top-k
+// launch, which writes the dispatch this kernel starts from (its expert list,
+// offsets and row maps), and a dependant may start before that launch has
+// written them. A dependant's own wait returns only after this grid has
+// completed, hence after the dispatch was complete.
 // ---------------------------------------------------------------------------
 template <int BPL, bool kGateUp, int RPS>
 __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArgs a, FmaGeometry g) {
   pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
   __shared__ int s_wsum[kFmaConsumers + 1];
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   uint8_t* act = smem + g.act_off;
 
   // 1) the single-token experts, in the order of the expert list (the
-  //    dispatch's output: complete before this grid can start, read through L2)
+  //    dispatch's output, complete once the wait above returned; read through L2)
   const int n_act = __ldcg(a.expert_list);
   int n_single = 0;
   for (int base = 0; base < n_act; base += 32 * kWarps) {
@@ -131,12 +136,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   // 2) this CTA's share of the units (gate/up: row pairs; down: rows)
   const long total = (long)n_single * N;
   const long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
-  if (lo >= hi) {                                         // uniform across the CTA
-    // no work, but the grid must not complete before the previous one: the
-    // next kernel's wait covers this grid only
-    pdl_wait();
-    return;
-  }
+  if (lo >= hi) return;                                   // uniform across the CTA
   uint64_t* full = s_bars;
   uint64_t* empty = s_bars + kFmaMaxStages;
   if (threadIdx.x == 0) {
@@ -174,12 +174,11 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       uint32_t ph = 0;
       // activation rows: the slots whose row is still to be copied, in order
       int pend[4], n_pend = 0, n_loaded = 0, cur_key = -1, cur_si = -1;
-      bool waited = false, ok = true;
-      auto load_acts = [&]() -> bool {        // after the wait: copy the pending rows
-        if (!waited) {
-          pdl_wait();
+      bool fenced = false, ok = true;
+      auto load_acts = [&]() -> bool {        // copy the pending rows
+        if (!fenced) {
           asm volatile("fence.proxy.async;\n" ::: "memory");   // the previous grid's writes, then bulk reads
-          waited = true;
+          fenced = true;
         }
         for (int i = 0; i < n_pend; ++i) {
           if (n_loaded > 0 && !tc::wait_or_abort(&s_act[1], (uint32_t)((n_loaded - 1) & 1), abort))
@@ -237,7 +236,6 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
         if (++slot == g.nst) { slot = 0; ph ^= 1u; }
       }
       if (ok && n_pend > 0 && !load_acts()) ok = false;
-      if (!waited) pdl_wait();
       if (*abort) {     // let every issued copy land before the CTA can exit
         for (int s = 0; s < g.nst; ++s)
           if (filled[s]) mbar_wait(&full[s], last_ph[s]);
@@ -250,7 +248,6 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
     // over one half of K (half the activation registers), and combine their
     // partial sums through shared memory; K <= 2048: warp w takes row pair w;
     // down: warp w takes rows RPS*w ... of a stage
-    pdl_wait();                             // the previous grid's outputs (xscale)
     const int w = warp - 1;
     constexpr int BW = kSplit ? (BPL + 1) / 2 : BPL;     // blocks per lane of this warp
     const int half = kSplit ? (w & 1) : 0;

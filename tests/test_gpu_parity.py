@@ -201,6 +201,34 @@ def test_fused_layer_routing_and_dispatch_against_oracle(case, ref):
         check_x_op_f16(layer["x_op"], run.dense["x"], w.T, w.W)
 
 
+def test_layer_on_a_new_input_follows_its_own_routing(case):
+    """moe_layer on x, then at once on another input (x with every sign
+    flipped: other experts for every token), back to back on one stream: the
+    second output must match the oracle for the second input. The routed
+    expert kernels read the dispatch the routing chain writes in the same
+    call; reading it before that launch has finished would reuse the first
+    input's experts (the same buffers, valid but stale)."""
+    w, sample, run, gpu, layer = case
+    d = run.dense
+    x2 = np.ascontiguousarray(d["x"] ^ np.uint16(0x8000))
+    x2_dev = torch.from_numpy(x2.view(np.int16)).cuda()
+    run.layer(run.dev["x"])
+    y2 = run.layer(x2_dev)
+    torch.cuda.synchronize()
+    y2 = y2.cpu().numpy().astype(np.float64)
+    idx2 = run.layer.topk_idx.cpu().numpy()
+    tokens = np.arange(w.T) if sample is None else np.array(sample)
+    sub = dict(d, x=x2[tokens])
+    idx_o, _, flags = O.route(O.router_logits(sub["x"], d["w_router"]), w.k, **route_kw(w, d))
+    tied = flags != 0
+    assert not np.array_equal(np.sort(idx_o[~tied], axis=1), np.sort(gpu["idx"][tokens][~tied], axis=1))
+    np.testing.assert_array_equal(idx2[tokens][~tied], idx_o[~tied])
+    override = np.where(tied[:, None], idx2[tokens], idx_o) if np.any(tied) else None
+    ref = O.moe_layer(sub, w.k, expert_getter(w), idx_override=override, **layer_kw(w, d))
+    err, rms = max_rel_err(y2[tokens], ref["y"])
+    assert err <= TOL, (err, rms)
+
+
 def test_fused_layer_matches_stages_bitwise(case):
     w, sample, run, gpu, layer = case
     np.testing.assert_array_equal(layer["y"], gpu["y"])
