@@ -80,18 +80,19 @@ MOE_DEV float warp_max(float v) {
 // block = 32 * (kFmaConsumers + 1) threads (warp 0: producer); one CTA per SM;
 // dynamic shared memory = g.smem_bytes (the ring, then the activation buffer
 // at g.act_off).
-// The kernel lets its dependants launch at once (griddepcontrol.launch_
-// dependents), then waits for the previous kernel (griddepcontrol.wait)
-// before it reads anything: for one token the previous kernel is the top-k
-// launch, which writes the dispatch this kernel starts from (its expert list,
-// offsets and row maps), and a dependant may start before that launch has
-// written them. A dependant's own wait returns only after this grid has
-// completed, hence after the dispatch was complete.
+// gate/up: waits for the previous kernel (griddepcontrol.wait) before it
+// reads anything (for one token the previous kernel is the top-k launch,
+// which writes the dispatch this kernel starts from: expert list, offsets,
+// row maps) and only then lets its dependants launch, so that when the down
+// projection starts, the dispatch is complete.
+// down: reads the dispatch and streams its first weight stages at once (they
+// land while the gate/up grid's last CTAs finish); it waits for the previous
+// kernel only before it copies the expert's h row, the gate/up output.
 // ---------------------------------------------------------------------------
 template <int BPL, bool kGateUp, int RPS>
 __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArgs a, FmaGeometry g) {
+  if (kGateUp) pdl_wait();
   pdl_trigger();
-  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int16_t s_list[1024];      // single-token experts, ascending (E <= 1024)
   __shared__ int s_wsum[kFmaConsumers + 1];
@@ -136,7 +137,12 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
   // 2) this CTA's share of the units (gate/up: row pairs; down: rows)
   const long total = (long)n_single * N;
   const long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
-  if (lo >= hi) return;                                   // uniform across the CTA
+  if (lo >= hi) {                                         // uniform across the CTA
+    // no work; the grid must still not complete before the previous one (the
+    // next kernel's wait covers this grid only)
+    if (!kGateUp) pdl_wait();
+    return;
+  }
   uint64_t* full = s_bars;
   uint64_t* empty = s_bars + kFmaMaxStages;
   if (threadIdx.x == 0) {
@@ -173,10 +179,15 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
       int si = si0, r = r_lo, slot = 0, k = 0;
       uint32_t ph = 0;
       // activation rows: the slots whose row is still to be copied, in order
+      // (at most 4 deferred)
       int pend[4], n_pend = 0, n_loaded = 0, cur_key = -1, cur_si = -1;
-      bool fenced = false, ok = true;
+      bool fenced = false, ok = true, waited = kGateUp;
       auto load_acts = [&]() -> bool {        // copy the pending rows
         if (!fenced) {
+          if (!waited) {
+            pdl_wait();                       // down: the gate/up grid's h rows
+            waited = true;
+          }
           asm volatile("fence.proxy.async;\n" ::: "memory");   // the previous grid's writes, then bulk reads
           fenced = true;
         }
@@ -207,8 +218,10 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
           }
         }
         // a new activation row goes out ahead of the stage's weights (it is
-        // small, and the consumers need it before the stage)
-        if (n_pend > 0 && !load_acts()) { ok = false; break; }
+        // small, and the consumers need it before the stage); the down
+        // kernel's first h row waits until the ring is full (the weights of
+        // its first stages do not depend on the previous grid)
+        if (n_pend > 0 && (waited || filled[slot] || n_pend == 4) && !load_acts()) { ok = false; break; }
         if (!tc::wait_or_abort(&empty[slot], ph ^ 1u, abort)) { ok = false; break; }
         const size_t row = (size_t)s_list[si] * N + r;
         const uint32_t cb = n * qrow;
@@ -236,6 +249,7 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
         if (++slot == g.nst) { slot = 0; ph ^= 1u; }
       }
       if (ok && n_pend > 0 && !load_acts()) ok = false;
+      if (!waited) pdl_wait();                // the grid must not complete before the previous one
       if (*abort) {     // let every issued copy land before the CTA can exit
         for (int s = 0; s < g.nst; ++s)
           if (filled[s]) mbar_wait(&full[s], last_ph[s]);
