@@ -436,6 +436,95 @@ def measure(args, w, steps, rank, local_rank, world, act=None):
     return out
 
 
+def measure_streamed(args, base, tokens=16, slots=128):
+    """Decode with the routed experts streamed from host memory through the
+    expert cache (moe_expert_ffn_streamed): the layer of `base` (weights
+    seeded as that workload) with every expert in page-locked host memory, a
+    cache of `slots` experts on the device, and a fresh token each step (the
+    cache starts empty). One step = route, dispatch, read the expert list
+    back, the streamed routed experts, combine; CUDA events around it on the
+    launching stream. The bound is the host link: the same bytes copied
+    host -> device alone (pinned, one copy) give the peak."""
+    import dataclasses
+
+    import torch
+
+    import mxfp4_routed_expert_04_b200 as M
+    import synth
+
+    w = dataclasses.replace(base, T=1)
+    wt = dataclasses.replace(base, T=tokens)                 # the token rows, same weights
+    dense = synth.dense_inputs(w)
+    xs = synth.dense_inputs(wt)["x"]
+    dev = {n: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+           for n, a in dense.items() if n != "x"}
+    (Ng, Kg), (Nd, Kd) = synth.expert_shapes(w)
+    shp = {"wg_q": (Ng, Kg // 2), "wg_s": (Ng, Kg // 32), "wu_q": (Ng, Kg // 2),
+           "wu_s": (Ng, Kg // 32), "wd_q": (Nd, Kd // 2), "wd_s": (Nd, Kd // 32)}
+    host = {n: torch.empty((w.E,) + s, dtype=torch.uint8, pin_memory=True) for n, s in shp.items()}
+    for e0 in range(0, w.E, 32):
+        ids = list(range(e0, min(w.E, e0 + 32)))
+        ex = synth.expert_weights(w, ids)
+        for n in shp:
+            host[n][e0:e0 + len(ids)].copy_(torch.from_numpy(ex[n]))
+    names = ("wg_q", "wg_s", "wu_q", "wu_s", "wd_q", "wd_s")
+    dims = M.MoeDims.of(w)
+    # the layer's buffers; no routed expert is resident (the step calls used
+    # here never read the routed weights of the layer)
+    layer = M.MoeLayer(dims, dict(dev, wg_q=None, wg_s=None, wu_q=None, wu_s=None, wd_q=None,
+                                  wd_s=None))
+    cache = M.ExpertCache(dims, slots, [tuple(host[n][e] for n in names) for e in range(w.E)])
+    x = torch.empty(1, w.H, dtype=torch.int16, device="cuda")
+    xs_dev = torch.from_numpy(xs.view(np.int16)).cuda()
+    stream = torch.cuda.current_stream()
+    L = layer
+
+    def step(t):
+        x.copy_(xs_dev[t:t + 1])
+        M.moe_route(dims, x, dev["w_router"], L.topk_idx, L.topk_w, None, L.ws)
+        M.moe_permute(dims, L.topk_idx, x, L.counts, L.offsets, L.expert_list, L.row_token,
+                      L.row_slot, L.slot_row, L.x_op, L.ws)
+        lst = L.expert_list[:1 + w.k].cpu().tolist()      # the dispatch read back (a sync)
+        cache.ffn(lst[1:1 + lst[0]], L.x_op, L.offsets, L.row_token, L.y_perm, L.ws)
+        M.moe_combine(dims, L.y_perm, L.slot_row, L.topk_w, x, dev["w_sgate"], dev["ws_gate"],
+                      dev["ws_up"], dev["ws_down"], None, L.y, L.ws)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(tokens)]
+    torch.cuda.synchronize()
+    for t in range(tokens):
+        a, b = evs[t]
+        a.record(stream)
+        step(t)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    st = cache.stats()
+    cache.close()
+    # the host link alone: one pinned copy of the same number of bytes
+    nbytes = max(st["bytes_copied"], 1 << 20)
+    src = host["wg_q"].view(-1)[: min(nbytes, host["wg_q"].numel())]
+    dst = torch.empty_like(src, device="cuda")
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dst.copy_(src, non_blocking=True)
+    a.record(stream)
+    dst.copy_(src, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    link_gbs = src.numel() / (a.elapsed_time(b) * 1e-3) / 1e9
+    total_s = sum(ms) * 1e-3
+    h2d_gbs = st["bytes_copied"] / total_s / 1e9
+    return {"value": tokens / total_s, "unit": "tokens/s", "steps": tokens,
+            "ms_per_step": sum(ms) / tokens,
+            "config": {"workload": workload_label(w) + f", experts in host memory, {slots}-slot "
+                                                      f"device cache (LRU), {tokens} distinct tokens",
+                       "act_mode": "bf16"},
+            "cache": st, "hit_rate": st["hits"] / max(1, st["hits"] + st["misses"]),
+            "roofline": {"bound": "host link", "achieved": h2d_gbs, "peak": link_gbs,
+                         "unit": "GB/s", "frac": h2d_gbs / link_gbs,
+                         "peak_kind": "measured in this run: one pinned host-to-device copy"}}
+
+
 def run_ours(args, w):
     """The headline workload plus the extra workloads, one after the other on
     the same GPU(s); rank 0 returns the JSON line's dict."""
@@ -461,6 +550,12 @@ def run_ours(args, w):
         r = measure(args, synth.WORKLOADS[name], min(args.steps, 10), rank, local_rank, world)
         if r is not None:
             extras[name] = r
+    if args.streamed:
+        gc.collect()
+        torch.cuda.empty_cache()
+        r = measure_streamed(args, w)
+        if rank == 0:
+            extras["decode1_streamed"] = r
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -595,6 +690,8 @@ def main():
                          "reported under 'workloads' (default with the decode1 headline: "
                          + ",".join(EXTRA_DEFAULT) + ")")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-streamed", dest="streamed", action="store_false",
+                    help="skip the decode measurement with experts streamed from host memory")
     ap.add_argument("--act", choices=["bf16", "mxfp4"], default=None,
                     help="activation operand of the routed experts (default: mxfp4 for "
                          "prefill workloads, bf16 otherwise)")
@@ -614,6 +711,9 @@ def main():
         w = dataclasses.replace(w, T=args.tokens, name=f"{w.name}-T{args.tokens}")
     if args.no_extra or args.experts or args.tokens:
         args.extra = []
+        args.streamed = False
+    if args.workload != "decode1":
+        args.streamed = False
     elif args.extra is None:
         args.extra = list(EXTRA_DEFAULT) if args.workload == "decode1" else []
     else:

@@ -257,6 +257,42 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
                           const uint8_t* wd_q, const uint8_t* wd_s,
                           float* y_perm, void* ws, size_t ws_bytes, void* stream);
 
+/* --- routed experts streamed from host memory --------------------------------
+ * (rabbit README: the routed experts do not stay resident; they "stream on
+ * demand through a per-layer LRU cache", and with "per-expert early drain" an
+ * expert's matmul starts the moment its own bytes land.)
+ * A cache of `slots` expert slots in device memory (caller-owned, sized by
+ * moe_expert_cache_bytes, 256-byte aligned) in front of experts kept in host
+ * memory. MOE_ACT_BF16 layers only.
+ *
+ * moe_expert_ffn_streamed computes what moe_expert_ffn computes (the same
+ * kernels, bit for bit) for the experts listed in `active` (HOST array of
+ * n_active distinct ids, e.g. expert_list[1..] of moe_permute read back;
+ * n_active <= slots): experts already in a slot (hits) keep it; every other
+ * one takes the least recently used slot that this call does not use and is
+ * copied there from host_experts (HOST array of E*6 pointers: per expert its
+ * wg_q, wg_s, wu_q, wu_s, wd_q, wd_s in the canonical layout, in page-locked
+ * host memory for the copies to be asynchronous) on the cache's own copy
+ * stream, after the last launch that read the slot. Each expert's gate/up and
+ * down launches wait (on `stream`) only for their own expert's copy, in list
+ * order; hits start at once. x_op, offsets, row_token, y_perm, ws as for
+ * moe_expert_ffn. The cache is not capturable in a CUDA graph (its copies run
+ * on a stream of its own). Calls on one cache are serialised by a lock.
+ */
+typedef struct moe_expert_cache moe_expert_cache;   /* opaque, host side */
+size_t moe_expert_cache_bytes(const moe_dims* dims, int32_t slots);
+moe_status moe_expert_cache_create(const moe_dims* dims, int32_t slots, void* dev_mem, size_t dev_bytes,
+                                   moe_expert_cache** out);
+/* Waits for the cache's copies, then frees its host-side state (not dev_mem). */
+moe_status moe_expert_cache_destroy(moe_expert_cache* cache);
+/* Running totals: experts found in a slot, experts copied, bytes copied. */
+moe_status moe_expert_cache_stats(const moe_expert_cache* cache, int64_t* hits, int64_t* misses,
+                                  int64_t* bytes_copied);
+moe_status moe_expert_ffn_streamed(moe_expert_cache* cache, const moe_dims* dims, const int32_t* active,
+                                   int32_t n_active, const void* x_op, const int32_t* offsets,
+                                   const int32_t* row_token, const uint8_t* const* host_experts,
+                                   float* y_perm, void* ws, size_t ws_bytes, void* stream);
+
 /* --- MXFP4 tensor-core operands ----------------------------------------------
  * (No counterpart in the pages: data layout of this library.)
  * moe_tile_scales: canonical row-major E8M0 scales [rows, K/32] (src) -> the

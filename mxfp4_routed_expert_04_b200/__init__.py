@@ -19,7 +19,8 @@ __all__ = [
     "moe_device_status", "moe_route", "moe_route_biased", "moe_route_noalloc", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_latent_down", "moe_layer", "moe_mxf4_layout_of", "moe_tile_scales",
     "moe_selftest_bounded_wait", "STATUS_BAD_EXPERT", "STATUS_REPEATED_EXPERT",
-    "STATUS_WAIT_TIMEOUT", "SCORE_SOFTMAX", "SCORE_SIGMOID", "MoeLayer",
+    "STATUS_WAIT_TIMEOUT", "SCORE_SOFTMAX", "SCORE_SIGMOID", "MoeLayer", "ExpertCache",
+    "moe_expert_cache_bytes",
 ]
 
 # bits of the device status word (moe_device_status)
@@ -101,9 +102,18 @@ _sigs = {
     "moe_tile_scales": [_P, ctypes.c_int64, ctypes.c_int32, _P, _P],
     "moe_selftest_bounded_wait": [_P, _P, ctypes.c_int, ctypes.c_uint32, _P],
 }
+_sigs.update({
+    "moe_expert_cache_create": [_D, ctypes.c_int32, _P, _Z, ctypes.POINTER(_P)],
+    "moe_expert_cache_destroy": [_P],
+    "moe_expert_cache_stats": [_P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                               ctypes.POINTER(ctypes.c_int64)],
+    "moe_expert_ffn_streamed": [_P, _D, _P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _Z, _P],
+})
 for _n, _a in _sigs.items():
     getattr(_lib, _n).argtypes = _a
     getattr(_lib, _n).restype = ctypes.c_int
+_lib.moe_expert_cache_bytes.restype = ctypes.c_size_t
+_lib.moe_expert_cache_bytes.argtypes = [_D, ctypes.c_int32]
 
 
 class MoeError(RuntimeError):
@@ -238,6 +248,60 @@ def moe_latent_down(dims, x, w_lat_down, x_lat, ws, stream=None):
 def moe_layer(dims, args: MoeLayerArgs, ws, stream=None):
     _check(_lib.moe_layer(ctypes.byref(dims), ctypes.byref(args), _ptr(ws), _nbytes(ws),
                           _stream(stream)))
+
+
+def moe_expert_cache_bytes(dims, slots: int) -> int:
+    return _lib.moe_expert_cache_bytes(ctypes.byref(dims), int(slots))
+
+
+class ExpertCache:
+    """An LRU cache of `slots` routed experts in device memory (one torch
+    buffer) in front of experts kept in host memory (moe_expert_cache_*).
+
+    host_experts: a sequence of E tuples (wg_q, wg_s, wu_q, wu_s, wd_q, wd_s)
+    of host tensors (page-locked for asynchronous copies) in the canonical
+    layout."""
+
+    def __init__(self, dims: MoeDims, slots: int, host_experts, device="cuda"):
+        self.dims = dims
+        nbytes = moe_expert_cache_bytes(dims, slots)
+        if nbytes == 0:
+            raise MoeError(2, _lib.moe_last_error().decode())
+        self.mem = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.mem.data_ptr()) % 256
+        self._host = list(host_experts)         # keeps the host tensors alive
+        ptrs = (ctypes.c_void_p * (6 * dims.E))()
+        for e, arrs in enumerate(self._host):
+            for a, t in enumerate(arrs):
+                ptrs[6 * e + a] = t.data_ptr()
+        self._ptrs = ptrs
+        h = ctypes.c_void_p()
+        _check(_lib.moe_expert_cache_create(ctypes.byref(dims), int(slots), self.mem.data_ptr() + off,
+                                            nbytes, ctypes.byref(h)))
+        self._h = h
+
+    def ffn(self, active, x_op, offsets, row_token, y_perm, ws, stream=None):
+        """moe_expert_ffn_streamed for the experts in `active` (host ints)."""
+        act = (ctypes.c_int32 * max(1, len(active)))(*[int(e) for e in active])
+        _check(_lib.moe_expert_ffn_streamed(self._h, ctypes.byref(self.dims), act, len(active),
+                                            _ptr(x_op), _ptr(offsets), _ptr(row_token), self._ptrs,
+                                            _ptr(y_perm), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+    def stats(self):
+        h, m, b = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib.moe_expert_cache_stats(self._h, ctypes.byref(h), ctypes.byref(m), ctypes.byref(b)))
+        return {"hits": h.value, "misses": m.value, "bytes_copied": b.value}
+
+    def close(self):
+        if self._h:
+            _lib.moe_expert_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ---------------------------------------------------------------------------

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "../../include/moe_mxfp4.h"
 #include "kernels.h"
@@ -993,6 +994,221 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
   if ((s = device_state(&ds)) != MOE_OK) return s;
   return do_expert_ffn(p, *ds, x_op, offsets, expert_list, row_token, wg_q, wg_s, wu_q, wu_s, wd_q,
                        wd_s, y_perm, ws, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// Routed experts streamed from host memory through an LRU cache of expert
+// slots in device memory (rabbit README: routed experts stay off the
+// accelerator and "stream on demand through a per-layer LRU cache"; its
+// feature list: per-expert early drain, an expert's matmul starts the moment
+// its own bytes land).
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+struct moe_expert_cache {
+  int dev = 0;
+  int32_t slots = 0;
+  int E = 0, I = 0, W = 0;
+  uint8_t* base = nullptr;              // slot 0; slot s at base + s * slot_bytes
+  size_t slot_bytes = 0;
+  size_t off[6] = {};                   // wg_q, wg_s, wu_q, wu_s, wd_q, wd_s inside a slot
+  size_t len[6] = {};
+  int32_t* one_list = nullptr;          // {1, 0}: the expert list of a one-expert problem
+  cudaStream_t copy = nullptr;          // the copy engine's stream
+  std::vector<int32_t> slot_expert;     // expert held by each slot (-1: none)
+  std::vector<int64_t> slot_used;       // last call that used each slot (LRU order)
+  std::vector<int32_t> expert_slot;     // slot of each expert (-1: not cached)
+  std::vector<cudaEvent_t> loaded;      // a slot's copy has landed
+  std::vector<cudaEvent_t> released;    // the last launch reading a slot has run
+  int64_t calls = 0, hits = 0, misses = 0, bytes = 0;
+  std::mutex mu;
+};
+
+namespace {
+
+// Byte layout of one slot: the six arrays of one expert, each at a 256-byte
+// boundary; the whole slot a multiple of 256 bytes.
+size_t cache_layout(int I, int W, size_t (&off)[6], size_t (&len)[6]) {
+  const size_t gq = (size_t)I * W / 2, gs = (size_t)I * W / 32;
+  const size_t l[6] = {gq, gs, gq, gs, gq, gs};   // down is [W, I]: the same sizes
+  size_t o = 0;
+  for (int i = 0; i < 6; ++i) {
+    off[i] = o;
+    len[i] = l[i];
+    o = align_up(o + l[i], 256);
+  }
+  return o;
+}
+
+const int32_t kOneList[2] = {1, 0};
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_expert_cache_bytes(const moe_dims* dims, int32_t slots) {
+  Plan p;
+  if (make_plan(dims, p) != MOE_OK || slots < 1) return 0;
+  size_t off[6], len[6];
+  return 256 + (size_t)slots * cache_layout(p.I, p.W, off, len);
+}
+
+moe_status moe_expert_cache_create(const moe_dims* dims, int32_t slots, void* dev_mem, size_t dev_bytes,
+                                   moe_expert_cache** out) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (p.mode != MOE_ACT_BF16)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "expert streaming serves MOE_ACT_BF16 (decode) layers");
+  if (slots < 1 || slots > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "slots=%d outside [1, 65536]", slots);
+  CHECK_PTR(dev_mem);
+  if (((uintptr_t)dev_mem & 255u) != 0) return fail(MOE_ERR_ALIGNMENT, "dev_mem not 256-byte aligned");
+  if (dev_bytes < moe_expert_cache_bytes(dims, slots))
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "dev_mem %zu bytes < %zu needed", dev_bytes,
+                moe_expert_cache_bytes(dims, slots));
+  moe_expert_cache* c = new moe_expert_cache;
+  cudaGetDevice(&c->dev);
+  c->slots = slots;
+  c->E = p.E; c->I = p.I; c->W = p.W;
+  c->one_list = static_cast<int32_t*>(dev_mem);
+  c->base = static_cast<uint8_t*>(dev_mem) + 256;
+  c->slot_bytes = cache_layout(p.I, p.W, c->off, c->len);
+  c->slot_expert.assign(slots, -1);
+  c->slot_used.assign(slots, -1);
+  c->expert_slot.assign(p.E, -1);
+  cudaError_t e = cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking);
+  c->loaded.assign(slots, nullptr);
+  c->released.assign(slots, nullptr);
+  for (int i = 0; i < slots && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&c->loaded[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->released[i], cudaEventDisableTiming);
+  }
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->one_list, kOneList, sizeof(kOneList), cudaMemcpyHostToDevice, c->copy);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->copy);
+  if (e != cudaSuccess) {
+    moe_expert_cache_destroy(c);
+    return fail(MOE_ERR_CUDA, "expert cache setup: %s", cudaGetErrorString(e));
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+moe_status moe_expert_cache_destroy(moe_expert_cache* c) {
+  if (!c) return MOE_OK;
+  if (c->copy) cudaStreamSynchronize(c->copy);
+  for (cudaEvent_t ev : c->loaded)
+    if (ev) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : c->released)
+    if (ev) cudaEventDestroy(ev);
+  if (c->copy) cudaStreamDestroy(c->copy);
+  delete c;
+  return MOE_OK;
+}
+
+moe_status moe_expert_cache_stats(const moe_expert_cache* c, int64_t* hits, int64_t* misses,
+                                  int64_t* bytes_copied) {
+  if (!c || !hits || !misses || !bytes_copied) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  moe_expert_cache* m = const_cast<moe_expert_cache*>(c);
+  std::lock_guard<std::mutex> lk(m->mu);
+  *hits = c->hits;
+  *misses = c->misses;
+  *bytes_copied = c->bytes;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn_streamed(moe_expert_cache* c, const moe_dims* dims, const int32_t* active,
+                                   int32_t n_active, const void* x_op, const int32_t* offsets,
+                                   const int32_t* row_token, const uint8_t* const* host_experts,
+                                   float* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, p);
+  if (s != MOE_OK) return s;
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cache is NULL");
+  if (p.E != c->E || p.I != c->I || p.W != c->W || p.mode != MOE_ACT_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "dims do not match the cache");
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != c->dev)
+    return fail(MOE_ERR_INVALID_ARG, "the cache belongs to device %d", c->dev);
+  CHECK_PTR(x_op); CHECK_PTR(offsets); CHECK_PTR(row_token); CHECK_PTR(host_experts); CHECK_PTR(y_perm);
+  if (n_active < 0 || n_active > p.E) return fail(MOE_ERR_INVALID_ARG, "n_active=%d outside [0, E]", n_active);
+  if (n_active > 0) CHECK_PTR(active);
+  if (n_active > c->slots)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%d active experts > %d cache slots", n_active, c->slots);
+  for (int i = 0; i < n_active; ++i) {
+    if (active[i] < 0 || active[i] >= p.E) return fail(MOE_ERR_INVALID_ARG, "active[%d]=%d outside [0, E)", i, active[i]);
+    for (int j = 0; j < i; ++j)
+      if (active[j] == active[i]) return fail(MOE_ERR_INVALID_ARG, "expert %d listed twice", active[i]);
+    for (int a = 0; a < 6; ++a)
+      if (!host_experts[(size_t)active[i] * 6 + a])
+        return fail(MOE_ERR_INVALID_ARG, "host_experts[%d][%d] is NULL", active[i], a);
+  }
+  if ((s = check_ws(p, ws, ws_bytes)) != MOE_OK) return s;
+  DeviceState* ds;
+  if ((s = device_state(&ds)) != MOE_OK) return s;
+  // each expert runs as a one-expert problem: offsets shifted to its pair of
+  // entries, the expert list {1, 0}, the weights of its slot (extent E = 1);
+  // the workspace layout stays the full plan's (rows are global row ids)
+  Plan p1 = p;
+  p1.E = 1;
+  const cudaStream_t st = (cudaStream_t)stream;
+  std::lock_guard<std::mutex> lk(c->mu);
+  const int64_t call = ++c->calls;
+  // 1) slots: hits keep theirs; misses take the least recently used slot
+  //    that this call does not use, and are copied in list order
+  std::vector<int32_t> slot_of(n_active, -1);
+  std::vector<char> miss(n_active, 0);
+  for (int i = 0; i < n_active; ++i) {
+    const int e = active[i];
+    if (c->expert_slot[e] >= 0) {
+      slot_of[i] = c->expert_slot[e];
+      c->slot_used[slot_of[i]] = call;
+      ++c->hits;
+    }
+  }
+  cudaError_t err = cudaSuccess;
+  for (int i = 0; i < n_active && err == cudaSuccess; ++i) {
+    if (slot_of[i] >= 0) continue;
+    int best = -1;
+    for (int t = 0; t < c->slots; ++t)
+      if (c->slot_used[t] != call && (best < 0 || c->slot_used[t] < c->slot_used[best])) best = t;
+    const int e = active[i];
+    if (c->slot_expert[best] >= 0) c->expert_slot[c->slot_expert[best]] = -1;
+    c->slot_expert[best] = e;
+    c->expert_slot[e] = best;
+    c->slot_used[best] = call;
+    slot_of[i] = best;
+    miss[i] = 1;
+    ++c->misses;
+    // the copy overwrites the slot only after the last launch that read it
+    uint8_t* dst = c->base + (size_t)best * c->slot_bytes;
+    err = cudaStreamWaitEvent(c->copy, c->released[best], 0);
+    for (int a = 0; a < 6 && err == cudaSuccess; ++a) {
+      err = cudaMemcpyAsync(dst + c->off[a], host_experts[(size_t)e * 6 + a], c->len[a],
+                            cudaMemcpyHostToDevice, c->copy);
+      c->bytes += (int64_t)c->len[a];
+    }
+    if (err == cudaSuccess) err = cudaEventRecord(c->loaded[best], c->copy);
+  }
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "expert copy: %s", cudaGetErrorString(err));
+  // 2) each expert's FFN as soon as its own bytes have landed (cache hits at
+  //    once), in list order on the caller's stream
+  for (int i = 0; i < n_active; ++i) {
+    const int e = active[i];
+    const int t = slot_of[i];
+    uint8_t* b = c->base + (size_t)t * c->slot_bytes;
+    if ((err = cudaStreamWaitEvent(st, c->loaded[t], 0)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "expert wait: %s", cudaGetErrorString(err));
+    if ((s = do_expert_ffn(p1, *ds, x_op, offsets + e, c->one_list, row_token, b + c->off[0],
+                           b + c->off[1], b + c->off[2], b + c->off[3], b + c->off[4], b + c->off[5],
+                           y_perm, ws, st)) != MOE_OK)
+      return s;
+    if ((err = cudaEventRecord(c->released[t], st)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "expert release: %s", cudaGetErrorString(err));
+  }
+  return MOE_OK;
 }
 
 moe_status moe_combine(const moe_dims* dims, const float* y_perm, const int32_t* slot_row,

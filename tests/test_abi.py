@@ -149,3 +149,21 @@ def test_selftest_bounded_wait_validates_arguments():
     assert lib.moe_selftest_bounded_wait(FAKE, FAKE + 4, 1, 16, None) == 3      # misaligned source
     assert lib.moe_selftest_bounded_wait(FAKE, None, 0, 0, None) == 1           # limit 0
     assert lib.moe_selftest_bounded_wait(FAKE, None, 0, 5000, None) == 1        # limit too large
+
+
+def test_expert_cache_validates_arguments():
+    d = _dims()
+    assert M.moe_expert_cache_bytes(d, 0) == 0
+    assert M.moe_expert_cache_bytes(_dims(T=0), 4) == 0
+    n = M.moe_expert_cache_bytes(d, 4)
+    assert n > 4 * 3 * (128 * 256 // 2) and n % 256 == 0
+    out = ctypes.c_void_p()
+    lib = M._lib
+    assert lib.moe_expert_cache_create(ctypes.byref(d), 4, None, n, ctypes.byref(out)) == 1
+    assert lib.moe_expert_cache_create(ctypes.byref(d), 4, FAKE + 16, n, ctypes.byref(out)) == 3
+    assert lib.moe_expert_cache_create(ctypes.byref(d), 4, FAKE, n - 1, ctypes.byref(out)) == 4
+    assert lib.moe_expert_cache_create(ctypes.byref(_dims(act_mode=1)), 4, FAKE, n,
+                                       ctypes.byref(out)) == 2
+    assert lib.moe_expert_ffn_streamed(None, ctypes.byref(d), None, 0, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, M.moe_workspace_size(d), None) == 1
+    assert lib.moe_expert_cache_destroy(None) == 0
