@@ -709,10 +709,10 @@ def main():
         w = dataclasses.replace(w, E=args.experts, name=f"{w.name}-E{args.experts}")
     if args.tokens:
         w = dataclasses.replace(w, T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    if args.workload != "decode1":
+        args.streamed = False
     if args.no_extra or args.experts or args.tokens:
         args.extra = []
-        args.streamed = False
-    if args.workload != "decode1":
         args.streamed = False
     elif args.extra is None:
         args.extra = list(EXTRA_DEFAULT) if args.workload == "decode1" else []

@@ -123,3 +123,24 @@ def test_reference_arm_never_maps_the_product_library(repo_root):
                          capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr
     assert res.stdout.split() == ["clean", "clean", "oracle"], res.stdout
+
+
+def test_bench_argument_defaults(monkeypatch, repo_root):
+    """The extras and the streamed line default per workload (no GPU needed:
+    main() is stopped before any measurement)."""
+    b = _bench()
+    seen = {}
+
+    def fake_run(args, w):
+        seen.update(extra=list(args.extra), streamed=args.streamed, name=w.name)
+        return None
+    monkeypatch.setattr(b, "run_ours", fake_run)
+    for argv, want in ((["bench.py"], (["decode32", "latent16", "prefill4096"], True, "decode1")),
+                       (["bench.py", "--workload", "prefill4096"], ([], False, "prefill4096")),
+                       (["bench.py", "--no-extra"], ([], False, "decode1")),
+                       (["bench.py", "--extra", "latent16"], (["latent16"], True, "decode1")),
+                       (["bench.py", "--no-streamed"], (["decode32", "latent16", "prefill4096"],
+                                                        False, "decode1"))):
+        monkeypatch.setattr(sys, "argv", argv)
+        b.main()
+        assert (seen["extra"], seen["streamed"], seen["name"]) == want, argv
