@@ -212,11 +212,10 @@ moe_status moe_route_noalloc(const moe_dims* dims, const uint16_t* x, const uint
  *     two that maps the row's largest magnitude into [2^14, 2^15).
  *   x_op format, MOE_ACT_MXFP4: ONE ROW PER PERMUTED ROW, ready for the tensor
  *     cores (offsets of the parts from moe_mxf4_layout_of):
- *       codes [T, W/2] uint8, ONE ROW PER TOKEN (low nibble = even element;
- *         OCP MX v1.0 conversion of the token's bf16 row, ties to even): the
- *         gate/up GEMM gathers the rows of each tile by row_token;
- *       E8M0 scales in the TILED layout below, K = W, one row per permuted
- *         row r (the scales of token row_token[r]);
+ *       codes [T*k, W/2] uint8 (low nibble = even element; OCP MX v1.0
+ *         conversion of the token's bf16 row, ties to even), row r = token
+ *         row_token[r];
+ *       E8M0 scales in the TILED layout below, K = W;
  *       the tile list: tiles[t] = {expert, first permuted row, rows, 0} int32x4,
  *         each expert's rows cut into tiles of at most tile_rows consecutive
  *         rows, experts in expert_list order; tile_base[e] int32 = the first

@@ -177,7 +177,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
     p.xop_bytes = p.xop_scale_off + (size_t)p.T * 4;
     p.xop_tiles_off = p.xop_tbase_off = p.xop_ntiles_off = 0;
   } else {
-    p.xop_scale_off = align_up((size_t)p.T * p.W / 2, 256);   // codes: one row per token
+    p.xop_scale_off = align_up((size_t)p.R * p.W / 2, 256);
     p.xop_tiles_off = align_up(p.xop_scale_off + (size_t)p.max_tiles * (p.W / 128) * 512, 256);
     p.xop_tbase_off = align_up(p.xop_tiles_off + (size_t)p.max_tiles * 16, 256);
     p.xop_ntiles_off = align_up(p.xop_tbase_off + (size_t)p.E * 4, 256);
@@ -635,7 +635,6 @@ moe_status join_before(cudaEvent_t ev, cudaStream_t st) {
 // the shared expert's stream there, well after that work is done, so that the
 // join never delays a launch)
 moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* x_op,
-                              const int32_t* row_token,
                               const uint8_t* wg_q, const uint8_t* wg_s, const uint8_t* wu_q,
                               const uint8_t* wu_s, const uint8_t* wd_q, const uint8_t* wd_s,
                               float* y_perm, void* ws, cudaStream_t st, cudaEvent_t join = nullptr) {
@@ -649,10 +648,9 @@ moe_status do_expert_ffn_mxf4(const Plan& p, const DeviceState& ds, const void* 
   memset(&g, 0, sizeof(g));
   if ((s = code_map(&g.map_a0, wg_q, (uint64_t)p.E * p.I, p.W / 2, 128, "gate weights")) != MOE_OK ||
       (s = code_map(&g.map_a1, wu_q, (uint64_t)p.E * p.I, p.W / 2, 128, "up weights")) != MOE_OK ||
-      (s = code_map(&g.map_b, static_cast<const uint8_t*>(x_op), (uint64_t)p.T, p.W / 2, 1,
-                    "token codes")) != MOE_OK)
+      (s = code_map(&g.map_b, static_cast<const uint8_t*>(x_op), (uint64_t)p.R, p.W / 2,
+                    moe::kTileRows, "token codes")) != MOE_OK)
     return s;
-  g.row_token = row_token;
   g.sa0 = wg_s; g.sa1 = wu_s;
   g.bs = at<uint8_t>(xop, p.xop_scale_off);
   g.tiles = tiles; g.n_tiles = n_tiles;
@@ -686,8 +684,7 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st,
                          cudaEvent_t join = nullptr) {
   if (p.mode == MOE_ACT_MXFP4)
-    return do_expert_ffn_mxf4(p, ds, x_op, row_token, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st,
-                              join);
+    return do_expert_ffn_mxf4(p, ds, x_op, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st, join);
   const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
   moe::GateUpArgs g;
   g.x16 = static_cast<const __half*>(x_op);

@@ -13,14 +13,10 @@
 // about the same time (once from HBM, then from L2).
 //
 // Every operand arrives by TMA on one mbarrier per stage (no generic-proxy
-// copies on the data path): weight codes as 2-D tensor tiles with the
-// 128-byte swizzle (rows of 128 bytes = 256 elements of K); token codes for
-// gate/up gathered row by row from the one quantised copy of each token
-// (tile::gather4: four token rows per copy, rows chosen by row_token, into
-// the same swizzled tile), h codes for down as 2-D tiles of consecutive
-// permuted rows; the weight and token scales as contiguous 512-byte blocks of
-// the tiled scale layout (sf_tiled_offset), which tcgen05.cp moves into
-// tensor memory.
+// copies on the data path): weight codes and token codes as 2-D tensor tiles
+// with the 128-byte swizzle (rows of 128 bytes = 256 elements of K), the
+// weight and token scales as contiguous 512-byte blocks of the tiled scale
+// layout (sf_tiled_offset), which tcgen05.cp moves into tensor memory.
 //
 // Each stage carries two 128-row weight tiles that share the token tile (gate
 // and up rows for gate/up, two consecutive row tiles of Wd for down): two
@@ -77,7 +73,7 @@ static_assert(Shape<true>::kStageBytes % 1024 == 0 && Shape<false>::kStageBytes 
               "stages must keep the 1024-byte alignment of the swizzled tiles");
 static_assert(Shape<true>::kColSfb + 8 <= kTmemCols && Shape<false>::kColSfb + 8 <= kTmemCols,
               "tensor memory columns");
-static_assert(kTileRows % 16 == 0 && kTileRows <= 128 && kTileRows / 4 <= 32, "tile rows");
+static_assert(kTileRows % 16 == 0 && kTileRows <= 128, "tile rows");
 
 // MXFP4 encoding of 32 fp32 values (one block): 16 bytes of codes (element
 // 2j in the low nibble of byte j) and the E8M0 scale code. Same rule as the
@@ -241,67 +237,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    // lane 0 arms the stages and loads the weights, the scales and (down)
-    // the h tile; gate/up: lanes 0 .. kTileRows/4 - 1 gather four token rows
-    // each (rows past the tile's count repeat its first row: those result
-    // columns are never stored)
-    constexpr int kGather = kTileRows / 4;
-    uint32_t last_ph[kStages];
-    bool filled[kStages];
+    if (lane == 0) {
+      uint32_t last_ph[kStages];
+      bool filled[kStages];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) { last_ph[s] = 0; filled[s] = false; }
-    int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (long q = blockIdx.x; q < items && ok; q += gridDim.x) {
-      const Item it = item_of(q, NT, a.tiles);
-      const int ya = it.tile.x * a.M + it.mt * (kGateUp ? 128 : 256);
-      const bool two = kGateUp || it.mt * 256 + 128 < a.M;
-      const uint8_t* sfa0 = a.sa0 + ((size_t)(ya / 128) * k128) * 512;
-      const uint8_t* sfa1 = kGateUp ? a.sa1 + ((size_t)(ya / 128) * k128) * 512
-                                    : sfa0 + (size_t)k128 * 512;
-      const uint8_t* sfb = a.bs + ((size_t)it.t * k128) * 512;
-      int rt[4] = {0, 0, 0, 0};
-      if (kGateUp && lane < kGather) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int n = 4 * lane + i;
-          rt[i] = __ldg(a.row_token + it.tile.y + (n < it.tile.z ? n : 0));
-        }
-      }
-      for (int kt = 0; kt < KT; ++kt) {
-        int okw = 0;
-        if (lane == 0) okw = tc::wait_or_abort(&empty[s], ph ^ 1u, abort) ? 1 : 0;
-        if (!__shfl_sync(0xFFFFFFFFu, okw, 0)) { ok = false; break; }
-        uint8_t* st = smem + s * S::kStageBytes;
-        if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) { last_ph[s] = 0; filled[s] = false; }
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (long q = blockIdx.x; q < items && ok; q += gridDim.x) {
+        const Item it = item_of(q, NT, a.tiles);
+        const int ya = it.tile.x * a.M + it.mt * (kGateUp ? 128 : 256);
+        const bool two = kGateUp || it.mt * 256 + 128 < a.M;
+        const uint8_t* sfa0 = a.sa0 + ((size_t)(ya / 128) * k128) * 512;
+        const uint8_t* sfa1 = kGateUp ? a.sa1 + ((size_t)(ya / 128) * k128) * 512
+                                      : sfa0 + (size_t)k128 * 512;
+        const uint8_t* sfb = a.bs + ((size_t)it.t * k128) * 512;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!tc::wait_or_abort(&empty[s], ph ^ 1u, abort)) { ok = false; break; }
+          uint8_t* st = smem + s * S::kStageBytes;
           const uint32_t sf_bytes = (kt == KT - 1 && kb_last == 2) ? 512u : 1024u;
           const int na = two ? 2 : 1;
           mbar_expect_tx(&full[s], na * kATileBytes + kBTileBytes + (na + 1) * sf_bytes);
           tc::tma_load_2d(st, &a.map_a0, kt * 128, ya, &full[s]);
           if (kGateUp) tc::tma_load_2d(st + kATileBytes, &a.map_a1, kt * 128, ya, &full[s]);
           else if (two) tc::tma_load_2d(st + kATileBytes, &a.map_a0, kt * 128, ya + 128, &full[s]);
-          if (!kGateUp) tc::tma_load_2d(st + S::kOffB, &a.map_b, kt * 128, it.tile.y, &full[s]);
+          tc::tma_load_2d(st + S::kOffB, &a.map_b, kt * 128, it.tile.y, &full[s]);
           bulk_g2s(st + S::kOffSfa, sfa0 + kt * 1024, sf_bytes, &full[s]);
           if (two) bulk_g2s(st + S::kOffSfa + kSfBytes, sfa1 + kt * 1024, sf_bytes, &full[s]);
           bulk_g2s(st + S::kOffSfb, sfb + kt * 1024, sf_bytes, &full[s]);
+          last_ph[s] = ph;
+          filled[s] = true;
+          if (++s == kStages) { s = 0; ph ^= 1u; }
         }
-        if (kGateUp) {
-          __syncwarp();                        // the stage is armed before any row lands
-          if (lane < kGather)
-            tc::tma_gather4(st + S::kOffB + lane * 512, &a.map_b, kt * 128, rt[0], rt[1], rt[2],
-                            rt[3], &full[s]);
-        }
-        last_ph[s] = ph;
-        filled[s] = true;
-        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
-    }
-    __syncwarp();
-    if (lane == 0 && *abort) {     // let every issued copy land before the CTA can exit
+      if (*abort) {     // let every issued copy land before the CTA can exit
 #pragma unroll
-      for (int s2 = 0; s2 < kStages; ++s2)
-        if (filled[s2]) mbar_wait(&full[s2], last_ph[s2]);
+        for (int s2 = 0; s2 < kStages; ++s2)
+          if (filled[s2]) mbar_wait(&full[s2], last_ph[s2]);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------

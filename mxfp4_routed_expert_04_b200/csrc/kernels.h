@@ -113,14 +113,12 @@ constexpr int kTileRows = 112;
 struct Mxf4GemmArgs {
   CUtensorMap map_a0;        // gate/up: gate weights; down: down weights
   CUtensorMap map_a1;        // gate/up: up weights
-  CUtensorMap map_b;         // gate/up: x codes [T, K/2] in one-row boxes, rows gathered by
-                             // row_token; down: h codes [R, K/2] in boxes of kTileRows rows
+  CUtensorMap map_b;         // token codes: x rows (gate/up) or h rows (down), [R, K/2]
   const uint8_t* sa0;        // tiled weight scales
   const uint8_t* sa1;
   const uint8_t* bs;         // tiled token scales
   const int4* tiles;         // k_tile_list output
   const int32_t* n_tiles;
-  const int32_t* row_token;  // gate/up: token of each permuted row (the gather); down: NULL
   uint8_t* hq;               // gate/up out: h codes [R, M/2]
   uint8_t* hs;               // gate/up out: h scales, tiled (K = M)
   float* y;                  // down out: y_perm [R, M]

@@ -218,11 +218,11 @@ __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__
 
 // grid T, block 256; W a multiple of 128. MXFP4 activation operand of the
 // tensor-core path: token t's row quantised block by block (the conversion in
-// the file header); the codes once, to q[t] (the gate/up GEMM gathers the
-// rows of a tile by row_token), the scales for each of its k permuted rows
-// r = slot_row[t, j] into the tiled layout at (tile, n) of row r (tile_base
-// from k_tile_list, tiles of kTileRows consecutive rows of one expert).
-// Writes nothing when the permutation was rejected (expert_list[0] == 0 then).
+// the file header) and written to each of its k permuted rows
+// r = slot_row[t, j]: codes to q[r] and scales into the tiled layout at
+// (tile, n) of row r (tile_base from k_tile_list, tiles of kTileRows
+// consecutive rows of one expert). Writes nothing when the permutation was
+// rejected (expert_list[0] == 0 then).
 __global__ void __launch_bounds__(256) k_act_to_mxfp4_perm(
     const uint16_t* __restrict__ x, int W, int k, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ slot_row, const int32_t* __restrict__ offsets,
@@ -273,9 +273,10 @@ __global__ void __launch_bounds__(256) k_act_to_mxfp4_perm(
       packed |= c << (4 * j);
     }
     if (ok) {
-      *reinterpret_cast<uint32_t*>(q + (size_t)tok * (W / 2) + i / 2) = packed;
-      if ((threadIdx.x & 3) == 0)
-        for (int j = 0; j < k; ++j) sf[sf_tiled_offset(s_tile[j], k128, s_n[j], i / 32)] = (uint8_t)code_s;
+      for (int j = 0; j < k; ++j) {
+        *reinterpret_cast<uint32_t*>(q + (size_t)s_row[j] * (W / 2) + i / 2) = packed;
+        if ((threadIdx.x & 3) == 0) sf[sf_tiled_offset(s_tile[j], k128, s_n[j], i / 32)] = (uint8_t)code_s;
+      }
     }
   }
 }

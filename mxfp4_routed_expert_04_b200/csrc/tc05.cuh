@@ -125,17 +125,6 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64
         "r"(smem_u32(bar))
       : "memory");
 }
-// Four rows r0..r3 of a 2-D map whose box is one row high, at column x,
-// into 4 consecutive box rows at dst (TMA tile::gather4).
-MOE_DEV void tma_gather4(void* dst, const CUtensorMap* map, int x, int r0, int r1, int r2, int r3,
-                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1),
-        "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
 MOE_DEV void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

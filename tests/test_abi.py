@@ -120,7 +120,7 @@ def test_mxf4_layout_only_for_mxfp4_activations():
     # x_op parts in order, 256-byte aligned, inside moe_x_op_size
     parts = [lay.x_codes, lay.x_scales, lay.tiles, lay.tile_base, lay.n_tiles]
     assert parts == sorted(parts) and all(o % 256 == 0 for o in parts)
-    assert lay.x_scales >= d1.T * W // 2                # codes: one row per token
+    assert lay.x_scales >= R * W // 2
     assert lay.tiles >= lay.x_scales + lay.max_tiles * (W // 128) * 512
     assert lay.n_tiles + 4 <= M.moe_x_op_size(d1)
     # h regions inside the workspace, disjoint

@@ -87,7 +87,7 @@ def _mxf4_operands(run, gpu):
     n_tiles = int(xo[lay.n_tiles:lay.n_tiles + 4].view(np.int32)[0])
     tiles = xo[lay.tiles:lay.tiles + 16 * n_tiles].view(np.int32).reshape(n_tiles, 4)
     tile_base = xo[lay.tile_base:lay.tile_base + 4 * w.E].view(np.int32)
-    x_codes = xo[:w.T * w.W // 2].reshape(w.T, w.W // 2)      # one row per token (gathered)
+    x_codes = xo[:R * w.W // 2].reshape(R, w.W // 2)
     x_scales = _untile(xo[lay.x_scales:], tiles, R, w.W)
     ws = L.ws
     h_codes = ws[lay.h_codes:lay.h_codes + R * w.I // 2].cpu().numpy().reshape(R, w.I // 2)
@@ -160,13 +160,11 @@ def test_tile_list(case):
 
 
 def test_x_operand_bit_exact(case):
-    """Token t's codes are the MXFP4 encoding of its row (once per token; the
-    gate/up GEMM gathers them by row_token), and every permuted row r holds
-    the scales of token row_token[r] in the tiled layout."""
+    """Every permuted row r holds the MXFP4 encoding of token row_token[r]."""
     w, sample, run, gpu = case
     codes, scales = O.mxfp4_quantize(O.bf16_to_f64(run.dense["x"]))
     tok = gpu["row_token"]
-    np.testing.assert_array_equal(gpu["x_codes"], O.mxfp4_pack(codes))
+    np.testing.assert_array_equal(gpu["x_codes"], O.mxfp4_pack(codes)[tok])
     np.testing.assert_array_equal(gpu["x_scales"], scales[tok])
 
 
