@@ -62,6 +62,11 @@ int tc_splits(long units, int K, size_t split_bytes) {
   return S;
 }
 
+// 32-bit word of the 256-byte status region (cleared by moe_workspace_init)
+// where the one-token launch's counters start: kRouted1SyncWords words
+constexpr int kSyncWord = 16;
+static_assert(4 * (kSyncWord + moe::kRouted1SyncWords) <= 256, "counters inside the status region");
+
 struct Plan {
   int T, H, I, E, k, Is, L, W, R, mode;
   moe::RouteCfg rc;          // router variant (bias pointer filled per call)
@@ -150,7 +155,7 @@ moe_status make_plan(const moe_dims* d, Plan& p) {
                : 0;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 256); return r; };
-  p.off_status = take(256);
+  p.off_status = take(256);            // status word, then (from int kSyncWord) the one-token counters
   // + the sigmoid-gate column (+ the latent down-projection columns on the
   // tcgen05 GEMM)
   p.off_router = take((size_t)p.S_router * p.T * (p.E + 1 + (p.rows ? 0 : p.L)) * 4);
@@ -355,6 +360,43 @@ FmaPlan fma_plan(int K, bool gate_up) {
 }
 // the CUDA-core path serves single-token experts when both projections fit it
 bool fma_path(const Plan& p) { return fma_plan(p.W, true).g.ok && fma_plan(p.I, false).g.ok; }
+
+// one token: the CUDA-core path in one launch, when its down role's two h
+// buffers fit beside the ring
+bool routed1_path(const Plan& p) {
+  if (p.T != 1 || p.k > moe::kRouted1MaxK) return false;
+  moe::FmaGeometry gg, gd;
+  moe::routed1_geometry(p.W, p.I, (size_t)MOE_FMA_SMEM_KB * 1024, gg, gd);
+  return gg.ok;
+}
+
+// One token: both projections of its experts in one launch (k_fma_routed1),
+// one CTA per SM taking chunks from the counters in the status region.
+moe_status launch_routed1(const DeviceState& ds, const Plan& p, const moe::FmaArgs& a, cudaStream_t st) {
+  const char* what = "expert gate/up + down (cuda cores, one launch)";
+  moe::FmaGeometry gg, gd;
+  moe::routed1_geometry(a.W, a.I, (size_t)MOE_FMA_SMEM_KB * 1024, gg, gd);
+  const int bg = fma_plan(a.W, true).bpl, bd = fma_plan(a.I, false).bpl;
+  if (!gg.ok || !bg || !bd) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: no geometry", what);
+  using K = void (*)(moe::FmaArgs, moe::FmaGeometry, moe::FmaGeometry);
+  static const K table[4][4] = {
+      {moe::k_fma_routed1<1, 1, 8>, moe::k_fma_routed1<1, 2, 4>, moe::k_fma_routed1<1, 4, 2>, moe::k_fma_routed1<1, 8, 1>},
+      {moe::k_fma_routed1<2, 1, 8>, moe::k_fma_routed1<2, 2, 4>, moe::k_fma_routed1<2, 4, 2>, moe::k_fma_routed1<2, 8, 1>},
+      {moe::k_fma_routed1<4, 1, 8>, moe::k_fma_routed1<4, 2, 4>, moe::k_fma_routed1<4, 4, 2>, moe::k_fma_routed1<4, 8, 1>},
+      {moe::k_fma_routed1<8, 1, 8>, moe::k_fma_routed1<8, 2, 4>, moe::k_fma_routed1<8, 4, 2>, moe::k_fma_routed1<8, 8, 1>}};
+  auto idx = [](int bpl) { return bpl == 1 ? 0 : bpl == 2 ? 1 : bpl == 4 ? 2 : 3; };
+  const K kern = table[idx(bg)][idx(bd)];
+  if (gd.rps != (bd == 1 ? 8 : bd == 2 ? 4 : bd == 4 ? 2 : 1))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: down rows per warp %d", what, gd.rps);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)gg.smem_bytes);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s setup: %s", what, cudaGetErrorString(e));
+  const long n = std::min(p.E, p.k);
+  const long chunks = n * ((a.I + gg.units - 1) / gg.units + (a.W + gd.units - 1) / gd.units);
+  const int grid = (int)std::min<long>(ds.num_sms, std::max(1L, chunks));
+  launch_pdl(kern, dim3((unsigned)grid), dim3(32 * moe::kRouted1Warps), gg.smem_bytes, st, a, gg, gd);
+  return launched(what);
+}
 
 template <bool kGateUp>
 moe_status launch_fma(const DeviceState& ds, const moe::FmaArgs& a, cudaStream_t st) {
@@ -704,8 +746,14 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   f.wg_q = wg_q; f.wg_s = wg_s; f.wu_q = wu_q; f.wu_s = wu_s; f.wd_q = wd_q; f.wd_s = wd_s;
   f.y_perm = y_perm;
   f.status = at<int32_t>(ws, p.off_status);
+  f.sync = at<int32_t>(ws, p.off_status) + kSyncWord;
   f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
   g.min_tokens = fma ? 2 : 1;
+  if (fma && routed1_path(p)) {
+    // one token: every active expert has exactly one row; both projections in one launch
+    moe_status s = join_before(join, st);
+    return s != MOE_OK ? s : launch_routed1(ds, p, f, st);
+  }
   // one token: its k experts are distinct, so every active expert has exactly
   // one token and the tensor-core kernels would find no work
   const bool mma = !(fma && p.T == 1);

@@ -89,18 +89,31 @@ struct FmaArgs {
   const uint8_t *wg_q, *wg_s, *wu_q, *wu_s, *wd_q, *wd_s;
   float* y_perm;             // down: [R, W]
   int32_t* status;           // device status word
+  int32_t* sync;             // one-token launch: [0] finished CTAs, [1 + s] h row pairs of expert slot s
   int W, I, E, R;
 };
 // Launch geometry: rps rows per consumer warp of a down stage, units per stage
 // (gate/up: row pairs; down: rows), code_bytes = one matrix's codes of a
 // stage, sbuf_off / sbuf2_off = offsets of the E8M0 spans (the second:
 // gate/up only), nst ring stages, act_off = the activation row buffer.
+// act_stride: the one-token launch's down role keeps two f16 h buffers
+// (f16 row, then K/32 fp32 block scales) act_stride bytes apart.
 struct FmaGeometry {
   int ok, rps, nst, units;
-  uint32_t code_bytes, sbuf_off, sbuf2_off, stage_bytes, act_off, smem_bytes;
+  uint32_t code_bytes, sbuf_off, sbuf2_off, stage_bytes, act_off, smem_bytes, act_stride;
 };
-FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget);
+FmaGeometry fma_geometry(int K, bool gate_up, size_t smem_budget, bool routed1 = false);
 template <int BPL, bool kGateUp, int RPS> __global__ void k_fma_gemv(FmaArgs a, FmaGeometry g);
+// One token: gate/up and down of all its experts in one launch, chunks taken
+// from device counters (gate/up first); gg / gd share the ring (stage_bytes,
+// nst) and the activation region (act_off). sync holds 3 + kRouted1MaxK words.
+constexpr int kRouted1MaxK = 32;     // experts of the token (k <= 32)
+constexpr int kRouted1SyncWords = 3 + kRouted1MaxK;
+constexpr int kRouted1Warps = kFmaConsumers + 2;   // producer, consumers, signal warp
+template <int BG, int BD, int RPSD>
+__global__ void k_fma_routed1(FmaArgs a, FmaGeometry gg, FmaGeometry gd);
+// the common geometry of k_fma_routed1 (ok = 0 when it does not fit)
+void routed1_geometry(int W, int I, size_t smem_budget, FmaGeometry& gg, FmaGeometry& gd);
 
 // --- grouped MXFP4 GEMM on tcgen05 (many tokens per expert) ----------------
 // Token rows are grouped in tiles of at most kTileRows consecutive permuted

@@ -11,6 +11,7 @@ oracle on the same seeded inputs:
 * activation operand exact (bf16 -> f16 with a power-of-two row scale);
 * expert outputs, shared expert and the layer output: max |err| <= 1e-2 x RMS.
 """
+import dataclasses
 import gc
 
 import numpy as np
@@ -383,3 +384,37 @@ def test_router_variant_selection_differs_from_softmax():
         plain = O.route(lg, w.k)[0]
         var = O.route(lg, w.k, **route_kw(w, d))[0]
         assert not np.array_equal(np.sort(plain, axis=1), np.sort(var, axis=1)), w.name
+
+
+def test_one_token_launch_clears_its_counters():
+    """One token runs both expert projections in one launch whose roles hand
+    h over through per-expert counters in the workspace's status region; the
+    last CTA puts them back to zero. Calls in a row (different inputs, the
+    stage calls and the fused layer) each match the oracle, leave the status
+    word clear and the counters at zero, and a repeated input gives the same
+    bits."""
+    import mxfp4_routed_expert_04_b200 as M
+    w = ROWS_T1
+    run = DeviceRun(w)
+    L = run.layer
+    counters = slice(64, 64 + 4 * 33)
+    first = None
+    for i in range(3):
+        d = dict(run.dense)
+        if i:       # another token (other experts), the same weights
+            d["x"] = synth.dense_inputs(dataclasses.replace(w, seed=w.seed + 7 * i))["x"]
+        run.dev["x"].copy_(torch.from_numpy(d["x"].view(np.int16)).cuda())
+        gpu = run.run_stages()
+        assert M.moe_device_status(L.ws) == 0
+        assert not L.ws[counters].any()
+        tie = np.any(O.route(O.router_logits(d["x"], d["w_router"]), w.k)[2])
+        ref = O.moe_layer(d, w.k, expert_getter(w), idx_override=gpu["idx"] if tie else None)
+        err, _ = max_rel_err(gpu["y"], ref["y"])
+        assert err <= TOL, (i, err)
+        y_layer = run.run_layer()
+        assert not L.ws[counters].any()
+        np.testing.assert_array_equal(y_layer, gpu["y"])
+        if i == 0:
+            first = gpu["y_perm"]
+    run.dev["x"].copy_(torch.from_numpy(run.dense["x"].view(np.int16)).cuda())
+    np.testing.assert_array_equal(run.run_stages()["y_perm"], first)
