@@ -292,7 +292,8 @@ def measure(args, w, steps, rank, local_rank, world, act=None):
     # (dispatch, activation operand), combine 1; shared expert 3 (gate/up,
     # SwiGLU finaliser, down), or 2 for one token on the row GEMV and for 128+
     # tokens (SwiGLU in the GEMM epilogue); routed experts 4 or 5 (bf16: two
-    # GEMV pairs; 2 for one token, whose experts all have a single token) or 3
+    # GEMV pairs; 1 for one token, whose experts all have a single token and
+    # run both projections in one launch) or 3
     # (mxfp4: tile list + two tcgen05 GEMMs); latent projections 3 (the down
     # projection rides with the router rows; its bf16 rounding, the routed sum
     # at width L, the up-projection GEMM)
@@ -310,7 +311,7 @@ def measure(args, w, steps, rank, local_rank, world, act=None):
     # writes the dispatch and the activation operand)
     fused_dispatch = w.T == 1 and act == "bf16" and not w.L
     launches_per_step = (5 - (1 if fused_combine else 0) - (2 if fused_dispatch else 0) + shared
-                         + (3 if act == "mxfp4" else (2 if w.T == 1 else routed_multi)) + (3 if w.L else 0))
+                         + (3 if act == "mxfp4" else (1 if w.T == 1 else routed_multi)) + (3 if w.L else 0))
 
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -45,6 +45,11 @@ bool rows_k_ok(int K) { return K == 1024 || K == 2048 || K == 4096 || K == 8192;
 bool rows_path_for(int T, int H, int Is) { return T == 1 && rows_k_ok(H) && rows_k_ok(Is); }
 constexpr size_t kRowsSmemBudget = 220 * 1024;
 constexpr int kRowsFreeSMs = 8;     // SMs a side-stream row GEMV leaves to the routing chain
+// one token: the router row GEMV (8.4 MB at decode1) takes 3/8 of the SMs,
+// and in moe_layer the shared expert's first half (67 MB) the others from the
+// start, so that both end close to when the top-k does (with all SMs for the
+// router, the shared expert starts only as the router's CTAs leave)
+constexpr int kLayerRouterEighths = 3;
 
 // Token tile of the tcgen05 bf16 GEMM: the MMA's N, a multiple of 16 up to 128.
 int tc_tile_tokens(int T) { return T >= 128 ? 128 : (T + 15) / 16 * 16; }
@@ -298,16 +303,20 @@ moe_status device_state(DeviceState** out) {
 
 // single-token row GEMV: one CTA per SM (at most max_ctas), ring depth from
 // the shared-memory budget
-moe_status launch_rows(const DeviceState& ds, moe::RowsArgs& r, bool swiglu, bool x_f32, int max_ctas,
-                       cudaStream_t st, const char* what, bool pdl = true) {
-  const long units = swiglu ? r.rows[0] : (long)r.rows[0] + r.rows[1] + r.rows[2];
-  const int grid = (int)std::max<long>(1, std::min<long>(units, max_ctas));
-  // slots of a stage: the units of a CTA rounded up to a power of two (at
-  // most 16 MMA rows), so that a CTA's few rows come in whole-row stages
+// slots of a stage: the units of a CTA rounded up to a power of two (at most
+// 16 MMA rows), so that a CTA's few rows come in whole-row stages; the slots
+// set the K chunk of a stage and so the order of each row's sum
+int rows_slots(long units, int grid, bool swiglu) {
   const long per = (units + grid - 1) / grid;
   int pp = 1;
   while (pp < per && pp < (swiglu ? 8 : 16)) pp <<= 1;
-  r.slots = swiglu ? 2 * pp : pp;
+  return swiglu ? 2 * pp : pp;
+}
+moe_status launch_rows(const DeviceState& ds, moe::RowsArgs& r, bool swiglu, bool x_f32, int max_ctas,
+                       cudaStream_t st, const char* what, bool pdl = true, int force_slots = 0) {
+  const long units = swiglu ? r.rows[0] : (long)r.rows[0] + r.rows[1] + r.rows[2];
+  const int grid = (int)std::max<long>(1, std::min<long>(units, max_ctas));
+  r.slots = force_slots > 0 ? force_slots : rows_slots(units, grid, swiglu);
   r.nst = moe::rows_stages(r.K, r.slots, x_f32, kRowsSmemBudget);
   if (!r.nst) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: K=%d too long for the row GEMV", what, r.K);
   const size_t smem = (size_t)r.nst * moe::rows_stage_bytes(r.K, r.slots) + moe::rows_act_bytes(r.K, x_f32);
@@ -364,7 +373,7 @@ bool fma_path(const Plan& p) { return fma_plan(p.W, true).g.ok && fma_plan(p.I, 
 // one token: the CUDA-core path in one launch, when its down role's two h
 // buffers fit beside the ring
 bool routed1_path(const Plan& p) {
-  if (p.T != 1 || p.k > moe::kRouted1MaxK) return false;
+  if (p.T != 1 || p.k > moe::kRouted1MaxK || p.mode != MOE_ACT_BF16 || !fma_path(p)) return false;
   moe::FmaGeometry gg, gd;
   moe::routed1_geometry(p.W, p.I, (size_t)MOE_FMA_SMEM_KB * 1024, gg, gd);
   return gg.ok;
@@ -507,12 +516,21 @@ moe_status round_latent(const Plan& p, const float* part, int ld, uint16_t* x_la
 // rounded to bf16 into x_lat after the top-k).
 // (fuse: one token in bf16 mode, the top-k launch also writes the dispatch
 // and the activation operand; moe_permute is then skipped)
+// one token: the router row GEMV's CTAs, and its stage slots for the rows it
+// carries in moe_layer (router, sigmoid gate, latent down); the sigmoid-gate
+// row alone uses the same slots, so that it has the same bits either way
+int router_ctas(const DeviceState& ds) { return std::max(1, ds.num_sms * kLayerRouterEighths / 8); }
+int router_slots(const Plan& p, const DeviceState& ds) {
+  const long units = (long)p.E + 1 + p.L;
+  return rows_slots(units, (int)std::min<long>(units, router_ctas(ds)), false);
+}
+
 moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, const uint16_t* wr,
                     const float* e_bias, int32_t* idx, float* w, float* logits, void* ws,
                     cudaStream_t st, const uint16_t* w_sgate = nullptr,
                     const uint16_t* w_ld = nullptr, uint16_t* x_lat = nullptr,
                     const moe::TopkFuse* fuse = nullptr) {
-  const moe::TopkFuse tf = fuse ? *fuse : moe::TopkFuse{};
+  moe::TopkFuse tf = fuse ? *fuse : moe::TopkFuse{};
   moe::RouteCfg rc = p.rc;
   rc.bias = e_bias;
   float* part = at<float>(ws, p.off_router);
@@ -525,7 +543,17 @@ moe_status do_route(const Plan& p, const DeviceState& ds, const uint16_t* x, con
     if (w_sgate) { r.w[seg] = w_sgate; r.rows[seg] = 1; r.out[seg] = at<float>(ws, p.off_gl); ++seg; }
     if (w_ld) { r.w[seg] = w_ld; r.rows[seg] = p.L; r.out[seg] = at<float>(ws, p.off_ld); }
     r.x = x; r.K = p.H; r.status = at<int32_t>(ws, p.off_status);
-    if ((s = launch_rows(ds, r, false, false, ds.num_sms, st, "router gemv")) != MOE_OK) return s;
+    if (tf.x16 && p.H == tf.W) {
+      // one token: the router launch writes the activation operand (its CTAs
+      // hold x already, and it runs before the shared expert loads HBM)
+      r.x16 = tf.x16; r.xscale = tf.xscale;
+      tf.x16 = nullptr;
+    }
+    // (the same share of the SMs and stage geometry in moe_route and
+    // moe_layer, so that both give the same bits)
+    if ((s = launch_rows(ds, r, false, false, router_ctas(ds), st, "router gemv", true,
+                         router_slots(p, ds))) != MOE_OK)
+      return s;
     launch_pdl(moe::k_topk, dim3(p.T), dim3(moe::kTopkThreads), 0, st, (const float*)part, 1, p.T, p.E,
                p.E, p.k, idx, w, logits, (float*)nullptr, tf, rc);
     if ((s = launched("top-k")) != MOE_OK) return s;
@@ -572,7 +600,7 @@ moe_status do_shared_up(const Plan& p, const DeviceState& ds, const uint16_t* x,
     memset(&g, 0, sizeof(g));
     g.w[0] = w_sgate; g.rows[0] = 1; g.out[0] = at<float>(ws, p.off_gl);
     g.x = x; g.K = p.H; g.status = r.status;
-    return launch_rows(ds, g, false, false, 1, st, "shared gate gemv");
+    return launch_rows(ds, g, false, false, 1, st, "shared gate gemv", true, router_slots(p, ds));
   }
   uint16_t* h_hi = at<uint16_t>(ws, p.off_hsb);
   uint16_t* h_lo = h_hi + (size_t)p.T * p.Is;
@@ -1331,6 +1359,7 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
     tf.x16 = static_cast<__half*>(a->x_op); tf.xscale = at<float>(a->x_op, p.xop_scale_off);
   }
   if (a->e_bias && !aligned16(a->e_bias)) return fail(MOE_ERR_ALIGNMENT, "e_bias not 16-byte aligned");
+  const int router_sms = p.rows ? router_ctas(*ds) : 0;
   if ((s = do_route(p, *ds, a->x, a->w_router, a->e_bias, a->topk_idx, a->topk_w, nullptr, ws, st,
                     sgate_with_router ? a->w_sgate : nullptr, p.L ? a->w_lat_down : nullptr,
                     a->x_lat, fused_dispatch ? &tf : nullptr)) != MOE_OK)
@@ -1341,7 +1370,7 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
     return fail(MOE_ERR_CUDA, "fork: %s", cudaGetErrorString(e));
   // (the row GEMV leaves a few SMs to the routing chain's small kernels)
   if ((s = do_shared_up(p, *ds, a->x, a->w_sgate, a->ws_gate, a->ws_up, ws, ds->side, sgate_with_router,
-                        ds->num_sms - kRowsFreeSMs)) != MOE_OK)
+                        ds->num_sms - (router_sms ? router_sms : kRowsFreeSMs))) != MOE_OK)
     return s;
   if ((e = cudaEventRecord(ds->ev_shared, ds->side)) != cudaSuccess)
     return fail(MOE_ERR_CUDA, "event: %s", cudaGetErrorString(e));

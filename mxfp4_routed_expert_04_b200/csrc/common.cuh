@@ -177,12 +177,18 @@ MOE_DEV void decode_block(uint32_t wg, uint32_t wg8, uint32_t (&a0)[4], uint32_t
   a1[0] = lo[2]; a1[1] = hi[2]; a1[2] = lo[3]; a1[3] = hi[3];
 }
 
-// power-of-two scale mapping a block maximum m into [2^14, 2^15) as f16
-MOE_DEV void f16_block_scale(float m, float& scale, float& inv) {
+// Operands of the CUDA-core GEMVs (the f16 token rows and h rows) have their
+// largest magnitude in [2^14, 2^15): their products are exact in the fp32
+// FMAs that sum them, and every bf16 value keeps all its bits down to 2^-29
+// of the maximum.
+constexpr int kF16OpTop = 15;
+
+// power-of-two scale mapping a block maximum m into [2^(top-1), 2^top) as f16
+MOE_DEV void f16_block_scale(float m, float& scale, float& inv, int top = 15) {
   if (!(m > 0.0f) || !isfinite(m)) { scale = 1.0f; inv = 1.0f; return; }
   const int ex = max(-100, min(127, frexp_exponent(m)));   // m = f * 2^ex, f in [0.5, 1)
-  scale = pow2_f32(ex - 15);
-  inv = pow2_f32(15 - ex);
+  scale = pow2_f32(ex - top);
+  inv = pow2_f32(top - ex);
 }
 
 // Sum of S split-K partials p[0], p[stride], ... in the order s = 0, 1, ...;

@@ -31,7 +31,7 @@
 // gate/up writes h = silu(g) * u in fp32 to h32; down reads h32 of the
 // expert's token and converts it to f16 with one power-of-two scale per
 // 32-element block (the block's largest |h| maps into [2^14, 2^15): relative
-// rounding <= 2^-11).
+// rounding <= 2^-11). The token rows come the same way, one scale per row.
 // Every wait is bounded: on a timeout the CTA raises an abort flag, the
 // status word gets kStatusWaitTimeout and every role stops (the results are
 // then undefined); copies in flight land before the CTA exits.
@@ -313,12 +313,8 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
                 m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
                                    fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
               }
-              float inv = 1.0f, sc = 1.0f;
-              if (m > 0.0f && isfinite(m)) {
-                const int ex = max(-100, min(127, frexp_exponent(m)));
-                sc = pow2_f32(ex - 15);
-                inv = pow2_f32(15 - ex);
-              }
+              float sc, inv;
+              f16_block_scale(m, sc, inv, kF16OpTop);
               sts32(hsc + 4u * b, __float_as_uint(sc));
 #pragma unroll
               for (int q = 0; q < 4; ++q) {          // 16 bytes of f16 from 32 bytes of fp32
@@ -509,7 +505,7 @@ MOE_DEV void convert_h_row(const float* hrow, int K, uint32_t hb, uint32_t hsc) 
 #pragma unroll
     for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
     float sc, inv;
-    f16_block_scale(m, sc, inv);
+    f16_block_scale(m, sc, inv, kF16OpTop);
     sts32(hsc + 4u * blk, __float_as_uint(sc));
 #pragma unroll
     for (int q = 0; q < 4; ++q) {

@@ -244,6 +244,35 @@ __global__ void __launch_bounds__(32 * (kRowsConsumers + 1), 1) k_rows_bf16(Rows
       r += n;
       while (seg < 2 && r == seg_units(seg)) { r = 0; ++seg; }
     }
+    if (!kSwiGLU && !kXF32 && a.x16 && blockIdx.x == 0) {
+      // the activation operand from the row in shared memory: every warp
+      // takes the largest |x| over the whole row (no barrier), then converts
+      // its sixteenth of the row
+      const uint32_t xs = smem_u32(act);
+      float m = 0.0f;
+      for (int i = lane; i < K / 8; i += 32) {
+        const uint4 v = lds16(xs + 16u * i);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(wv[j] & 0xFFFFu)), fabsf(bf16_to_f32(wv[j] >> 16))));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      float scale, inv;
+      f16_block_scale(m, scale, inv, kF16OpTop);
+      for (int i = w * 32 + lane; i < K / 8; i += 32 * kRowsConsumers) {
+        const uint4 v = lds16(xs + 16u * i);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(bf16_to_f32(wv[j] & 0xFFFFu) * inv, bf16_to_f32(wv[j] >> 16) * inv);
+          o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(a.x16 + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      if (w == 0 && lane == 0) *a.xscale = scale;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0 && *abort) atomicOr(a.status, kStatusWaitTimeout);

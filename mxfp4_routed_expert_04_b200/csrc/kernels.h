@@ -165,6 +165,11 @@ struct RowsArgs {
   const float* topk_w;       // [k]
   const float* gate_logit;   // [1]
   int k;
+  // optional, plain mode with bf16 x: CTA 0 also writes x as the f16
+  // activation operand of the single-token expert GEMVs (the row's largest
+  // |x| mapped into [2^14, 2^15) by a power-of-two scale, written to xscale)
+  __half* x16;               // [K] or NULL
+  float* xscale;             // [1]
 };
 template <bool kSwiGLU, bool kXF32> __global__ void k_rows_bf16(RowsArgs a);
 // K a power of two in 1024..8192: a stage holds `slots` row slots (plain:
@@ -236,7 +241,7 @@ struct TopkFuse {
   int32_t *counts, *offsets, *expert_list, *row_token, *row_slot, *slot_row;
   const uint16_t* x;         // [W] bf16
   int W;                     // a multiple of 8
-  __half* x16;               // [W]
+  __half* x16;               // [W], or NULL when the router launch writes the operand
   float* xscale;             // [1]
 };
 // How k_topk scores and selects (the default is the softmax router):

@@ -196,12 +196,8 @@ __global__ void __launch_bounds__(256) k_act_to_f16(const uint16_t* __restrict__
     for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16lo(wv[j])), fabsf(bf16hi(wv[j]))));
   }
   m = block_max_256(m);
-  float scale = 1.0f, inv = 1.0f;
-  if (m > 0.0f && isfinite(m)) {
-    const int ex = max(-100, min(127, frexp_exponent(m)));
-    scale = pow2_f32(ex - 15);
-    inv = pow2_f32(15 - ex);
-  }
+  float scale, inv;
+  f16_block_scale(m, scale, inv, kF16OpTop);
   for (int i = threadIdx.x * 8; i < W; i += 256 * 8) {
     const uint4 v = ldg16(row + i);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};

@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
   }
   __syncthreads();
   if (warp != 0) {
-    if (fuse) {
+    if (fuse && f.x16) {
       // the activation operand: the row's largest magnitude, then f16 with
       // the power-of-two scale that maps it into [2^14, 2^15)
       __shared__ float s_max[kTopkThreads / 32];
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kTopkThreads) k_topk(const float* __restrict__
       m = s_max[1];
       for (int w2 = 2; w2 < kTopkThreads / 32; ++w2) m = fmaxf(m, s_max[w2]);
       float scale, inv;
-      f16_block_scale(m, scale, inv);
+      f16_block_scale(m, scale, inv, kF16OpTop);
       for (int i = tid * 8; i < f.W; i += nthr * 8) {
         const uint4 xv = ldg16(f.x + i);
         const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
