@@ -113,7 +113,7 @@ def layer_flops(w):
     return f
 
 
-# sources of the single-token expert kernels whose DRAM counters profiles/traffic.json holds
+# sources of the single-token expert kernel whose DRAM counters profiles/traffic.json holds
 TRAFFIC_SOURCES = ("gemv_fma.cu", "common.cuh", "tc05.cuh")
 
 
@@ -400,7 +400,7 @@ def measure(args, w, steps, rank, local_rank, world, act=None):
         # for other widths, on the per-warp GEMV pair
         multi = ("k_mma_gateup" if w.W % 512 == 0 else "k_gateup_mxfp4",
                  "k_mma_down" if w.I % 512 == 0 else "k_down_mxfp4")
-        kernel = ("moe_expert_ffn (k_fma_gemv)" if w.T == 1
+        kernel = ("moe_expert_ffn (k_fma_routed1: gate/up and down in one launch)" if w.T == 1
                   else "moe_expert_ffn (k_fma_gemv + %s + %s)" % multi)
         roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": peak, "unit": "GB/s",
                 "frac": hbm_gbs / peak, "peak_kind": peak_kind}
