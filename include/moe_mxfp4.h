@@ -135,8 +135,11 @@ size_t moe_workspace_size(const moe_dims* dims);
  * moe_expert_ffn (x_op below). Returns 0 for invalid dims. */
 size_t moe_x_op_size(const moe_dims* dims);
 
-/* Clear the device status word in `ws` (enqueued on `stream`). Call once
- * after allocating a workspace. */
+/* Clear the device status word in `ws` and the counters the one-token
+ * routed launch hands work out with (enqueued on `stream`). Call once after
+ * allocating a workspace, before its first use: those counters must start at
+ * zero (every one-token call leaves them at zero again). Calls that share a
+ * workspace must not overlap in time. */
 moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, void* stream);
 
 /* Wait for `stream`, then copy the device status word into *host_status
@@ -242,7 +245,9 @@ moe_status moe_permute(const moe_dims* dims, const int32_t* topk_idx, const uint
  * its token t = row_token[r]:
  *   y_perm[r] = Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) )      [W] fp32
  * Weights in the canonical MXFP4 layout above, decoded exactly (E2M1 value x
- * E8M0 scale); products accumulate in fp32.
+ * E8M0 scale); products accumulate in fp32. One token (T = 1, MOE_ACT_BF16):
+ * both projections of its experts run in one launch whose CTAs take work
+ * from counters in `ws` (see moe_workspace_init).
  * MOE_ACT_MXFP4 (tcgen05 block-scaled MMAs): x and h = silu(Wg x) * (Wu x)
  * enter their products as MXFP4 (h quantised per 32-element block along I);
  * wg_s, wu_s and wd_s must then be in the TILED layout (moe_tile_scales of the
