@@ -2,10 +2,11 @@
 //
 // k_permute: per-expert histogram, exclusive scan and a stable placement of
 // the T*k (token, slot) pairs: rows grouped by expert, ascending token inside
-// an expert. One CTA of 1024 threads walks the pairs in chunks of 1024 in
-// (token, slot) order; inside a chunk a pair's rank among equal experts comes
-// from __match_any_sync within its warp plus a per-(warp, expert) exclusive
-// scan over the 32 warps, so the placement is deterministic.
+// an expert. One CTA of 1024 threads walks the pairs in chunks of 8192 in
+// (token, slot) order, each warp over 256 consecutive pairs in 8 rounds;
+// a pair's rank among equal experts comes from __match_any_sync within its
+// round, its warp's count from the earlier rounds, and a per-(warp, expert)
+// exclusive scan over the 32 warps, so the placement is deterministic.
 //
 // k_act_to_f16: bf16 activation rows -> f16 rows with one power-of-two scale
 // per row (the largest magnitude maps into [2^14, 2^15); bf16 values keep all
@@ -24,6 +25,7 @@ namespace moe {
 
 constexpr int kPermThreads = 1024;
 constexpr int kPermWarps = kPermThreads / 32;
+constexpr int kPermSub = 8;            // rounds of 32 pairs per warp and chunk
 
 // cursors [E], a flag word, and (more than one warp of pairs) the per-warp
 // counts [32][E]
@@ -132,15 +134,29 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
     }
     return;
   }
-  // chunk by chunk
-  for (int base = 0; base < R; base += kPermThreads) {
+  // chunk by chunk: warp w takes the kPermSub * 32 consecutive pairs
+  // base + w * kPermSub * 32 ..., kPermSub rounds of 32; a pair's rank among
+  // equal experts = the earlier rounds' count in its warp's row of whist plus
+  // its lower peers in the round; then one exclusive scan over the warps per
+  // expert turns the rows into bases (the histogram work is per chunk, so
+  // large chunks keep it small against the pairs)
+  for (int base = 0; base < R; base += kPermThreads * kPermSub) {
     for (int i = tid; i < kPermWarps * E; i += kPermThreads) whist[i] = 0;
     __syncthreads();
-    const int p = base + tid;
-    const int e = (p < R) ? idx[p] : -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && rank == 0) whist[warp * E + e] = __popc(peers);
+    const int wbase = base + warp * 32 * kPermSub;
+    int es[kPermSub], rk[kPermSub];
+#pragma unroll
+    for (int s = 0; s < kPermSub; ++s) {
+      const int p = wbase + 32 * s + lane;
+      const int e = (p < R) ? idx[p] : -1;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      const int prev = (e >= 0) ? whist[warp * E + e] : 0;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] = prev + __popc(peers);
+      __syncwarp();
+      es[s] = e;
+      rk[s] = prev + __popc(peers & ((1u << lane) - 1u));
+    }
     __syncthreads();
     for (int ee = tid; ee < E; ee += kPermThreads) {
       int run = cnt[ee];
@@ -152,12 +168,16 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(const int32_t* __restr
       cnt[ee] = run;
     }
     __syncthreads();
-    if (e >= 0) {
-      const int pos = whist[warp * E + e] + rank;
-      const int t = p / k;
-      row_token[pos] = t;
-      row_slot[pos] = p - t * k;
-      slot_row[p] = pos;
+#pragma unroll
+    for (int s = 0; s < kPermSub; ++s) {
+      if (es[s] >= 0) {
+        const int p = wbase + 32 * s + lane;
+        const int pos = whist[warp * E + es[s]] + rk[s];
+        const int t = p / k;
+        row_token[pos] = t;
+        row_slot[pos] = p - t * k;
+        slot_row[p] = pos;
+      }
     }
     __syncthreads();
   }
