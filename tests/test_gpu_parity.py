@@ -418,3 +418,47 @@ def test_one_token_launch_clears_its_counters():
             first = gpu["y_perm"]
     run.dev["x"].copy_(torch.from_numpy(run.dense["x"].view(np.int16)).cuda())
     np.testing.assert_array_equal(run.run_stages()["y_perm"], first)
+
+
+def test_one_token_thirty_two_experts():
+    """The one-launch routed path at its largest k (32 experts of one token)."""
+    w = _small(T=1, E=40, k=32)
+    run = DeviceRun(w)
+    gpu = run.run_stages()
+    ref = O.moe_layer(run.dense, w.k, expert_getter(w), idx_override=gpu["idx"])
+    assert int(gpu["expert_list"][0]) == 32
+    err, _ = max_rel_err(gpu["y_perm"][gpu["slot_row"][0]], ref["y_perm"][ref["slot_row"][0]])
+    assert err <= TOL, err
+    err, _ = max_rel_err(gpu["y"], ref["y"])
+    assert err <= TOL, err
+    assert M_status(run) == 0
+
+
+def M_status(run):
+    import mxfp4_routed_expert_04_b200 as M
+    return M.moe_device_status(run.layer.ws)
+
+
+def test_one_token_emptied_dispatch_then_a_normal_call():
+    """An invalid expert index empties the one-token dispatch; the one-launch
+    routed call on it streams nothing and leaves its counters at zero, and
+    the next call on a valid dispatch matches the oracle."""
+    import mxfp4_routed_expert_04_b200 as M
+    w = _small(T=1, E=8, k=2)
+    run = DeviceRun(w)
+    L = run.layer
+    bad = torch.tensor([[1, 8]], dtype=torch.int32, device="cuda")
+    M.moe_permute(run.dims, bad, run.dev["x"], L.counts, L.offsets, L.expert_list, L.row_token,
+                  L.row_slot, L.slot_row, L.x_op, L.ws)
+    assert int(L.expert_list[0]) == 0
+    lw = L.w
+    M.moe_expert_ffn(run.dims, L.x_op, L.offsets, L.expert_list, L.row_token, lw["wg_q"], lw["wg_s"],
+                     lw["wu_q"], lw["wu_s"], lw["wd_q"], lw["wd_s"], L.y_perm, L.ws)
+    torch.cuda.synchronize()
+    assert M.moe_device_status(L.ws) & M.STATUS_BAD_EXPERT
+    M.moe_workspace_init(run.dims, L.ws)
+    gpu = run.run_stages()
+    assert M.moe_device_status(L.ws) == 0
+    ref = O.moe_layer(run.dense, w.k, expert_getter(w), idx_override=gpu["idx"])
+    err, _ = max_rel_err(gpu["y"], ref["y"])
+    assert err <= TOL, err
