@@ -77,7 +77,7 @@ def mxfp4_dequant(q, s) -> np.ndarray:
     q: [..., N, K/2] uint8, two E2M1 codes per byte; element 2j of a row is the
        LOW nibble of byte j, element 2j+1 the HIGH nibble (reading: the pages do
        not state the nibble order; this is the order of the OCP reference
-       packing and of the rest of this build).
+       packing and of the C++ oracle and the CUDA kernels).
     s: [..., N, K/32] uint8 E8M0 codes, one per 32 consecutive elements of a row.
     """
     q = np.asarray(q, dtype=np.uint8)
