@@ -301,24 +301,38 @@ __global__ void __launch_bounds__(kThreads, 1) k_mxf4_gemm(const __grid_constant
         if (lane == 0) {
           const uint8_t* st = smem + s * S::kStageBytes;
           const int nkb = (kt == KT - 1) ? kb_last : 4;
-          for (int b = 0; b < nkb / 2; ++b) {
-            tc::cp_sf_block(sfa0 + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfa + b * 512)));
-            if (two)
-              tc::cp_sf_block(sfa1 + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfa + kSfBytes + b * 512)));
-            tc::cp_sf_block(sfb + 4 * b, tc::desc_sf(smem_u32(st + S::kOffSfb + b * 512)));
+          // descriptors of the stage's first blocks; a later block only moves
+          // the 14-bit address field (16-byte units: +2 per 32 bytes of a
+          // swizzled row, +32 per 512-byte scale block), which cannot carry:
+          // the stages are 1024-byte aligned below 228 KB
+          const uint64_t dsa0 = tc::desc_sf(smem_u32(st + S::kOffSfa));
+          const uint64_t dsa1 = tc::desc_sf(smem_u32(st + S::kOffSfa + kSfBytes));
+          const uint64_t dsb = tc::desc_sf(smem_u32(st + S::kOffSfb));
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            if (b < nkb / 2) {
+              tc::cp_sf_block(sfa0 + 4 * b, dsa0 + 32u * b);
+              if (two) tc::cp_sf_block(sfa1 + 4 * b, dsa1 + 32u * b);
+              tc::cp_sf_block(sfb + 4 * b, dsb + 32u * b);
+            }
           }
-          const uint32_t a0 = smem_u32(st), a1 = smem_u32(st + kATileBytes), bb = smem_u32(st + S::kOffB);
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint32_t id = (kb & 1) ? 2u : 0u;            // byte of the 32-bit scale column
-            const uint32_t col = 4u * (uint32_t)(kb >> 1);
-            const uint32_t idk = tc::idesc_sf_id(idesc, id);
-            const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-            const uint64_t bdesc = tc::desc_sw128(bb + 32 * kb);
-            tc::mma_mxf4(d0, tc::desc_sw128(a0 + 32 * kb), bdesc, idk, (sfa0 + col) | (id << 30),
-                         (sfb + col) | (id << 30), acc);
-            if (two)
-              tc::mma_mxf4(d1, tc::desc_sw128(a1 + 32 * kb), bdesc, idk, (sfa1 + col) | (id << 30),
-                           (sfb + col) | (id << 30), acc);
+          const uint64_t da0 = tc::desc_sw128(smem_u32(st)), da1 = tc::desc_sw128(smem_u32(st + kATileBytes));
+          const uint64_t db = tc::desc_sw128(smem_u32(st + S::kOffB));
+          const uint32_t idk0 = tc::idesc_sf_id(idesc, 0u), idk2 = tc::idesc_sf_id(idesc, 2u);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            if (kb < nkb) {
+              const uint32_t id = (kb & 1) ? 2u : 0u;          // byte of the 32-bit scale column
+              const uint32_t col = 4u * (uint32_t)(kb >> 1);
+              const uint32_t idk = (kb & 1) ? idk2 : idk0;
+              const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+              const uint64_t bdesc = db + 2u * kb;
+              tc::mma_mxf4(d0, da0 + 2u * kb, bdesc, idk, (sfa0 + col) | (id << 30), (sfb + col) | (id << 30),
+                           acc);
+              if (two)
+                tc::mma_mxf4(d1, da1 + 2u * kb, bdesc, idk, (sfa1 + col) | (id << 30),
+                             (sfb + col) | (id << 30), acc);
+            }
           }
           tc::commit(&empty[s]);
           if (kt == KT - 1) tc::commit(&acc_full[buf]);
