@@ -196,14 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_bf16_gemm(const __grid_constant
         tc::fence_after_sync();
         if (lane == 0) {
           const uint8_t* st = smem + s * stage_bytes;
-          const uint32_t a0 = smem_u32(st), a1 = smem_u32(st + kTileBytes);
-          const uint32_t bb = smem_u32(st + 2 * kTileBytes);
+          // descriptors of the stage's tiles, built once; a K block or the
+          // second B tile only moves the 14-bit address field (16-byte units),
+          // which cannot carry below 228 KB of shared memory
+          const uint64_t da0 = tc::desc_sw128(smem_u32(st)), da1 = tc::desc_sw128(smem_u32(st + kTileBytes));
+          const uint64_t db = tc::desc_sw128(smem_u32(st + 2 * kTileBytes));
+          const uint32_t bstep = (uint32_t)btile >> 4;
+#pragma unroll
           for (int kb = 0; kb < 4; ++kb) {                 // K = 16 per MMA: 32 bytes
             for (int p = 0; p < a.passes; ++p) {
               const uint32_t acc = (j > 0 || kb > 0 || p > 0) ? 1u : 0u;
-              const uint64_t bdesc = tc::desc_sw128(bb + p * btile + 32 * kb);
-              mma_bf16_tc(d0, tc::desc_sw128(a0 + 32 * kb), bdesc, idesc, acc);
-              if (w.two) mma_bf16_tc(d1, tc::desc_sw128(a1 + 32 * kb), bdesc, idesc, acc);
+              const uint64_t bdesc = db + p * bstep + 2u * kb;
+              mma_bf16_tc(d0, da0 + 2u * kb, bdesc, idesc, acc);
+              if (w.two) mma_bf16_tc(d1, da1 + 2u * kb, bdesc, idesc, acc);
             }
           }
           tc::commit(&empty[s]);
