@@ -752,7 +752,8 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
                          const int32_t* row_token, const uint8_t* wg_q, const uint8_t* wg_s,
                          const uint8_t* wu_q, const uint8_t* wu_s, const uint8_t* wd_q,
                          const uint8_t* wd_s, float* y_perm, void* ws, cudaStream_t st,
-                         cudaEvent_t join = nullptr) {
+                         cudaEvent_t join = nullptr, const void* l2_next = nullptr,
+                         size_t l2_next_bytes = 0) {
   if (p.mode == MOE_ACT_MXFP4)
     return do_expert_ffn_mxf4(p, ds, x_op, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, y_perm, ws, st, join);
   const long ny = p.E < p.R ? p.E : p.R;     // most experts that can be active
@@ -773,6 +774,8 @@ moe_status do_expert_ffn(const Plan& p, const DeviceState& ds, const void* x_op,
   f.offsets = offsets; f.expert_list = expert_list; f.row_token = row_token;
   f.wg_q = wg_q; f.wg_s = wg_s; f.wu_q = wu_q; f.wu_s = wu_s; f.wd_q = wd_q; f.wd_s = wd_s;
   f.y_perm = y_perm;
+  f.l2_next = l2_next && l2_next_bytes >= 16 && aligned16(l2_next) ? l2_next : nullptr;
+  f.l2_next_bytes = f.l2_next ? (uint64_t)(l2_next_bytes & ~(size_t)15) : 0;
   f.status = at<int32_t>(ws, p.off_status);
   f.sync = at<int32_t>(ws, p.off_status) + kSyncWord;
   f.W = p.W; f.I = p.I; f.E = p.E; f.R = p.R;
@@ -1384,8 +1387,12 @@ moe_status moe_layer(const moe_dims* dims, const moe_layer_args* a, void* ws, si
   // shared down projection, the first reader of its output (a joined launch
   // loses the early start of programmatic serialisation, a few microseconds,
   // wherever the join sits)
+  // (one token: as the routed launch's chunks run out, its CTAs prefetch the
+  // shared down weights, which the next launch reads, into L2)
+  const bool sd_next = combine_in_shared_down(p);
   if ((s = do_expert_ffn(p, *ds, a->x_op, a->offsets, a->expert_list, a->row_token, a->wg_q,
-                         a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st)) != MOE_OK)
+                         a->wg_s, a->wu_q, a->wu_s, a->wd_q, a->wd_s, a->y_perm, ws, st, nullptr,
+                         sd_next ? a->ws_down : nullptr, sd_next ? (size_t)p.H * p.Is * 2 : 0)) != MOE_OK)
     return s;
   if ((s = join_before(ds->ev_shared, st)) != MOE_OK) return s;
   if (combine_in_shared_down(p))

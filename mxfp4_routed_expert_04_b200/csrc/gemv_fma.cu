@@ -456,6 +456,9 @@ __global__ void __launch_bounds__(32 * (kFmaConsumers + 1), 1) k_fma_gemv(FmaArg
 // taken, so every h row a down chunk waits for is being produced by running
 // CTAs whatever the residency. Every wait is bounded (a timeout raises the
 // abort flag and kStatusWaitTimeout).
+// When a CTA finds no chunk left, it prefetches its share of the next
+// kernel's weights (FmaArgs::l2_next) into L2: the HBM is otherwise idle
+// while the last stages are computed.
 // Counters: sync[0] finished CTAs, sync[1 + s] h row pairs of expert slot s,
 // sync[kSyncGateUp] / sync[kSyncDown] the next chunk of each kind; the last
 // CTA to finish puts them all back to zero (the workspace clear zeroes them
@@ -478,6 +481,35 @@ MOE_DEV int ld_acquire_gpu(const int32_t* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+// Sums over the warp of R per-lane values (R = 1, 2, 4, 8) in reduce-scatter
+// form: log2 R halving steps (each lane keeps half of its values and adds the
+// partner's copy of that half: R - 1 shuffles in all), then a butterfly over
+// the remaining 32 / R lanes; returns the sum of value `row` = lane / (32 / R),
+// the same in all 32 / R lanes of the group.
+template <int R>
+MOE_DEV float warp_sum_rows(const float (&v)[R], int lane, int& row) {
+  constexpr int kSteps = R == 8 ? 3 : R == 4 ? 2 : R == 2 ? 1 : 0;
+  static_assert(R == (1 << kSteps), "R must be 1, 2, 4 or 8");
+  float c[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) c[i] = v[i];
+#pragma unroll
+  for (int s = 0; s < kSteps; ++s) {
+    const int n = R >> s, off = 16 >> s;
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float keep = up ? c[n / 2 + i] : c[i];
+      const float send = up ? c[i] : c[n / 2 + i];
+      c[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16 >> kSteps; off >= 1; off >>= 1) c[0] += __shfl_xor_sync(0xFFFFFFFFu, c[0], off);
+  row = lane >> (5 - kSteps);
+  return c[0];
 }
 
 // place 16 bytes read in rotated order qq into x[4 qq .. 4 qq + 3] without
@@ -636,6 +668,15 @@ __global__ void __launch_bounds__(32 * kRouted1Warps, 1)
         if (lane == 0) {
           s_job[slot] = make_int4(kJobDone, 0, 0, 0);
           tc::mbar_arrive(&S.full[slot]);
+          // no chunks left: this CTA's share of what the next kernel reads
+          // into L2, while the last stages of the launch are still computed
+          if (a.l2_next) {
+            const uint64_t per = ((a.l2_next_bytes + gridDim.x - 1) / gridDim.x + 15) & ~(uint64_t)15;
+            const uint64_t lo = per * blockIdx.x;
+            const uint64_t hi = min(lo + per, a.l2_next_bytes);
+            for (uint64_t o = lo; o < hi; o += 32768)
+              tc::prefetch_l2(static_cast<const uint8_t*>(a.l2_next) + o, (uint32_t)min((uint64_t)32768, hi - o));
+          }
         }
         break;
       }
@@ -855,13 +896,11 @@ __global__ void __launch_bounds__(32 * kRouted1Warps, 1)
               }
             }
           }
-#pragma unroll
-          for (int rr = 0; rr < RPSD; ++rr) {
-            if (u0 + rr < n) {
-              const float sum = warp_sum(acc[rr]);
-              if (lane == 0) a.y_perm[(size_t)r0 * a.W + r + u0 + rr] = sum;
-            }
-          }
+          // the RPSD row sums in one reduce-scatter; lane row * 32 / RPSD
+          // writes row `row`
+          int row;
+          const float sum = warp_sum_rows<RPSD>(acc, lane, row);
+          if ((lane & (32 / RPSD - 1)) == 0 && u0 + row < n) a.y_perm[(size_t)r0 * a.W + r + u0 + row] = sum;
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&S.hdone[slot]);   // this warp is done with the slot

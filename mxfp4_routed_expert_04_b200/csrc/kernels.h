@@ -90,6 +90,11 @@ struct FmaArgs {
   float* y_perm;             // down: [R, W]
   int32_t* status;           // device status word
   int32_t* sync;             // one-token launch: [0] finished CTAs, [1 + s] h row pairs of expert slot s
+  // one-token launch: bytes the next kernel of the stream reads (16-byte
+  // aligned, a multiple of 16), prefetched into L2 by each CTA as the chunks
+  // run out (its 1/gridDim share); NULL: none
+  const void* l2_next;
+  uint64_t l2_next_bytes;
   int W, I, E, R;
 };
 // Launch geometry: rps rows per consumer warp of a down stage, units per stage

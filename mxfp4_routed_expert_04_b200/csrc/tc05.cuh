@@ -125,6 +125,12 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64
         "r"(smem_u32(bar))
       : "memory");
 }
+// bulk prefetch of global memory into L2 (no completion to wait for):
+// address 16-byte aligned, bytes a multiple of 16
+MOE_DEV void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
 MOE_DEV void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
