@@ -357,8 +357,11 @@ def measure(args, w, steps, rank, local_rank, world, act=None):
         M.moe_expert_ffn(dims, layer.x_op, layer.offsets, layer.expert_list, layer.row_token, lw["wg_q"],
                          lw["wg_s"], lw["wu_q"], lw["wu_s"], lw["wd_q"], lw["wd_s"],
                          layer.y_perm, layer.ws, stream)
+    # (an NVTX range, so that a profiler can pick out these launches)
+    torch.cuda.nvtx.range_push("ffn_alone")
     timed(ffn, 3)
     ffn_ms = statistics.mean(timed(ffn, max(5, steps)))
+    torch.cuda.nvtx.range_pop()
 
     # end to end through moe_layer with host buffers
     x_host = x.cpu().pin_memory()

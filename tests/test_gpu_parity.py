@@ -397,7 +397,8 @@ def test_one_token_launch_clears_its_counters():
     w = ROWS_T1
     run = DeviceRun(w)
     L = run.layer
-    counters = slice(64, 64 + 4 * 33)
+    # every counter of the launch: 3 + k_max (32) words from word 16
+    counters = slice(64, 64 + 4 * 35)
     first = None
     for i in range(3):
         d = dict(run.dense)
