@@ -73,11 +73,6 @@ MOE_DEV float warp_sum(float v) {
   for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
   return v;
 }
-MOE_DEV float warp_max(float v) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-  return v;
-}
 
 }  // namespace
 

@@ -89,8 +89,6 @@ MOE_DEV float e8m0_byte(uint32_t w, bool plain) {
   if (plain) return __uint_as_float((i < 3 ? (w << (23 - 8 * i)) : (w >> 1)) & 0x7F800000u);
   return e8m0_to_f32((w >> (8 * i)) & 0xFFu);
 }
-// Value of E8M0 code c; `plain`: c is known to be neither 0 nor 255
-MOE_DEV float e8m0_value(uint32_t c, bool plain) { return plain ? __uint_as_float(c << 23) : e8m0_to_f32(c); }
 
 MOE_DEV void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
