@@ -22,7 +22,8 @@
 //   fma.rn.f32.f16 (exact f16 x f16 products, fp32 sums) and one fp32 FMA for
 //   the block scale (E8M0 decoded without a branch, codes 0 and 255 included);
 //   the rows of a warp are computed interleaved for independent FMA chains;
-//   a row's sum is a 5-step warp shuffle reduction.
+//   a row's sum is a 5-step warp shuffle reduction (the one-token launch's
+//   down warps sum their rows in one reduce-scatter, warp_sum_rows).
 //
 // One token (every expert single-token): k_fma_routed1 runs both projections
 // in one launch whose CTAs take chunks from device counters (below); more
