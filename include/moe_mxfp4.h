@@ -3,8 +3,9 @@
  * B200 (sm_100a).
  *
  * The layer (rabbit README, ferrumox/rabbit, model table row "MoE routing":
- * "softmax top-10 of 512 + gated shared expert", routed experts read as OCP
- * MXFP4; the "expert matmul" phase of its decode-step breakdown) computes, for
+ * softmax routing to 10 of 512 experts plus a gated shared expert, routed
+ * experts read as OCP MXFP4; the "expert matmul" phase of its decode-step
+ * breakdown) computes, for
  * every token t of x [T, H]:
  *
  *   logits = Wr x_t                         router, fp32 accumulate
@@ -84,9 +85,10 @@ typedef enum {
 } moe_act_mode;
 
 /* How the router scores experts (rabbit README, model table row "MoE
- * routing": "softmax top-10 of 512" for Qwen3.8-Max, "noaux_tc sigmoid" for
- * GLM-5.2, "grouped routing" for Kimi Linear; the pages name the last two
- * only, so their definitions here are readings). */
+ * routing": a softmax over 512 experts keeping the best 10 for Qwen3.8-Max,
+ * the router named noaux_tc sigmoid for GLM-5.2 and grouped routing for Kimi
+ * Linear; the pages name the last two only, so their definitions here are
+ * readings). */
 typedef enum {
   /* softmax: experts ranked by logit; w = the softmax renormalised over the
    * selected experts (times route_scale). */
@@ -155,7 +157,7 @@ moe_status moe_workspace_init(const moe_dims* dims, void* ws, size_t ws_bytes, v
 moe_status moe_device_status(const void* ws, int32_t* host_status, void* stream);
 
 /* --- a1-a2: router ---------------------------------------------------------
- * (rabbit README, model table row "MoE routing": softmax top-10 of 512; the
+ * (rabbit README, model table row "MoE routing": softmax routing to 10 of 512 experts; the
  * lowest-index tie-break and the renormalisation are readings of it.)
  * logits[t, e] = sum_h x[t, h] Wr[e, h] (bf16 products are exact, fp32
  * accumulation), p = softmax(logits[t]) in fp32, the k largest logits are
@@ -263,9 +265,10 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
                           float* y_perm, void* ws, size_t ws_bytes, void* stream);
 
 /* --- routed experts streamed from host memory --------------------------------
- * (rabbit README: the routed experts do not stay resident; they "stream on
- * demand through a per-layer LRU cache", and with "per-expert early drain" an
- * expert's matmul starts the moment its own bytes land.)
+ * (rabbit README: the routed experts do not stay resident but are fetched
+ * when a token needs them, through an LRU cache per layer, and its per-expert
+ * early drain starts an expert's matmul as soon as that expert's own bytes
+ * have arrived.)
  * A cache of `slots` expert slots in device memory (caller-owned, sized by
  * moe_expert_cache_bytes, 256-byte aligned) in front of experts kept in host
  * memory. MOE_ACT_BF16 layers only.
@@ -321,8 +324,8 @@ typedef struct {
 moe_status moe_mxf4_layout_of(const moe_dims* dims, moe_mxf4_layout* out);
 
 /* --- a8-a9 (+a10 up): shared expert and combine ------------------------------
- * (rabbit README, model table row "MoE routing": "+ gated shared expert"; the
- * per-token sigmoid gate is a reading.)
+ * (rabbit README, model table row "MoE routing": a gated shared expert runs
+ * beside the routed ones; the per-token sigmoid gate is a reading.)
  *   s_t = sigmoid(w_sgate . x_t) * Ws_down (silu(Ws_gate x_t) * (Ws_up x_t))
  *   y_t = [W_lu] (sum_j topk_w[t, j] * y_perm[slot_row[t, j]]) + s_t
  * W_lu is applied only for latent layers (w_lat_up non-NULL iff L > 0).

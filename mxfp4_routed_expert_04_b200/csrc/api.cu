@@ -1078,9 +1078,9 @@ moe_status moe_expert_ffn(const moe_dims* dims, const void* x_op, const int32_t*
 // ---------------------------------------------------------------------------
 // Routed experts streamed from host memory through an LRU cache of expert
 // slots in device memory (rabbit README: routed experts stay off the
-// accelerator and "stream on demand through a per-layer LRU cache"; its
-// feature list: per-expert early drain, an expert's matmul starts the moment
-// its own bytes land).
+// accelerator and are fetched when needed through an LRU cache per layer; its
+// feature list: per-expert early drain, an expert's matmul starts as soon as
+// its own bytes have arrived).
 // ---------------------------------------------------------------------------
 }  // extern "C"
 

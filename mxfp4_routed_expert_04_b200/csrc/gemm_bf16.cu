@@ -1,6 +1,6 @@
 // Dense bf16 GEMMs on tcgen05 (kind::f16, fp32 accumulation in tensor memory):
 // the router logits (rabbit README, model table row "MoE routing") and the
-// always-applied gated shared expert (rabbit README: "+ gated shared expert"),
+// always-applied gated shared expert (rabbit README, the same row),
 // for any number of tokens.
 //
 // Orientation as in the MXFP4 GEMM: the MMA's M side is 128 weight rows, its

@@ -4,7 +4,8 @@
 //
 // The contraction is the routed expert of the rabbit README ("expert matmul"
 // phase; model table row "MoE routing") with activations quantised to MXFP4
-// like the weights (Kimi K3 page: "MXFP4 routed experts", read byte for byte).
+// like the weights (Kimi K3 page: its routed experts are MXFP4, read byte for
+// byte).
 //
 // Orientation: the MMA's M side is 128 weight rows of one expert, its N side
 // one tile of at most kTileRows of that expert's permuted rows, K the

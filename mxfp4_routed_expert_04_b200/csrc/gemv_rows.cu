@@ -1,5 +1,5 @@
 // bf16 GEMV for a single token: the router logits and the sigmoid-gate logit
-// (rabbit README, model table row "MoE routing"; "+ gated shared expert"),
+// (rabbit README, model table row "MoE routing", with its gated shared expert),
 // the latent down-projection rows, and the shared expert's SwiGLU and down
 // projection.
 //

@@ -1,5 +1,5 @@
 // Router tail: softmax top-k with renormalised weights (rabbit README, model
-// table row "MoE routing": softmax top-10 of 512), and the two other routers
+// table row "MoE routing": a softmax router keeping 10 of 512 experts), and the two other routers
 // the same table names: "noaux_tc sigmoid" (GLM-5.2; read as sigmoid scores,
 // a per-expert bias that steers the selection only, weights renormalised over
 // the unbiased scores and scaled) and "grouped routing" (Kimi Linear; read as

@@ -295,7 +295,7 @@ void moe_o_router_logits(const uint16_t* x, const uint16_t* wr, int T, int H, in
 }
 
 // --- a2: top-k selection and weights ------------------------------------------------
-// score_fn 0 (softmax; rabbit README "softmax top-10 of 512"): the scores are
+// score_fn 0 (softmax; rabbit README, the softmax router keeping 10 of 512): the scores are
 // the logits themselves for selection (the softmax is monotone, so ranking by
 // logit ranks by probability), and w_j = exp(l_j - m) / sum_sel exp(l_i - m),
 // m the largest selected logit: the full softmax renormalised over the
@@ -455,7 +455,7 @@ int moe_o_expert_ffn(const double* x, int n, int W, int I, const uint8_t* wg_q,
 // --- a8: gated shared expert ----------------------------------------------------------
 // s[t] = sigmoid(x[t] . w_sg) * Wsd (silu(Wsg x[t]) * (Wsu x[t])), bf16 weights.
 // Reading: the gate is one sigmoid scalar per token from a weight vector w_sg
-// (the pages say only "gated shared expert"); the shared expert always runs.
+// (the pages only call it a gated shared expert); the shared expert always runs.
 void moe_o_shared_expert(const uint16_t* x, int T, int H, int Is, const uint16_t* ws_gate,
                          const uint16_t* ws_up, const uint16_t* ws_down, const uint16_t* w_sgate,
                          double* s, double* gate) {

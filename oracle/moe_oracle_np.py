@@ -18,9 +18,9 @@ or reordering beyond what each definition states.
 
 Sources. The pages describe the layer only by its shape:
 
-* rabbit README (ferrumox/rabbit), model table, row "MoE routing":
-  "softmax top-10 of 512 + gated shared expert"; row "native quantization
-  read": OCP MXFP4 routed experts, read byte for byte.
+* rabbit README (ferrumox/rabbit), model table, row "MoE routing": softmax
+  routing to 10 of 512 experts plus a gated shared expert; row "native
+  quantization read": OCP MXFP4 routed experts, read byte for byte.
 * rabbit README, phase breakdown: the "expert matmul" phase is the routed
   experts' matmuls, the part of a decode step this layer reproduces.
 * "Ran Moonshot's 2.8T-parameter Kimi K3 on a GPU-less mini-PC" (wpnews),
@@ -32,7 +32,7 @@ the E2M1/E8M0 encodings and 32-element blocks follow the OCP Microscaling
 Formats (MX) v1.0 specification, section 5 (MXFP4 = E2M1 elements, E8M0
 shared scale, block size 32); the SwiGLU expert, the sigmoid shared-expert
 gate, top-k renormalisation and the lowest-index tie-break are the plainest
-readings of "softmax top-k + gated shared expert".
+readings of a softmax top-k router with a gated shared expert.
 
 Pinned by tests/test_oracle_pins.py (values from the OCP definition, closed
 forms, brute force on tiny inputs, a dense-FFN special case computed by torch,
@@ -295,7 +295,7 @@ def expert_ffn(x_rows, wg, wu, wd, act: str = "exact"):
 
 
 # ---------------------------------------------------------------------------
-# a8: gated shared expert (rabbit README: "+ gated shared expert")
+# a8: gated shared expert (rabbit README, model table row "MoE routing")
 # ---------------------------------------------------------------------------
 
 def shared_expert(x_bits, ws_gate_bits, ws_up_bits, ws_down_bits, w_sgate_bits):
