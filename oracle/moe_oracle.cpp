@@ -24,7 +24,7 @@
 //
 // Sources (the pages describe the layer by its shape only):
 // * rabbit README (ferrumox/rabbit), model table, row "MoE routing": softmax
-//   top-10 of 512 plus a gated shared expert (Qwen3.8-Max); "Stable LatentMoE"
+//   routing to 10 of 512 experts plus a gated shared expert (Qwen3.8-Max); "Stable LatentMoE"
 //   (Kimi K3), "grouped routing" (Kimi Linear), "noaux_tc sigmoid" (GLM-5.2).
 //   Row "native quantization read": routed experts in OCP MXFP4.
 // * rabbit README, phase breakdown: the "expert matmul" phase is this layer's

@@ -321,8 +321,8 @@ def combine(y_perm, slot_row, w, shared_out=None, w_lat_up_bits=None):
     """y[t] = sum_j w[t, j] * y_perm[slot_row[t, j]]  (+ latent up-projection) + s[t].
 
     With a latent up-projection W_lu [H, L] the weighted sum is formed at width
-    L and mapped once: y[t] = W_lu (sum_j w y_perm) + s[t] (reading of
-    "routed experts compute in a narrower latent width")."""
+    L and mapped once: y[t] = W_lu (sum_j w y_perm) + s[t] (reading of the
+    Kimi K3 page's latent-width routed experts)."""
     y_perm = np.asarray(y_perm, dtype=np.float64)
     T, k = slot_row.shape
     acc = np.zeros((T, y_perm.shape[1]), dtype=np.float64)
